@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""SSM-layer decode throughput of the replay scheme on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the small-model-like decode layer (batch 256, 64 heads, head_dim
+64, d_state 128, 8 groups, fp32 checkpoint 2 MiB per request, bf16 x/B/C,
+interval 16), synthetic inputs from hybrid_model_ssm_replay_b200.inputs.
+One step = one interval of the replay scheme (ReplaySSM article s1): 16
+rssm_decode_step calls plus one rssm_flush, so every step moves the same
+bytes and the checkpoint-update cost is inside the number (s2). The value is
+whole-job tokens/s (requests x tokens, all ranks) over K timed steps; the
+state read per token (512 MiB) is larger than L2, so no flush of L2 is
+needed between steps. Under torchrun each rank runs its own replica of the
+layer (requests are independent: weak scaling, no collective on the data
+path); the barrier and the max-over-ranks time use torch.distributed.
+
+Also reported in the same JSON line: the conventional per-token
+read+write kernel on the same layer (the in-run comparison), the
+large-model-like layer (batch 512, 128 heads), the decode kernel's HBM
+roofline, an end-to-end number with host buffers, and the fp64 CPU oracle's
+throughput on a bounded sample (cpu_baseline).
+
+--impl reference times the fp64 CPU oracle (the checker; there is no
+installable reference implementation of this method) on the same workload
+and metric, on rank 0 only.
+"""
+import argparse
+import glob
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSM decode tokens/s at batch 256/512; achieved HBM GB/s vs B200 peak"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--fused", action="store_true", help="fold the buffer inside the 16th decode (no flush call)")
+    p.add_argument("--no-extra", action="store_true", help="skip the comparison / large-layer / e2e legs")
+    return p.parse_args()
+
+
+# --------------------------------------------------------------- helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
+
+
+def kernel_source_hash():
+    h = hashlib.sha1()
+    for name in ("rssm_kernels.cu", "rssm_device.cuh"):
+        with open(os.path.join(ROOT, "hybrid_model_ssm_replay_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def ncu_traffic(kernel_tag):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    sha = kernel_source_hash()
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        for line in open(path):
+            m = re.search(r"bench-traffic:\s*kernel=(\S+)\s+sha=(\w+)\s+bytes_per_launch=(\d+)", line)
+            if m and m.group(1) == kernel_tag and m.group(2) == sha:
+                return int(m.group(3))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.sw_power_cap,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 6:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0, t1):
+        sel = [p for (t, p) in self.samples if t0 - 0.05 <= t <= t1 + 0.05]
+        if not sel:
+            sel = [p for (_, p) in self.samples]
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[0]) for p in sel if num(p[0]) is not None]
+        mx = [num(p[1]) for p in sel if num(p[1]) is not None]
+        names = ["sw_power_cap", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+        reasons = sorted({names[i] for p in sel for i in range(4) if p[2 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(sel)}
+
+
+def smi_gpu_id(torch, dev):
+    try:
+        pr = torch.cuda.get_device_properties(dev)
+        return "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            return vis.split(",")[dev]
+        return dev
+
+
+# ------------------------------------------------------ analytic bytes
+
+def shape_bytes(shape, in_bytes=2):
+    H, P, N, G = shape.nheads, shape.head_dim, shape.d_state, shape.ngroups
+    return dict(state=4 * H * P * N, entry=H * P * in_bytes + G * N * in_bytes + 4 * H,
+                inputs=H * P * in_bytes + 2 * G * N * in_bytes + 4 * H, y=4 * H * P)
+
+
+def decode_bytes_per_request(shape, pos):
+    """Algorithmic HBM bytes of one replay-decode token of one request at
+    buffer position pos: checkpoint read, pos buffered entries read, the
+    new entry written, the token's inputs read, y written."""
+    b = shape_bytes(shape)
+    return b["state"] + pos * b["entry"] + b["entry"] + b["inputs"] + b["y"]
+
+
+def flush_bytes_per_request(shape, T):
+    b = shape_bytes(shape)
+    return 2 * b["state"] + T * b["entry"]
+
+
+def conv_bytes_per_request(shape):
+    b = shape_bytes(shape)
+    return 2 * b["state"] + b["inputs"] + b["y"]
+
+
+# --------------------------------------------------------- our arm (GPU)
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from hybrid_model_ssm_replay_b200 import rssm
+    from hybrid_model_ssm_replay_b200.inputs import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    rssm.lib()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    K, W = args.steps, args.warmup
+    wl = WORKLOADS["small_b256"]
+    shape = wl["shape"]
+    L = shape.interval
+    WIN = 2 * L  # distinct tokens of inputs, cycled
+    inp = make_inputs(shape, WIN, wl["seed"] + rank, wl["in_dtype"], device=dev)
+    flags = rssm.RSSM_FLAG_FUSED_FLUSH if args.fused else 0
+    desc = rssm.make_desc(shape.batch, shape.nheads, shape.head_dim, shape.d_state, shape.ngroups,
+                          interval=L, flags=flags)
+    st = rssm.RssmState(desc, dev)
+    st.ckpt.copy_(inp["ckpt"])
+    y = torch.empty((L, shape.batch, shape.nheads, shape.head_dim), device=dev)
+    stream = torch.cuda.current_stream()
+    n_dec = K * L
+    ev_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_dec)]
+    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+
+    def step(k, timed):
+        base = (k % (WIN // L)) * L
+        for i in range(L):
+            t = base + i
+            if timed:
+                ev_d[k * L + i][0].record(stream)
+            rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"],
+                                  y[i])
+            if timed:
+                ev_d[k * L + i][1].record(stream)
+        if not args.fused:
+            if timed:
+                ev_f[k][0].record(stream)
+            rssm.rssm_flush(st, inp["A"])
+            if timed:
+                ev_f[k][1].record(stream)
+
+    sampler = ClockSampler(smi_gpu_id(torch, local))
+    sampler.start()
+    for k in range(W):
+        step(k, False)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    start.record(stream)
+    for k in range(K):
+        step(k, True)
+    end.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier()
+    torch.cuda.synchronize()
+    ms_local = start.elapsed_time(end)
+    ms = max_over_ranks(ms_local)
+    if rssm.rssm_get_error(st) != 0:
+        raise RuntimeError("device error during the timed run")
+    time.sleep(0.06)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    tokens = world * shape.batch * L * K
+    value = tokens / (ms / 1e3)
+    dec_ms = [a.elapsed_time(b) for a, b in ev_d]
+    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+    dec_bytes = sum(decode_bytes_per_request(shape, i) for i in range(L)) / L * shape.batch
+    peak, peak_src = measured_peaks()
+    achieved = dec_bytes / (dec_avg_ms / 1e3) / 1e9
+    traffic = ncu_traffic("replay_decode_small_b256")
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "small_b256: replay decode, batch 256, 64 heads, head_dim 64, d_state 128, "
+                               "8 groups, fp32 checkpoint, bf16 x/B/C, interval 16",
+                   "batch_per_gpu": shape.batch, "tokens_per_step": shape.batch * L * world,
+                   "step": "16 x rssm_decode_step + " + ("fused fold" if args.fused else "1 x rssm_flush"),
+                   "l2": "no flush: the 512 MiB fp32 state read each token exceeds the 126 MB L2",
+                   "parallelism": f"replicas x{world} (independent requests)"},
+        "roofline": {"kernel": "k_replay (rssm_decode_step)", "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "algorithmic_bytes_per_launch": dec_bytes,
+                     "avg_launch_us": dec_avg_ms * 1e3},
+        "gpu_launches": K * (L + (0 if args.fused else 1)),
+        "clocks": clocks,
+    }
+    if not args.fused:
+        fl_ms = [a.elapsed_time(b) for a, b in ev_f]
+        fl_avg = sum(fl_ms) / len(fl_ms)
+        fl_bytes = flush_bytes_per_request(shape, L) * shape.batch
+        out["flush_kernel"] = {"avg_launch_us": fl_avg * 1e3, "achieved_gbs": fl_bytes / (fl_avg / 1e3) / 1e9,
+                               "frac": fl_bytes / (fl_avg / 1e3) / 1e9 / peak}
+    if not args.no_extra:
+        out["conventional"] = conv_leg(rssm, torch, shape, inp, K, W, dev, barrier, max_over_ranks, world, peak)
+        out["speedup_vs_conventional"] = value / out["conventional"]["value"]
+        out["e2e"] = e2e_leg(rssm, torch, st, shape, inp, max(2, min(K, 20)), W, dev, barrier, max_over_ranks,
+                             world, args.fused)
+        del st, inp, y
+        torch.cuda.empty_cache()
+        out["large_b512"] = large_leg(rssm, torch, WORKLOADS["large_b512"], max(2, min(K, 50)), W, dev, barrier,
+                                      max_over_ranks, world, peak, args.fused)
+    if rank == 0 and world == 1:
+        out["cpu_baseline"] = cpu_baseline()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+
+
+def conv_leg(rssm, torch, shape, inp, K, W, dev, barrier, max_over_ranks, world, peak):
+    desc = rssm.make_desc(shape.batch, shape.nheads, shape.head_dim, shape.d_state, shape.ngroups)
+    h = inp["ckpt"].clone()
+    L = shape.interval
+    y = torch.empty((shape.batch, shape.nheads, shape.head_dim), device=dev)
+    n_win = inp["x"].shape[0]
+
+    def step(k):
+        for i in range(L):
+            t = (k * L + i) % n_win
+            rssm.rssm_conv_step(desc, h, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"], y)
+
+    for k in range(W):
+        step(k)
+    torch.cuda.synchronize()
+    barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for k in range(K):
+        step(k)
+    e.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(s.elapsed_time(e))
+    per_launch = ms / (K * L)
+    gbs = conv_bytes_per_request(shape) * shape.batch / (per_launch / 1e3) / 1e9
+    return {"kernel": "k_conv (rssm_conv_step)", "value": world * shape.batch * L * K / (ms / 1e3), "unit": UNIT,
+            "avg_launch_us": per_launch * 1e3, "achieved_gbs": gbs, "frac": gbs / peak}
+
+
+def e2e_leg(rssm, torch, st, shape, inp, K, W, dev, barrier, max_over_ranks, world, fused):
+    """Same metric through the public API with host buffers: every step
+    copies its 16 tokens of inputs from pinned host memory and reads the 16
+    outputs back, inside the timed region."""
+    L = shape.interval
+    hx = inp["x"][:L].cpu().pin_memory()
+    hB = inp["B"][:L].cpu().pin_memory()
+    hC = inp["C"][:L].cpu().pin_memory()
+    hdt = inp["dt"][:L].cpu().pin_memory()
+    dx, dB, dC, ddt = (torch.empty_like(inp[k][:L]) for k in ("x", "B", "C", "dt"))
+    y = torch.empty((L, shape.batch, shape.nheads, shape.head_dim), device=dev)
+    hy = torch.empty(y.shape, dtype=torch.float32).pin_memory()
+    st.pos.zero_()
+
+    def step():
+        dx.copy_(hx, non_blocking=True)
+        dB.copy_(hB, non_blocking=True)
+        dC.copy_(hC, non_blocking=True)
+        ddt.copy_(hdt, non_blocking=True)
+        for i in range(L):
+            rssm.rssm_decode_step(st, dx[i], dB[i], dC[i], ddt[i], inp["A"], inp["D"], y[i])
+        if not fused:
+            rssm.rssm_flush(st, inp["A"])
+        hy.copy_(y, non_blocking=True)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(K):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(s.elapsed_time(e))
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hB, hC, hdt))
+    return {"value": world * shape.batch * L * K / (ms / 1e3), "unit": UNIT, "steps": K,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hy.numel() * 4,
+            "path": "pinned host -> cudaMemcpyAsync -> rssm_decode_step x16 + rssm_flush -> host"}
+
+
+def large_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak, fused):
+    from hybrid_model_ssm_replay_b200.inputs import make_inputs
+    shape = wl["shape"]
+    L = shape.interval
+    inp = make_inputs(shape, L, wl["seed"], wl["in_dtype"], device=dev)
+    desc = rssm.make_desc(shape.batch, shape.nheads, shape.head_dim, shape.d_state, shape.ngroups, interval=L,
+                          flags=rssm.RSSM_FLAG_FUSED_FLUSH if fused else 0)
+    st = rssm.RssmState(desc, dev)
+    st.ckpt.copy_(inp["ckpt"])
+    y = torch.empty((shape.batch, shape.nheads, shape.head_dim), device=dev)
+
+    def rstep():
+        for i in range(L):
+            rssm.rssm_decode_step(st, inp["x"][i], inp["B"][i], inp["C"][i], inp["dt"][i], inp["A"], inp["D"], y)
+        if not fused:
+            rssm.rssm_flush(st, inp["A"])
+
+    def cstep(h):
+        for i in range(L):
+            rssm.rssm_conv_step(desc, h, inp["x"][i], inp["B"][i], inp["C"][i], inp["dt"][i], inp["A"], inp["D"], y)
+
+    def timed(fn, *a):
+        for _ in range(W):
+            fn(*a)
+        torch.cuda.synchronize()
+        barrier()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(K):
+            fn(*a)
+        e.record()
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(s.elapsed_time(e))
+
+    ms_r = timed(rstep)
+    del st
+    h = inp["ckpt"].clone()
+    ms_c = timed(cstep, h)
+    tok = world * shape.batch * L * K
+    rep_bytes = (sum(decode_bytes_per_request(shape, i) for i in range(L)) +
+                 (0 if fused else flush_bytes_per_request(shape, L))) * shape.batch
+    return {"workload": "large_b512: batch 512, 128 heads, 64 x 128, 8 groups, interval 16", "steps": K,
+            "replay_tokens_per_s": tok / (ms_r / 1e3), "conventional_tokens_per_s": tok / (ms_c / 1e3),
+            "speedup": ms_c / ms_r, "replay_step_gbs": rep_bytes / (ms_r / K / 1e3) / 1e9,
+            "replay_step_frac": rep_bytes / (ms_r / K / 1e3) / 1e9 / peak,
+            "conventional_gbs": conv_bytes_per_request(shape) * shape.batch * L / (ms_c / K / 1e3) / 1e9}
+
+
+# ---------------------------------------------------- the CPU oracle arm
+
+def oracle_interval_sample(n_requests, seed=5):
+    """Inputs of n_requests requests of the small layer, one interval, in
+    fp64 numpy (same recipe as the GPU run, drawn on the CPU)."""
+    import torch
+    from hybrid_model_ssm_replay_b200.inputs import WORKLOADS, LayerShape, make_inputs
+    s = WORKLOADS["small_b256"]["shape"]
+    shape = LayerShape(n_requests, s.nheads, s.head_dim, s.d_state, s.ngroups, s.interval)
+    inp = make_inputs(shape, s.interval, seed, torch.bfloat16, device="cpu")
+    return {k: v.double().numpy() for k, v in inp.items()}, shape
+
+
+def oracle_interval(orc, f, b, L):
+    req = orc.ReplayRequest(f["ckpt"][b], f["B"].shape[2], L, f["A"], f["D"])
+    for t in range(L):
+        req.decode(f["x"][t, b], f["B"][t, b], f["C"][t, b], f["dt"][t, b])
+    req.flush()
+    return L
+
+
+def cpu_baseline(target_s=10.0):
+    from oracle import oracle as orc
+    f, shape = oracle_interval_sample(8)
+    L = shape.interval
+    oracle_interval(orc, f, 0, L)  # warm (loads the library)
+    tok, t0 = 0, time.perf_counter()
+    b = 0
+    while time.perf_counter() - t0 < target_s:
+        tok += oracle_interval(orc, f, b % shape.batch, L)
+        b += 1
+    dt = time.perf_counter() - t0
+    return {"value": tok / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{b} request-intervals of the small_b256 layer (16 replay decodes + 1 flush each, "
+                      f"fp64, single thread), {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import oracle as orc
+    f, shape = oracle_interval_sample(8)
+    L = shape.interval
+    oracle_interval(orc, f, 0, L)
+    for k in range(args.warmup):
+        oracle_interval(orc, f, k % shape.batch, L)
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        oracle_interval(orc, f, k % shape.batch, L)
+    dt = time.perf_counter() - t0
+    value = args.steps * L / dt
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "small_b256: replay decode, batch 256, 64 heads, head_dim 64, d_state 128, "
+                               "8 groups, interval 16",
+                   "step": "one request-interval (16 replay decodes + 1 flush) of the fp64 CPU oracle"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} request-intervals, single thread"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,238 @@
+// rssm_device.cuh -- device-side building blocks of librssm (sm_100a).
+//
+//  * shared-memory bulk copies (cp.async.bulk, completion on an mbarrier)
+//    and waits bounded by %globaltimer, so no kernel can spin forever;
+//  * Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers:
+//    As Easy as 1, 2, 3", SC'11);
+//  * the number formats of the precision split (ReplaySSM article,
+//    devotd.net "nvidia-replayssm-hybrid-model-ssm-decoding-state-buffer",
+//    s4 "Prevent low-precision errors from accumulating again"):
+//    stochastic rounding to bf16 / e4m3 in integer arithmetic on the fp32
+//    bits, nearest rounding to e4m3 (scales) and e2m1 (FP4 codes) with the
+//    hardware cvt instructions, and their decoders.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace rssm {
+
+constexpr int kThreads = 256;               // threads per CTA of every tile kernel
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxCap = 32;                 // buffer slots per request (interval + drafts)
+constexpr int kMaxTok = 8;                  // tokens per verify call (K + 1)
+constexpr unsigned long long kWaitNs = 2000000000ull;  // bound of one bulk-copy wait
+
+// ------------------------------------------------------------------ errors
+
+__device__ __forceinline__ void set_error(int32_t* err, int32_t code) {
+    if (err) atomicCAS(err, 0, code);
+}
+
+// ------------------------------------------------ mbarrier + bulk copies
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+// Global -> shared bulk copy; bytes and both addresses multiples of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Waits for phase `parity` of the barrier, at most limit_ns. True on completion.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+
+// ------------------------------------------------------------- loads
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Four consecutive input elements as float4 (16-byte / 8-byte vector loads).
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+    uint2 u = *reinterpret_cast<const uint2*>(p);
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+}
+
+__device__ __forceinline__ float dot4(float4 a, float4 b) {
+    return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
+}
+
+// Sum over aligned groups of `width` lanes (width a power of two <= 32).
+__device__ __forceinline__ float group_sum(float v, int width) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+        if (off < width) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+// ------------------------------------------------------------------ Philox
+
+// Philox4x32-10: ten rounds; round i uses key + i * (0x9E3779B9, 0xBB67AE85).
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
+#pragma unroll
+    for (int i = 0; i < 10; ++i) {
+        if (i) {
+            k.x += 0x9E3779B9u;
+            k.y += 0xBB67AE85u;
+        }
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+        c = make_uint4(hi1 ^ c.y ^ k.x, lo1, hi0 ^ c.w ^ k.y, lo0);
+    }
+    return c;
+}
+
+// ------------------------------------------------------ stochastic rounding
+// |v| = q (m + f) with q the target spacing at |v|; the magnitude rounds up
+// iff r < floor(f * 2^32). Worked on the fp32 bit pattern.
+
+// bf16 keeps the top 16 bits of fp32, so f * 2^16 is the low 16 bits.
+__device__ __forceinline__ uint32_t sr_bf16(float v, uint32_t r) {
+    const uint32_t u = __float_as_uint(v);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (u >> 16) | 0x40u;  // NaN stays NaN
+    return (u >> 16) + ((r >> 16) < (u & 0xFFFFu) ? 1u : 0u);
+}
+
+// OCP e4m3 ("fn"): bias 7, spacing 2^(E-3) for |v| >= 2^-6, 2^-9 below;
+// |v| >= 448 (and inf) saturates to 448, NaN -> 0x7F.
+__device__ __forceinline__ uint32_t sr_e4m3(float v, uint32_t r) {
+    const uint32_t u = __float_as_uint(v);
+    const uint32_t sign = (u >> 24) & 0x80u;
+    const uint32_t a = u & 0x7FFFFFFFu;
+    if (a > 0x7F800000u) return 0x7Fu;
+    if (a >= 0x43E00000u) return sign | 0x7Eu;
+    const int E = static_cast<int>(a >> 23) - 127;
+    uint32_t code, F;
+    if (E >= -6) {
+        code = (static_cast<uint32_t>(E + 7) << 3) | ((a >> 20) & 7u);
+        F = (a & 0xFFFFFu) << 12;
+    } else {
+        // below 2^-6: count steps of 2^-9 in the 24-bit significand M * 2^(E-23)
+        const uint32_t M = (E == -127) ? (a & 0x7FFFFFu) : ((a & 0x7FFFFFu) | 0x800000u);
+        const int sh = 14 - ((E == -127) ? -126 : E);   // >= 21
+        if (sh >= 56) {
+            code = 0u;
+            F = 0u;
+        } else {
+            code = (sh >= 32) ? 0u : (M >> sh);
+            const uint64_t frac = static_cast<uint64_t>(M) & ((1ull << sh) - 1ull);
+            F = (sh <= 32) ? static_cast<uint32_t>(frac << (32 - sh)) : static_cast<uint32_t>(frac >> (sh - 32));
+        }
+    }
+    return sign | (code + (r < F ? 1u : 0u));
+}
+
+// --------------------------------------------------------- nearest rounding
+
+// e4m3, round to nearest even, saturating (hardware conversion).
+__device__ __forceinline__ uint32_t e4m3_rn(float v) {
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(v));
+    return out & 0xFFu;
+}
+
+// Two e2m1 codes (nearest even, saturating to +-6): lo in bits 0..3, hi in 4..7.
+__device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+        "mov.b32 %0, {t, t, t, t};\n\t}"
+        : "=r"(out)
+        : "f"(hi), "f"(lo));
+    return out & 0xFFu;
+}
+
+__device__ __forceinline__ float e4m3_val(uint32_t c) {
+    const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+    const float mag = (e == 0u) ? static_cast<float>(m) * 0x1p-9f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+    return (c & 0x80u) ? -mag : mag;
+}
+
+__device__ __forceinline__ float bf16_val(uint32_t bits) { return __uint_as_float(bits << 16); }
+
+// Four e2m1 codes (16 bits, element 0 in the low nibble) to floats.
+__device__ __forceinline__ float4 fp4x4_val(uint32_t codes16) {
+    uint32_t h01, h23;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t}"
+        : "=r"(h01), "=r"(h23)
+        : "r"(codes16));
+    const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+    const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+    return make_float4(f01.x, f01.y, f23.x, f23.y);
+}
+
+// Four e4m3 codes (32 bits, element 0 in the low byte) to floats.
+__device__ __forceinline__ float4 e4m3x4_val(uint32_t w) {
+    return make_float4(e4m3_val(w & 0xFFu), e4m3_val((w >> 8) & 0xFFu), e4m3_val((w >> 16) & 0xFFu),
+                       e4m3_val(w >> 24));
+}
+
+// Four bf16 (two 32-bit words, element 0 in the low half) to floats.
+__device__ __forceinline__ float4 bf16x4_val(uint2 w) {
+    return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u),
+                       __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u));
+}
+
+// FP4 copy of 16 contiguous values held as one float4 by each of 4
+// consecutive lanes: scale = e4m3_rn(amax / 6), codes = e2m1_rn(v / scale),
+// all codes 0 when the scale is 0. All 32 lanes must call it. Returns this
+// lane's 16 code bits and sets *scale_code.
+__device__ __forceinline__ uint32_t fp4_quant_quad(float4 v, uint32_t* scale_code) {
+    float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    const uint32_t sc = e4m3_rn(__fdiv_rn(amax, 6.0f));
+    *scale_code = sc;
+    const float s = e4m3_val(sc);
+    if (s == 0.0f) return 0u;
+    const uint32_t c01 = e2m1x2_rn(__fdiv_rn(v.x, s), __fdiv_rn(v.y, s));
+    const uint32_t c23 = e2m1x2_rn(__fdiv_rn(v.z, s), __fdiv_rn(v.w, s));
+    return c01 | (c23 << 8);
+}
+
+}  // namespace rssm

@@ -1,0 +1,93 @@
+// rssm_internal.h -- argument blocks and launchers shared by the C ABI
+// (rssm_api.cu) and the kernels (rssm_kernels.cu). Not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rssm {
+
+enum Fmt : int { kF32 = 0, kBF16 = 1, kE4M3 = 2, kFP4 = 3 };
+
+// Shapes shared by every kernel. lpr = d_state / 4 lanes per state row.
+struct Shape {
+    int batch, H, P, N, G, L, cap, lpr;
+};
+
+// Replay decode / verify (ReplaySSM article s1, s3).
+struct ReplayArgs {
+    Shape s;
+    int ntok;        // tokens per request in this call: 1 (decode) or K+1 (verify)
+    int advance;     // decode: pos += 1 by the last CTA of the request
+    int fused;       // decode: fold the buffer when this token fills it (fp32 state)
+    const void* tile;            // read copy: fp32 / bf16 / e4m3 values or FP4 codes
+    const uint8_t* tile_scales;  // FP4 scales of the read copy
+    float* ckpt_w;               // fused flush: fp32 checkpoint written back
+    void* xbuf;
+    void* bbuf;
+    float* dtbuf;
+    int32_t* pos;
+    uint32_t* flush_count;
+    uint32_t* arrive;
+    int32_t* err;
+    const void* x;
+    const void* B;
+    const void* C;
+    const float* dt;
+    const float* A;
+    const float* D;
+    float* y;
+};
+
+// Fold of the buffer into the update copy (flush / refresh; s1, s4).
+struct FoldArgs {
+    Shape s;
+    int mode;          // 0: pos >= L only; 1: also any pos > 0; 2: every request
+    int out_fp4;       // also write the FP4 output copy
+    uint64_t seed;
+    void* upd;         // update copy (fp32 / bf16 / e4m3 values or FP4 codes)
+    uint8_t* upd_scales;
+    uint8_t* out_codes;
+    uint8_t* out_scales;
+    const void* xbuf;
+    const void* bbuf;
+    const float* dtbuf;
+    int32_t* pos;
+    uint32_t* flush_count;
+    uint32_t* arrive;
+    int32_t* err;
+    const float* A;
+};
+
+// Conventional step / verify (s1, s3: the scheme ReplaySSM replaces).
+struct ConvArgs {
+    Shape s;
+    int ntok;
+    float* h;              // step: state; verify: copies [ntok][batch][H][P][N]
+    const int32_t* cur;    // verify: copy holding the current state
+    int32_t* err;
+    const void* x;
+    const void* B;
+    const void* C;
+    const float* dt;
+    const float* A;
+    const float* D;
+    float* y;
+};
+
+// Launchers return cudaSuccess or the launch error. in_bf16 selects the
+// input element type.
+cudaError_t launch_replay(const ReplayArgs& a, int in_bf16, int read_fmt, cudaStream_t st);
+cudaError_t launch_fold(const FoldArgs& a, int in_bf16, int upd_fmt, cudaStream_t st);
+cudaError_t launch_conv(const ConvArgs& a, int in_bf16, int verify, cudaStream_t st);
+cudaError_t launch_accept(int batch, int K, int cap, const int32_t* n, int32_t* pos, int32_t* err, int add_one,
+                          cudaStream_t st);
+cudaError_t launch_round_test(int op, int64_t n, const float* v, uint64_t seed, uint32_t c1, uint32_t c2,
+                              uint32_t c3, void* out, cudaStream_t st);
+
+// Dynamic shared memory of one CTA, in bytes.
+size_t replay_smem_bytes(const Shape& s, int read_fmt, int ntok, int fused);
+size_t fold_smem_bytes(const Shape& s, int upd_fmt);
+size_t conv_smem_bytes(const Shape& s);
+
+}  // namespace rssm

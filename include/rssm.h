@@ -1,0 +1,260 @@
+/*
+ * rssm.h -- C ABI of librssm: replay-based decoding of the state-space (SSM)
+ * layers of hybrid SSM/attention models on NVIDIA B200 (sm_100a).
+ *
+ * Method: the ReplaySSM article (devotd.net news page
+ * "nvidia-replayssm-hybrid-model-ssm-decoding-state-buffer", English
+ * version), sections
+ *   s1 "Store recent inputs instead of the full state"
+ *   s3 "Roll back incorrect predictions using buffer positions"
+ *   s4 "Prevent low-precision errors from accumulating again".
+ * The article fixes the idea; the concrete layer is a Mamba-2-style selective
+ * SSM with one scalar decay per head h, head_dim P, d_state N, and G groups
+ * of H/G consecutive heads sharing B and C:
+ *     a_t = exp(dt_t A_h),  h_t = a_t h_{t-1} + dt_t x_t B_t^T,  y_t = h_t C_t + D_h x_t.
+ * Per request the library keeps a checkpoint of h taken at the start of an
+ * interval of L tokens plus a buffer of the inputs since then (x, B, dt; C
+ * is per token and is not kept). Every token reads the checkpoint once and
+ * replays the buffer; the checkpoint is rewritten only when the buffer
+ * fills (s1):
+ *     y_t = exp(A S_t) (h_ckpt C_t) + sum_{s<=t} dt_s exp(A (S_t - S_s)) (B_s . C_t) x_s + D x_t,
+ *     S_t = sum_{r<=t} dt_r over the interval.
+ *
+ * Conventions for every call:
+ *  - All array arguments are DEVICE pointers into memory the caller owns
+ *    (e.g. allocated through PyTorch). The library never allocates, frees or
+ *    synchronises; rssm_get_error is the only call that waits (on its
+ *    stream). Sizes come from rssm_state_field_bytes.
+ *  - Inputs are read-only; layouts are dense and row-major as documented.
+ *    Device pointers must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Work is
+ *    enqueued asynchronously; one state must be used from one stream.
+ *  - Arguments the host can check are checked before anything is launched;
+ *    a bad one returns a status and launches nothing.
+ *  - Kernels that find bad device state (a buffer position out of range, an
+ *    accepted count out of range) write the first error code into
+ *    state->err and leave that request untouched. They never trap, assert
+ *    or spin without a bound. rssm_get_error reads and clears the word.
+ */
+#ifndef RSSM_H
+#define RSSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RSSM_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define RSSM_API __attribute__((visibility("default")))
+#else
+#define RSSM_API
+#endif
+
+typedef enum rssm_status {
+    RSSM_OK = 0,
+    RSSM_ERR_INVALID_ARG = 1,  /* null pointer or bad enum value */
+    RSSM_ERR_SHAPE = 2,        /* sizes inconsistent or outside the supported range */
+    RSSM_ERR_UNSUPPORTED = 3,  /* valid but not implemented combination */
+    RSSM_ERR_CAPACITY = 4,     /* more tokens than the buffer can ever hold */
+    RSSM_ERR_CUDA = 5,         /* a CUDA runtime call failed */
+    RSSM_ERR_DEVICE = 6        /* rssm_get_error: a kernel reported bad device state */
+} rssm_status_t;
+
+/* Element formats. F32/BF16 for inputs and the update copy; E4M3 (OCP fp8)
+ * for the update copy; FP4 = e2m1 codes with one e4m3 scale per 16
+ * contiguous d_state elements. */
+typedef enum rssm_dtype { RSSM_F32 = 0, RSSM_BF16 = 1, RSSM_E4M3 = 2, RSSM_FP4 = 3 } rssm_dtype_t;
+
+typedef enum rssm_outcopy { RSSM_OUTCOPY_NONE = 0, RSSM_OUTCOPY_FP4 = 1 } rssm_outcopy_t;
+
+/* Codes a kernel writes into state->err (first error wins). */
+enum {
+    RSSM_DEVERR_NONE = 0,
+    RSSM_DEVERR_POS_RANGE = 1,    /* pos[b] < 0 or > capacity */
+    RSSM_DEVERR_CAPACITY = 2,     /* pos[b] + tokens > capacity */
+    RSSM_DEVERR_ACCEPT_RANGE = 3, /* accepted count outside 0..K */
+    RSSM_DEVERR_TIMEOUT = 4       /* a bulk copy did not complete within its bound */
+};
+
+/* desc.flags */
+#define RSSM_FLAG_FUSED_FLUSH 1u  /* rssm_decode_step folds the buffer itself on the
+                                     token that fills it (fp32 state only) */
+
+/* Layer description. Supported: batch >= 1; nheads % ngroups == 0;
+ * d_state in {16, 32, 64, 128}; 1 <= head_dim <= 256;
+ * head_dim * d_state <= 16384; 1 <= interval; capacity = interval +
+ * max_draft <= 32; FP4 state or copy needs head_dim * d_state % 256 == 0. */
+typedef struct rssm_desc {
+    int32_t batch;        /* requests */
+    int32_t nheads;       /* H */
+    int32_t head_dim;     /* P */
+    int32_t d_state;      /* N */
+    int32_t ngroups;      /* G */
+    int32_t interval;     /* L: tokens per checkpoint interval (16 in the article) */
+    int32_t max_draft;    /* K: most draft tokens per verify; buffer capacity L + K */
+    int32_t in_dtype;     /* RSSM_F32 or RSSM_BF16: x, B, C and the buffered x, B */
+    int32_t update_dtype; /* update copy: F32; BF16 or E4M3 (stochastic rounding);
+                             FP4 = one FP4 copy both read and updated (the
+                             shared-low-precision control of s4) */
+    int32_t out_copy;     /* RSSM_OUTCOPY_FP4: separate FP4 output copy (s4), read by
+                             decode/verify; requires update_dtype != FP4 */
+    uint32_t flags;       /* RSSM_FLAG_* */
+    uint32_t reserved;    /* must be 0 */
+    uint64_t seed;        /* Philox key of the stochastic rounding */
+} rssm_desc_t;
+
+/* Fields of the per-layer state, for rssm_state_field_bytes. Cap = L + K. */
+typedef enum rssm_field {
+    RSSM_FIELD_CKPT = 0,       /* update copy [batch][H][P][N] in update_dtype
+                                  (FP4: codes [batch][H][P][N/2]) */
+    RSSM_FIELD_CKPT_SCALES,    /* FP4 update copy only: e4m3 [batch][H][P][N/16] */
+    RSSM_FIELD_OUT_CODES,      /* FP4 output copy: codes [batch][H][P][N/2] */
+    RSSM_FIELD_OUT_SCALES,     /* FP4 output copy: e4m3 [batch][H][P][N/16] */
+    RSSM_FIELD_XBUF,           /* buffered x  [batch][H][Cap][P] in in_dtype */
+    RSSM_FIELD_BBUF,           /* buffered B  [batch][G][Cap][N] in in_dtype */
+    RSSM_FIELD_DTBUF,          /* buffered dt [batch][H][Cap] float */
+    RSSM_FIELD_POS,            /* int32 [batch]: valid buffer length */
+    RSSM_FIELD_FLUSH_COUNT,    /* uint32 [batch]: refreshes so far (Philox counter word) */
+    RSSM_FIELD_ARRIVE,         /* uint32 [batch]: scratch, must be zero before first use;
+                                  every call leaves it zero */
+    RSSM_FIELD_ERR,            /* int32 [1]: device error word, zero-initialised */
+    RSSM_NUM_FIELDS
+} rssm_field_t;
+
+/* FP4 codes: element 2k in the low nibble of byte k, 2k+1 in the high one.
+ * Unused fields may be NULL. */
+typedef struct rssm_state {
+    void *ckpt;
+    void *ckpt_scales;
+    void *out_codes;
+    void *out_scales;
+    void *xbuf;
+    void *bbuf;
+    float *dtbuf;
+    int32_t *pos;
+    uint32_t *flush_count;
+    uint32_t *arrive;
+    int32_t *err;
+} rssm_state_t;
+
+/* ABI version (RSSM_ABI_VERSION). */
+RSSM_API int rssm_abi_version(void);
+
+/* Static text for a status. Never NULL. */
+RSSM_API const char *rssm_status_string(rssm_status_t s);
+
+/* Validates a description: RSSM_OK, or the status any call would return. */
+RSSM_API rssm_status_t rssm_check_desc(const rssm_desc_t *desc);
+
+/* Bytes of one state field for this description; 0 when the field is unused
+ * or the description is invalid. Host-only; touches no device. */
+RSSM_API size_t rssm_state_field_bytes(const rssm_desc_t *desc, int32_t field);
+
+/* Standard decode of one token per request (s1): appends (x, B, dt) at
+ * slot pos[b], writes y, advances pos[b] by one. Reads the checkpoint (or,
+ * with an FP4 output copy, that copy) once; writes no state except the
+ * buffer slot. The caller calls rssm_flush / rssm_lowprec_refresh once
+ * pos reaches the interval, unless RSSM_FLAG_FUSED_FLUSH is set, in which
+ * case the token that fills the buffer also folds it and resets pos.
+ *   x [batch][H][P], B and C [batch][G][N] (in_dtype); dt [batch][H]
+ *   (float, already softplus-ed, > 0); A, D [H] float; y [batch][H][P] float.
+ * Device errors: pos[b] + 1 > capacity. */
+RSSM_API rssm_status_t rssm_decode_step(const rssm_desc_t *desc, const rssm_state_t *state,
+                               const void *x, const void *B, const void *C,
+                               const float *dt, const float *A, const float *D,
+                               float *y, void *stream);
+
+/* Interval flush of an fp32 state (s1): for every request with
+ * pos[b] >= interval (all requests with pos[b] > 0 when force != 0), fold
+ * the pos[b] buffered entries into the checkpoint in one read-modify-write
+ *     h <- exp(A S) h + sum_s dt_s exp(A (S - S_s)) x_s B_s^T,  S = sum of the pos dt,
+ * then pos[b] = 0 and flush_count[b] += 1. Other requests are untouched.
+ * A [H] float: the same decay parameters the decode calls received.
+ * Requires update_dtype F32 and no output copy (else RSSM_ERR_UNSUPPORTED;
+ * use rssm_lowprec_refresh). */
+RSSM_API rssm_status_t rssm_flush(const rssm_desc_t *desc, const rssm_state_t *state, const float *A,
+                         int32_t force, void *stream);
+
+/* Speculative verify (s3): writes the K+1 tokens (the pending token j = 0
+ * and K drafts) into slots pos..pos+K and computes their outputs from one
+ * read of the checkpoint. pos is NOT advanced and no state is created.
+ *   x [batch][K+1][H][P], B and C [batch][K+1][G][N], dt [batch][K+1][H],
+ *   y [batch][K+1][H][P].
+ * 0 <= K <= max_draft, else RSSM_ERR_CAPACITY. Device error: pos + K + 1 >
+ * capacity. */
+RSSM_API rssm_status_t rssm_verify(const rssm_desc_t *desc, const rssm_state_t *state, int32_t K,
+                          const void *x, const void *B, const void *C, const float *dt,
+                          const float *A, const float *D, float *y, void *stream);
+
+/* Accept after verify (s3): pos[b] += n_accepted[b] + 1, which marks the
+ * pending token and the first n accepted drafts valid and drops the rest.
+ * n_accepted: device int32 [batch], each in 0..max_draft (else device error,
+ * request untouched). Follow with rssm_flush / rssm_lowprec_refresh
+ * (force = 0), which fold requests whose pos reached the interval. */
+RSSM_API rssm_status_t rssm_accept(const rssm_desc_t *desc, const rssm_state_t *state,
+                          const int32_t *n_accepted, void *stream);
+
+/* Precision-split refresh (s4): as rssm_flush, on the low-precision state.
+ * Widens the update copy to fp32, folds the buffer, then
+ *   - BF16/E4M3 update copy: stochastic rounding with Philox4x32-10, key
+ *     (lo32(seed), hi32(seed)), counter (e/4, h, b, flush_count[b]), word
+ *     e%4, e = p*N + n; up iff r < floor(frac * 2^32);
+ *   - F32 update copy: stored as computed;
+ *   - FP4 update copy (shared control): re-quantised to nearest;
+ *   - FP4 output copy (out_copy): quantised from the fp32 result, before
+ *     stochastic rounding: scale = e4m3_rn(amax/6) per 16 elements, codes =
+ *     e2m1_rn(v / scale), all zero when the scale is zero.
+ * With force != 0 every request is refreshed, including pos[b] == 0, which
+ * (re)builds the output copy from the update copy. */
+RSSM_API rssm_status_t rssm_lowprec_refresh(const rssm_desc_t *desc, const rssm_state_t *state,
+                                   const float *A, int32_t force, void *stream);
+
+/* Conventional decode step, the in-run comparison (s1: read and write the
+ * whole state every token): h <- a h + dt x B^T; y = h C + D x.
+ * h [batch][H][P][N] float, updated in place; other arguments as in
+ * rssm_decode_step. Uses only the shape fields of desc. */
+RSSM_API rssm_status_t rssm_conv_step(const rssm_desc_t *desc, float *h, const void *x, const void *B,
+                             const void *C, const float *dt, const float *A, const float *D,
+                             float *y, void *stream);
+
+/* Conventional speculative verify (s3: one state copy per token for
+ * rollback): reads state copy cur[b] of copies [K+1][batch][H][P][N] and
+ * writes the state after token j into copy j, for j = 0..K, with outputs
+ * y [batch][K+1][H][P]. cur: device int32 [batch], each in 0..K. */
+RSSM_API rssm_status_t rssm_conv_verify(const rssm_desc_t *desc, float *copies, const int32_t *cur,
+                               int32_t K, const void *x, const void *B, const void *C,
+                               const float *dt, const float *A, const float *D, float *y,
+                               void *stream);
+
+/* Conventional accept: cur[b] = n_accepted[b] (the copy after the last
+ * accepted token becomes the state; nothing is copied). Values outside 0..K
+ * leave cur[b] unchanged and set *err (err may be NULL). */
+RSSM_API rssm_status_t rssm_conv_accept(const rssm_desc_t *desc, const int32_t *n_accepted, int32_t *cur,
+                               int32_t K, int32_t *err, void *stream);
+
+/* Reads and clears the device error word; waits for the stream first.
+ * *host_code receives the RSSM_DEVERR_* value. Returns RSSM_ERR_DEVICE when
+ * it was non-zero. */
+RSSM_API rssm_status_t rssm_get_error(const rssm_desc_t *desc, const rssm_state_t *state,
+                             int32_t *host_code, void *stream);
+
+/* Rounding functions of the refresh, exposed for bit-exact testing on the
+ * device code the refresh itself runs. For n input floats v:
+ *   op 0: SR to bf16      -> uint16 out[n]   (Philox counter (e/4, c1, c2, c3))
+ *   op 1: SR to e4m3      -> uint8  out[n]   (same counter)
+ *   op 2: e4m3 nearest-even, saturating -> uint8 out[n]
+ *   op 3: FP4 block copy  -> uint8 out[n/2] codes, then uint8 out[n/2 + n/16] scales
+ *   op 4: Philox word e%4 at (e/4, c1, c2, c3)  -> uint32 out[n]
+ * n must be a multiple of 16 for op 3. */
+RSSM_API rssm_status_t rssm_round_test(int32_t op, int64_t n, const float *v, uint64_t seed, uint32_t c1,
+                              uint32_t c2, uint32_t c3, void *out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RSSM_H */
