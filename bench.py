@@ -52,7 +52,10 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--fused", action="store_true", help="fold the buffer inside the 16th decode (no flush call)")
-    p.add_argument("--no-extra", action="store_true", help="skip the comparison / large-layer / e2e legs")
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the comparison, large-layer, e2e and CPU-baseline legs")
+    p.add_argument("--profile", action="store_true",
+                   help="untimed: run every hot kernel a few times on the bench workloads (for ncu)")
     return p.parse_args()
 
 
@@ -156,6 +159,24 @@ def smi_gpu_id(torch, dev):
         return dev
 
 
+# ---------------------------------------------------- multi-rank plumbing
+
+def reduce_max(value, dist=None, device=None):
+    """Max of a per-rank float over all ranks (the job's time is the slowest
+    rank's); identity on one rank."""
+    if dist is None or not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, max_ms):
+    """Whole-job units/s: every rank processed units_per_rank in at most max_ms."""
+    return world * units_per_rank / (max_ms / 1e3)
+
+
 # ------------------------------------------------------ analytic bytes
 
 def shape_bytes(shape, in_bytes=2):
@@ -206,11 +227,7 @@ def run_ours(args):
             dist.barrier()
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, dist, dev)
 
     K, W = args.steps, args.warmup
     wl = WORKLOADS["small_b256"]
@@ -271,8 +288,7 @@ def run_ours(args):
     sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1)
 
-    tokens = world * shape.batch * L * K
-    value = tokens / (ms / 1e3)
+    value = job_throughput(shape.batch * L * K, world, ms)
     dec_ms = [a.elapsed_time(b) for a, b in ev_d]
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
     dec_bytes = sum(decode_bytes_per_request(shape, i) for i in range(L)) / L * shape.batch
@@ -311,7 +327,7 @@ def run_ours(args):
         torch.cuda.empty_cache()
         out["large_b512"] = large_leg(rssm, torch, WORKLOADS["large_b512"], max(2, min(K, 50)), W, dev, barrier,
                                       max_over_ranks, world, peak, args.fused)
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.no_extra:
         out["cpu_baseline"] = cpu_baseline()
     if world > 1:
         dist.destroy_process_group()
@@ -506,8 +522,77 @@ def run_reference(args):
     }))
 
 
+def run_profile():
+    """Each hot kernel a few times, untimed, on the small_b256 layer: 2
+    intervals of replay decode + flush, the same with the fused fold, 32
+    conventional steps, 4 speculative steps (K = 4, replay and conventional)
+    and one interval of the bf16 + FP4 precision split."""
+    import torch
+
+    from hybrid_model_ssm_replay_b200 import rssm
+    from hybrid_model_ssm_replay_b200.inputs import WORKLOADS, LayerShape, accept_lengths, make_inputs
+    torch.cuda.set_device(0)
+    wl = WORKLOADS["small_b256"]
+    sh = wl["shape"]
+    L = sh.interval
+    inp = make_inputs(sh, L, wl["seed"], wl["in_dtype"], device="cuda")
+    y = torch.empty((sh.batch, sh.nheads, sh.head_dim), device="cuda")
+    for flags in (0, rssm.RSSM_FLAG_FUSED_FLUSH):
+        d = rssm.make_desc(sh.batch, sh.nheads, sh.head_dim, sh.d_state, sh.ngroups, interval=L, flags=flags)
+        st = rssm.RssmState(d)
+        st.ckpt.copy_(inp["ckpt"])
+        for _ in range(2):
+            for t in range(L):
+                rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"], y)
+            if not flags:
+                rssm.rssm_flush(st, inp["A"])
+        del st
+    d = rssm.make_desc(sh.batch, sh.nheads, sh.head_dim, sh.d_state, sh.ngroups)
+    h = inp["ckpt"].clone()
+    for t in range(2 * L):
+        rssm.rssm_conv_step(d, h, inp["x"][t % L], inp["B"][t % L], inp["C"][t % L], inp["dt"][t % L], inp["A"],
+                            inp["D"], y)
+    del h
+    K = 4
+    ssh = LayerShape(sh.batch, sh.nheads, sh.head_dim, sh.d_state, sh.ngroups, L, K)
+    si = make_inputs(ssh, 4, 3, wl["in_dtype"], device="cuda", ntok=K + 1)
+    n = accept_lengths(4, sh.batch, K, 3, device="cuda")
+    ds = rssm.make_desc(sh.batch, sh.nheads, sh.head_dim, sh.d_state, sh.ngroups, interval=L, max_draft=K)
+    st = rssm.RssmState(ds)
+    st.ckpt.copy_(si["ckpt"])
+    ys = torch.empty((sh.batch, K + 1, sh.nheads, sh.head_dim), device="cuda")
+    for s in range(4):
+        rssm.rssm_verify(st, K, si["x"][s], si["B"][s], si["C"][s], si["dt"][s], si["A"], si["D"], ys)
+        rssm.rssm_accept(st, n[s])
+        rssm.rssm_flush(st, si["A"], force=(s == 3))
+    del st
+    copies = torch.zeros((K + 1,) + tuple(si["ckpt"].shape), device="cuda")
+    copies[0].copy_(si["ckpt"])
+    cur = torch.zeros(sh.batch, dtype=torch.int32, device="cuda")
+    for s in range(4):
+        rssm.rssm_conv_verify(ds, copies, cur, K, si["x"][s], si["B"][s], si["C"][s], si["dt"][s], si["A"],
+                              si["D"], ys)
+        rssm.rssm_conv_accept(ds, n[s], cur, K)
+    del copies
+    dl = rssm.make_desc(sh.batch, sh.nheads, sh.head_dim, sh.d_state, sh.ngroups, interval=L,
+                        update_dtype=rssm.RSSM_BF16, out_copy=rssm.RSSM_OUTCOPY_FP4, seed=4)
+    st = rssm.RssmState(dl)
+    st.ckpt.copy_(inp["ckpt"].to(torch.bfloat16))
+    rssm.rssm_lowprec_refresh(st, inp["A"], force=True)
+    for t in range(L):
+        rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"], y)
+    rssm.rssm_lowprec_refresh(st, inp["A"])
+    torch.cuda.synchronize()
+    if rssm.rssm_get_error(st) != 0:
+        raise RuntimeError("device error")
+    print("profile run done")
+
+
 def main():
     args = parse_args()
+    if args.profile:
+        run_profile()
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -42,6 +42,7 @@ Shape shape_of(const rssm_desc_t* d) {
     s.L = d->interval;
     s.cap = cap_of(d);
     s.lpr = d->d_state / 4;
+    s.capr = (s.cap + 3) & ~3;
     return s;
 }
 
@@ -127,7 +128,7 @@ size_t rssm_state_field_bytes(const rssm_desc_t* d, int32_t field) {
         case RSSM_FIELD_OUT_SCALES: return d->out_copy == RSSM_OUTCOPY_FP4 ? n_state / 16 : 0;
         case RSSM_FIELD_XBUF: return Bz * H * cap * P * in_el;
         case RSSM_FIELD_BBUF: return Bz * G * cap * N * in_el;
-        case RSSM_FIELD_DTBUF: return Bz * H * cap * 4;
+        case RSSM_FIELD_DTBUF: return Bz * H * ((cap + 3) & ~static_cast<size_t>(3)) * 4;
         case RSSM_FIELD_POS: return Bz * 4;
         case RSSM_FIELD_FLUSH_COUNT: return Bz * 4;
         case RSSM_FIELD_ARRIVE: return Bz * 4;
@@ -242,6 +243,7 @@ static rssm_status_t conv_launch(const rssm_desc_t* d, float* h, const int32_t* 
     a.s = shape_of(d);
     a.s.L = 1;
     a.s.cap = 1;
+    a.s.capr = 4;
     a.ntok = ntok;
     a.h = h;
     a.cur = cur;
@@ -302,7 +304,8 @@ rssm_status_t rssm_get_error(const rssm_desc_t* d, const rssm_state_t* st, int32
 
 rssm_status_t rssm_round_test(int32_t op, int64_t n, const float* v, uint64_t seed, uint32_t c1, uint32_t c2,
                               uint32_t c3, void* out, void* stream) {
-    if (op < 0 || op > 4 || n < 0) return RSSM_ERR_INVALID_ARG;
+    if (op < 0 || op > 5 || n < 0) return RSSM_ERR_INVALID_ARG;
+    if (op == 5 && n % 16 != 0) return RSSM_ERR_SHAPE;
     if (op == 3 && n % 16 != 0) return RSSM_ERR_SHAPE;
     if (n > 0 && (!v || !out)) return RSSM_ERR_INVALID_ARG;
     return cuda_status(launch_round_test(op, n, v, seed, c1, c2, c3, out, static_cast<cudaStream_t>(stream)));

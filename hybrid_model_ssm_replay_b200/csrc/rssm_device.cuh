@@ -22,6 +22,9 @@ constexpr int kThreads = 256;               // threads per CTA of every tile ker
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxCap = 32;                 // buffer slots per request (interval + drafts)
 constexpr int kMaxTok = 8;                  // tokens per verify call (K + 1)
+constexpr int kMidTok = 5;                  // verify kernels specialised for K <= 4
+constexpr int kPipeStagesMax = 8;           // shared-memory stages of the pipelined replay kernel
+constexpr int kConsWarps = 8;               // warps of one consumer group
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bound of one bulk-copy wait
 
 // ------------------------------------------------------------------ errors
@@ -54,14 +57,16 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
         : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+// One bounded try: the thread may sleep until the phase completes or about
+// `hint_ns` pass. True once phase `parity` has completed.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
         : "memory");
     return ok != 0;
 }
@@ -72,11 +77,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
-// Waits for phase `parity` of the barrier, at most limit_ns. True on completion.
+// Waits for phase `parity` of the barrier, at most about limit_ns. True on completion.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity, 100000u)) return true;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait(bar, parity, 100000u)) {
         if (globaltimer_ns() - t0 > limit_ns) return false;
     }
     return true;
@@ -192,18 +197,18 @@ __device__ __forceinline__ float e4m3_val(uint32_t c) {
 
 __device__ __forceinline__ float bf16_val(uint32_t bits) { return __uint_as_float(bits << 16); }
 
-// Four e2m1 codes (16 bits, element 0 in the low nibble) to floats.
-__device__ __forceinline__ float4 fp4x4_val(uint32_t codes16) {
-    uint32_t h01, h23;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "mov.b32 {b0, b1, b2, b3}, %2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t}"
-        : "=r"(h01), "=r"(h23)
-        : "r"(codes16));
-    const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
-    const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
-    return make_float4(f01.x, f01.y, f23.x, f23.y);
+// Four e2m1 codes (16 bits, element 0 in the low nibble) times a scale, exactly.
+// Each nibble's magnitude bits go to bits 11..9 of an fp16 (the low exponent
+// bits and the top mantissa bit) and its sign to bit 15: the fp16 then holds
+// the e2m1 value times 2^-14 (e2m1's subnormal 0.5 lands on an fp16
+// subnormal), so scale2p14 = scale * 2^14 restores it. Products are exact.
+__device__ __forceinline__ float4 fp4x4_val(uint32_t codes16, float scale2p14) {
+    const uint32_t c0 = codes16 & 0xFFu, c1 = (codes16 >> 8) & 0xFFu;
+    const uint32_t w01 = ((c0 & 0x7u) << 9) | ((c0 & 0x8u) << 12) | ((c0 & 0x70u) << 21) | ((c0 & 0x80u) << 24);
+    const uint32_t w23 = ((c1 & 0x7u) << 9) | ((c1 & 0x8u) << 12) | ((c1 & 0x70u) << 21) | ((c1 & 0x80u) << 24);
+    const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&w01));
+    const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&w23));
+    return make_float4(f01.x * scale2p14, f01.y * scale2p14, f23.x * scale2p14, f23.y * scale2p14);
 }
 
 // Four e4m3 codes (32 bits, element 0 in the low byte) to floats.

@@ -9,9 +9,10 @@ namespace rssm {
 
 enum Fmt : int { kF32 = 0, kBF16 = 1, kE4M3 = 2, kFP4 = 3 };
 
-// Shapes shared by every kernel. lpr = d_state / 4 lanes per state row.
+// Shapes shared by every kernel. lpr = d_state / 4 lanes per state row;
+// capr = cap rounded up to 4 is the row stride of the dt buffer (16-byte rows).
 struct Shape {
-    int batch, H, P, N, G, L, cap, lpr;
+    int batch, H, P, N, G, L, cap, lpr, capr;
 };
 
 // Replay decode / verify (ReplaySSM article s1, s3).
@@ -37,6 +38,31 @@ struct ReplayArgs {
     const float* A;
     const float* D;
     float* y;
+};
+
+// Division by a run-time constant d (1 <= d < 2^31) for 0 <= x < 2^31:
+// q = (umulhi(x, mul) + x) >> shr (round-up reciprocal, Granlund-Montgomery).
+struct FastDiv {
+    uint32_t d, mul, shr;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+    FastDiv f;
+    f.d = d;
+    uint32_t s = 0;
+    while ((1ull << s) < d) ++s;
+    f.shr = s;
+    f.mul = static_cast<uint32_t>(((1ull << 32) * ((1ull << s) - d)) / d + 1);
+    return f;
+}
+
+// Shared-memory stage of the pipelined replay kernel: byte offsets of the
+// state tile, FP4 scales, x rows [cap][P], B rows [cap][N], C rows [ntok][N],
+// dt row [capr], this call's dt [8] and the position; `stages` stages.
+struct PipeLayout {
+    uint32_t stage_bytes, tile, scales, xrows, brows, crows, dtrow, dtnew, meta;
+    int stages;
+    FastDiv divH, divHpg;  // tile -> (request, head), head -> group
 };
 
 // Fold of the buffer into the update copy (flush / refresh; s1, s4).

@@ -44,13 +44,7 @@ __device__ __forceinline__ float4 tile_load4(const unsigned char* t, const unsig
     } else if constexpr (F == kE4M3) {
         return e4m3x4_val(reinterpret_cast<const uint32_t*>(t)[q]);
     } else {
-        const float s = e4m3_val(sc[q >> 2]);
-        float4 v = fp4x4_val(reinterpret_cast<const uint16_t*>(t)[q]);
-        v.x *= s;
-        v.y *= s;
-        v.z *= s;
-        v.w *= s;
-        return v;
+        return fp4x4_val(reinterpret_cast<const uint16_t*>(t)[q], e4m3_val(sc[q >> 2]) * 16384.0f);
     }
 }
 
@@ -80,55 +74,118 @@ __device__ __forceinline__ float warp_prefix(float v) {
     return v;
 }
 
-// The fold of s1: v[r][c] = alpha * tile[r][c] + sum_{s<T} xw[s][r] * B_s[c],
-// with xw[s][r] = dt_s exp(A (S_T - S_s)) x_s[r] staged in shared memory and
-// the lane's B_s columns held in registers, 16 slots at a time. `s32` is the
-// fp32 tile in shared memory (rewritten between chunks); brow(s, c) gives
-// B_s columns 4c..4c+3; emit(r, c, v, valid) is called by every lane for
-// the final values (valid = row in range).
+__host__ __device__ inline int round_up8(int x) { return (x + 7) & ~7; }
+
+constexpr int kRB = 8;  // fold: rows per thread (register block)
+
+// The fold of s1 as a register-blocked rank-T update:
+//   v[r][c] = alpha * tile[r][c] + sum_{s<T} xw[s][r] * B_s[c],
+// xw[s][r] = dt_s exp(A (S_T - S_s)) x_s[r] in shared memory with row stride
+// xs = round_up8(P). A thread owns kRB consecutive rows and one group of 4
+// columns, keeps their accumulators in registers and streams over s: per s
+// one float4 of B (brow(s, c)) and two float4 of xw. emit(r, c, v, valid)
+// is called by every lane for every owned row (valid = row in range).
 template <typename BRow, typename Emit>
-__device__ __forceinline__ void fold_rows(float* s32, const float* s_xw, int P, int N, int lpr, int T,
-                                          float alpha, BRow brow, Emit emit) {
+__device__ __forceinline__ void fold_tile(const float* s32, const float* s_xw, int xs, int P, int N, int lpr,
+                                          int T, float alpha, BRow brow, Emit emit) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int lsh = __ffs(lpr) - 1;
     const int rpw = 32 >> lsh, col4 = lane & (lpr - 1), rsub = lane >> lsh;
-    const int nchunk = T > 0 ? (T + 15) >> 4 : 1;
-    for (int ch = 0; ch < nchunk; ++ch) {
-        float4 br[16];
+    const int rows_per_pass = kWarps * rpw * kRB;
+    for (int base = 0; base < P; base += rows_per_pass) {
+        const int rb = base + (warp * rpw + rsub) * kRB;
+        float4 acc[kRB];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int s = ch * 16 + i;
-            br[i] = (s < T) ? brow(s, col4) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        const bool last = (ch == nchunk - 1);
-        for (int r0 = warp * rpw; r0 < P; r0 += kWarps * rpw) {
-            const int r = r0 + rsub;
-            const bool valid = r < P;
-            float4 v = valid ? reinterpret_cast<const float4*>(s32)[r * (N >> 2) + col4]
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-            if (ch == 0) {
+        for (int k = 0; k < kRB; ++k) {
+            const int r = rb + k;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r < P) {
+                v = reinterpret_cast<const float4*>(s32)[r * (N >> 2) + col4];
                 v.x *= alpha;
                 v.y *= alpha;
                 v.z *= alpha;
                 v.w *= alpha;
             }
+            acc[k] = v;
+        }
+        if (rb < P) {
+#pragma unroll 2
+            for (int s = 0; s < T; ++s) {
+                const float4 bv = brow(s, col4);
+                const float4* xw4 = reinterpret_cast<const float4*>(s_xw + s * xs + rb);
+                const float4 xa = xw4[0], xb = xw4[1];
+                const float w[kRB] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int s = ch * 16 + i;
-                if (s < T) {
-                    const float xw = valid ? s_xw[s * P + r] : 0.f;
-                    v.x = fmaf(xw, br[i].x, v.x);
-                    v.y = fmaf(xw, br[i].y, v.y);
-                    v.z = fmaf(xw, br[i].z, v.z);
-                    v.w = fmaf(xw, br[i].w, v.w);
+                for (int k = 0; k < kRB; ++k) {
+                    acc[k].x = fmaf(w[k], bv.x, acc[k].x);
+                    acc[k].y = fmaf(w[k], bv.y, acc[k].y);
+                    acc[k].z = fmaf(w[k], bv.z, acc[k].z);
+                    acc[k].w = fmaf(w[k], bv.w, acc[k].w);
                 }
             }
-            if (last)
-                emit(r, col4, v, valid);
-            else if (valid)
-                reinterpret_cast<float4*>(s32)[r * (N >> 2) + col4] = v;
         }
+#pragma unroll
+        for (int k = 0; k < kRB; ++k) emit(rb + k, col4, acc[k], rb + k < P);
     }
+}
+
+// Eight consecutive input elements as raw bits (one or two 16-byte accesses).
+template <typename TIn> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+    uint4 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = *reinterpret_cast<const uint4*>(p); }
+    __device__ __forceinline__ void store(__nv_bfloat16* p) const { *reinterpret_cast<uint4*>(p) = u; }
+    __device__ __forceinline__ float4 lo() const { return bf16x4_val(make_uint2(u.x, u.y)); }
+    __device__ __forceinline__ float4 hi() const { return bf16x4_val(make_uint2(u.z, u.w)); }
+};
+template <> struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p) {
+        a = reinterpret_cast<const float4*>(p)[0];
+        b = reinterpret_cast<const float4*>(p)[1];
+    }
+    __device__ __forceinline__ void store(float* p) const {
+        reinterpret_cast<float4*>(p)[0] = a;
+        reinterpret_cast<float4*>(p)[1] = b;
+    }
+    __device__ __forceinline__ float4 lo() const { return a; }
+    __device__ __forceinline__ float4 hi() const { return b; }
+};
+
+// Sums 8 per-lane partials (rows 0..7 of a warp's block) over the 32 lanes
+// with a transpose butterfly (9 shuffles instead of 40): lanes exchange the
+// half of their rows that the partner keeps. Lane l returns the total of
+// row (l >> 2) & 7. Fixed order, so the result is reproducible.
+__device__ __forceinline__ float warp_reduce8(const float (&v)[8]) {
+    const int lane = threadIdx.x & 31;
+    const bool b16 = lane & 16, b8 = lane & 8, b4 = lane & 4;
+    float w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float send = b16 ? v[i] : v[i + 4];
+        const float keep = b16 ? v[i + 4] : v[i];
+        w[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    float u[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = b8 ? w[i] : w[i + 2];
+        const float keep = b8 ? w[i + 2] : w[i];
+        u[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    const float send = b4 ? u[0] : u[1];
+    float z = (b4 ? u[1] : u[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
+    z += __shfl_xor_sync(0xffffffffu, z, 2);
+    z += __shfl_xor_sync(0xffffffffu, z, 1);
+    return z;
+}
+
+// Four floats back to the input element type (exact for values that came from it).
+__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
+    const uint2 u = make_uint2((__float_as_uint(v.x) >> 16) | (__float_as_uint(v.y) & 0xFFFF0000u),
+                               (__float_as_uint(v.z) >> 16) | (__float_as_uint(v.w) & 0xFFFF0000u));
+    *reinterpret_cast<uint2*>(p) = u;
 }
 
 // ---------------------------------------------------------------------------
@@ -136,31 +193,60 @@ __device__ __forceinline__ void fold_rows(float* s32, const float* s_xw, int P, 
 //   y_j = exp(A S_t) (h_ckpt C_j) + sum_{s<=t} dt_s exp(A (S_t - S_s)) (B_s . C_j) x_s + D x_t,
 //   t = pos + j, for the ntok tokens of this call; S = prefix sum of the
 //   buffered dt. The new tokens are appended at slots pos..pos+ntok-1.
+//   While the tile streams in, the CTA stages x_s of every slot in shared
+//   memory, forms the decay weights (warp 0) and the B_s . C_j products
+//   (all warps), in two rounds of independent loads (this call's inputs
+//   with pos, then the buffered slots). After the tile lands, each row's
+//   output is one reduction over the row's lanes of the h.C dot product and
+//   the replay terms (lane l takes slots s = l mod lanes).
 //   RF: format of the copy read (fp32 checkpoint, bf16/e4m3 update copy, or
-//   FP4 copy). NT: compile-time bound on ntok.
+//   FP4 copy). NT: compile-time bound on ntok. FUSED: the token that fills
+//   the buffer also folds it into the fp32 checkpoint. WIDE: d_state 128 and
+//   head_dim a multiple of 8 -- 16-byte staging, a warp owns 8 consecutive
+//   rows, lane l is slot l, and the 8 rows reduce together (warp_reduce8).
 // ---------------------------------------------------------------------------
-template <typename TIn, int RF, int NT, int FUSED>
-__global__ void __launch_bounds__(kThreads) k_replay(const ReplayArgs a) {
+// Minimum resident CTAs per SM the register allocation must allow.
+__host__ __device__ constexpr int replay_min_blocks(int nt, int fused) {
+    return fused ? 4 : (nt == 1 ? 6 : (nt <= kMidTok ? 4 : 3));
+}
+
+template <typename TIn, int RF, int NT, int FUSED, int WIDE>
+__global__ void __launch_bounds__(kThreads, replay_min_blocks(NT, FUSED)) k_replay(const ReplayArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t bar;
-    __shared__ float s_w[NT][kMaxCap];
-    __shared__ float s_g[NT][kMaxCap];
-    __shared__ float s_decay[NT];
+    __shared__ float s_w[NT][kMaxCap];  // dt_s exp(A (S_t - S_s)) for token j; 0 for s > t
+    __shared__ float s_g[NT][kMaxCap];  // B_s . C_j
+    __shared__ float s_decay[NT];       // exp(A S_t)
+    __shared__ int s_pos;
 
-    const int H = a.s.H, P = a.s.P, N = a.s.N, G = a.s.G, cap = a.s.cap, lpr = a.s.lpr;
+    const int H = a.s.H, P = a.s.P, N = a.s.N, G = a.s.G, cap = a.s.cap;
+    const int lpr = WIDE ? 32 : a.s.lpr;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.x / H, h = blockIdx.x - b * H;
     const int hpg = H / G, g = h / hpg;
     const int ntok = a.ntok;
     const int lsh = __ffs(lpr) - 1;
     const int rpw = 32 >> lsh, col4 = lane & (lpr - 1), rsub = lane >> lsh;
+    const int xs = round_up8(P);
     const size_t bh = static_cast<size_t>(b) * H + h;
+    const size_t bg = static_cast<size_t>(b) * G + g;
+
+    // per-CTA bases: token j adds j*HP (x, y), j*GN (B, C), j*H (dt); slot s adds s*P, s*N
+    const size_t HP = static_cast<size_t>(H) * P, GN = static_cast<size_t>(G) * N;
+    const TIn* xin = static_cast<const TIn*>(a.x) + static_cast<size_t>(b) * ntok * HP + static_cast<size_t>(h) * P;
+    const TIn* Bin = static_cast<const TIn*>(a.B) + static_cast<size_t>(b) * ntok * GN + static_cast<size_t>(g) * N;
+    const TIn* Cin = static_cast<const TIn*>(a.C) + static_cast<size_t>(b) * ntok * GN + static_cast<size_t>(g) * N;
+    const float* dtin = a.dt + static_cast<size_t>(b) * ntok * H + h;
+    float* yout = a.y + static_cast<size_t>(b) * ntok * HP + static_cast<size_t>(h) * P;
+    TIn* xb = static_cast<TIn*>(a.xbuf) + bh * cap * P;
+    TIn* bb = static_cast<TIn*>(a.bbuf) + bg * cap * N;
+    float* dtb = a.dtbuf + bh * a.s.capr;
 
     const uint32_t tb = tile_bytes(RF, P, N), sb = scale_bytes(RF, P, N);
     unsigned char* s_tile = smem;
     unsigned char* s_sc = smem + align16(tb);
-    float* s_hc = reinterpret_cast<float*>(smem + align16(tb) + align16(sb));    // [ntok][P]
-    float* s_xw = s_hc + ((ntok * P + 3) & ~3);                                   // fused fold: [L][P]
+    float* s_x = reinterpret_cast<float*>(smem + align16(tb) + align16(sb));  // [cap][xs]
+    float* s_B = s_x + cap * xs;                                              // fused: [L][N]
     const uint32_t bar_a = smem_u32(&bar);
 
     if (tid == 0) {
@@ -168,33 +254,103 @@ __global__ void __launch_bounds__(kThreads) k_replay(const ReplayArgs a) {
         mbar_expect_tx(bar_a, tb + sb);
         bulk_g2s(smem_u32(s_tile), static_cast<const unsigned char*>(a.tile) + bh * tb, tb, bar_a);
         if (RF == kFP4) bulk_g2s(smem_u32(s_sc), a.tile_scales + bh * sb, sb, bar_a);
+        s_pos = a.pos[b];  // the only read of pos: every thread uses this copy
     }
 
-    const TIn* xin = static_cast<const TIn*>(a.x);
-    const TIn* Bin = static_cast<const TIn*>(a.B);
-    const TIn* Cin = static_cast<const TIn*>(a.C);
-    TIn* xb = static_cast<TIn*>(a.xbuf);
-    TIn* bb = static_cast<TIn*>(a.bbuf);
-
+    // ---- round 0: C rows, this call's x and dt (with the position, above)
     float4 c4[NT];
 #pragma unroll
     for (int j = 0; j < NT; ++j)
-        c4[j] = (j < ntok) ? load4(Cin + ((static_cast<size_t>(b) * ntok + j) * G + g) * N + 4 * col4)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        c4[j] = (j < ntok) ? load4(Cin + j * GN + 4 * col4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int nq_new = WIDE ? (ntok * P) >> 3 : 0;  // 8-element chunks of this call's x
+    __syncthreads();  // barrier initialised and pos read before anyone uses them
 
-    const int pos = a.pos[b];
+    const int pos = s_pos;
     const int T = pos + ntok;
     const bool ok = pos >= 0 && T <= cap;
+    const bool fold_now = FUSED && RF == kF32 && NT == 1 && ok && T == a.s.L;
     if (!ok && tid == 0) set_error(a.err, (pos < 0 || pos > cap) ? RSSM_DEVERR_POS_RANGE : RSSM_DEVERR_CAPACITY);
-    __syncthreads();  // barrier initialised before anyone waits on it
+    // past the barrier no thread of this CTA reads pos again; once every CTA
+    // of the request has arrived, the last one moves it
+    if (a.advance && ok && tid == kThreads - 32)
+        request_done(a.arrive, b, H, a.pos, fold_now ? 0 : pos + 1, a.flush_count, fold_now);
 
     if (ok) {
         const float Ah = a.A[h];
+        // ---- round 1 (independent loads): the buffered slots s < pos and this
+        // call's tokens -> shared memory; this call's tokens -> the buffer
+        if constexpr (WIDE) {
+            Raw8<TIn> xr;
+            if (tid < nq_new) {
+                const int e = tid << 3, j = e / P, p = e - j * P;
+                xr.load(xin + j * HP + p);
+            }
+            for (int q = tid; q < ((pos * P) >> 3); q += kThreads) {
+                const int e = q << 3, sl = e / P, p = e - sl * P;
+                Raw8<TIn> r;
+                r.load(xb + e);
+                float4* d = reinterpret_cast<float4*>(s_x + sl * xs + p);
+                d[0] = r.lo();
+                d[1] = r.hi();
+            }
+            if (tid < nq_new) {
+                const int e = tid << 3, j = e / P, p = e - j * P;
+                float4* d = reinterpret_cast<float4*>(s_x + (pos + j) * xs + p);
+                d[0] = xr.lo();
+                d[1] = xr.hi();
+                xr.store(xb + (pos + j) * P + p);
+            }
+            for (int q = tid + kThreads; q < nq_new; q += kThreads) {  // many tokens
+                const int e = q << 3, j = e / P, p = e - j * P;
+                Raw8<TIn> r;
+                r.load(xin + j * HP + p);
+                float4* d = reinterpret_cast<float4*>(s_x + (pos + j) * xs + p);
+                d[0] = r.lo();
+                d[1] = r.hi();
+                r.store(xb + (pos + j) * P + p);
+            }
+        } else {
+            constexpr int kNew = 2;
+            TIn xn[kNew];
+#pragma unroll
+            for (int k = 0; k < kNew; ++k) {
+                const int i = tid + k * kThreads;
+                xn[k] = (i < ntok * P) ? xin[(i / P) * HP + (i % P)] : TIn(0.f);
+            }
+            constexpr int kOld = 4;
+            for (int base = 0; base < pos * P; base += kOld * kThreads) {
+                float xo[kOld];
+#pragma unroll
+                for (int k = 0; k < kOld; ++k) {
+                    const int i = base + tid + k * kThreads;
+                    xo[k] = (i < pos * P) ? to_f32(xb[i]) : 0.f;
+                }
+#pragma unroll
+                for (int k = 0; k < kOld; ++k) {
+                    const int i = base + tid + k * kThreads;
+                    if (i < pos * P) s_x[(i / P) * xs + (i % P)] = xo[k];
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kNew; ++k) {
+                const int i = tid + k * kThreads;
+                if (i < ntok * P) {
+                    const int j = i / P, p = i - j * P;
+                    s_x[(pos + j) * xs + p] = to_f32(xn[k]);
+                    xb[(pos + j) * P + p] = xn[k];
+                }
+            }
+            for (int i = tid + kNew * kThreads; i < ntok * P; i += kThreads) {  // large head_dim or many tokens
+                const int j = i / P, p = i - j * P;
+                const TIn v = xin[j * HP + p];
+                s_x[(pos + j) * xs + p] = to_f32(v);
+                xb[(pos + j) * P + p] = v;
+            }
+        }
         if (warp == 0) {
-            float dts = 0.f;
-            if (lane < T)
-                dts = (lane < pos) ? a.dtbuf[bh * cap + lane]
-                                   : a.dt[(static_cast<size_t>(b) * ntok + (lane - pos)) * H + h];
+            const float dnew = (lane >= pos && lane < T) ? dtin[(lane - pos) * H] : 0.f;
+            const float dts = (lane < pos) ? dtb[lane] : dnew;
+            if (lane >= pos && lane < T) dtb[lane] = dnew;
             const float Sx = warp_prefix(dts);
 #pragma unroll
             for (int j = 0; j < NT; ++j) {
@@ -205,98 +361,490 @@ __global__ void __launch_bounds__(kThreads) k_replay(const ReplayArgs a) {
                 }
             }
         }
-        // g[j][s] = B_s . C_j over the T slots (buffered ones and this call's)
-        for (int s0 = warp * rpw; s0 < T; s0 += kWarps * rpw) {
-            const int s = s0 + rsub;
-            float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (s < T)
-                bv = (s < pos) ? load4(bb + ((static_cast<size_t>(b) * G + g) * cap + s) * N + 4 * col4)
-                               : load4(Bin + ((static_cast<size_t>(b) * ntok + (s - pos)) * G + g) * N + 4 * col4);
+        // g[j][s] = B_s . C_j; the group's first head appends this call's B rows
+        const bool leader = (h == g * hpg);
+        for (int s0 = warp * rpw; s0 < T; s0 += 2 * kWarps * rpw) {
+            const int sa = s0 + rsub, sb2 = s0 + kWarps * rpw + rsub;
+            auto bload = [&](int sl) {
+                if (sl >= T) return make_float4(0.f, 0.f, 0.f, 0.f);
+                return (sl < pos) ? load4(bb + sl * N + 4 * col4) : load4(Bin + (sl - pos) * GN + 4 * col4);
+            };
+            const float4 bva = bload(sa), bvb = bload(sb2);
+            if (leader) {
+                if (sa >= pos && sa < T) store4(bb + sa * N + 4 * col4, bva);
+                if (sb2 >= pos && sb2 < T) store4(bb + sb2 * N + 4 * col4, bvb);
+            }
+            if (fold_now) {
+                if (sa < T) reinterpret_cast<float4*>(s_B)[sa * (N >> 2) + col4] = bva;
+                if (sb2 < T) reinterpret_cast<float4*>(s_B)[sb2 * (N >> 2) + col4] = bvb;
+            }
 #pragma unroll
             for (int j = 0; j < NT; ++j) {
                 if (j < ntok) {
-                    const float d = group_sum(dot4(bv, c4[j]), lpr);
-                    if (s < T && col4 == 0) s_g[j][s] = d;
+                    const float da = group_sum(dot4(bva, c4[j]), lpr);
+                    const float db = group_sum(dot4(bvb, c4[j]), lpr);
+                    if (col4 == 0) {
+                        if (sa < T) s_g[j][sa] = da;
+                        if (sb2 < T) s_g[j][sb2] = db;
+                    }
                 }
-            }
-        }
-        // append this call's tokens at slots pos..pos+ntok-1
-        for (int i = tid; i < ntok * P; i += kThreads) {
-            const int j = i / P, p = i - j * P;
-            xb[(bh * cap + pos + j) * P + p] = xin[((static_cast<size_t>(b) * ntok + j) * H + h) * P + p];
-        }
-        if (tid < ntok) a.dtbuf[bh * cap + pos + tid] = a.dt[(static_cast<size_t>(b) * ntok + tid) * H + h];
-        if (h == g * hpg) {
-            for (int i = tid; i < ntok * N; i += kThreads) {
-                const int j = i / N, n = i - j * N;
-                bb[((static_cast<size_t>(b) * G + g) * cap + pos + j) * N + n] =
-                    Bin[((static_cast<size_t>(b) * ntok + j) * G + g) * N + n];
             }
         }
     }
 
-    const bool arrived = mbar_wait_bounded(bar_a, 0, kWaitNs);
+    // one thread waits for the tile; the barrier publishes it (and the
+    // staged rows, weights and dot products) to the whole CTA
+    bool arrived = true;
+    if (tid == 0) arrived = mbar_wait_bounded(bar_a, 0, kWaitNs);
     if (__syncthreads_or(!arrived)) {
-        if (tid == 0) set_error(a.err, RSSM_DEVERR_TIMEOUT);
-        if (!arrived) mbar_wait_bounded(bar_a, 0, kWaitNs);
+        if (tid == 0) {
+            set_error(a.err, RSSM_DEVERR_TIMEOUT);
+            mbar_wait_bounded(bar_a, 0, kWaitNs);
+        }
         return;
     }
     if (!ok) return;
 
-    // h_ckpt . C_j for every row of the tile
-    for (int r0 = warp * rpw; r0 < P; r0 += kWarps * rpw) {
-        const int r = r0 + rsub;
-        const float4 hv = (r < P) ? tile_load4<RF>(s_tile, s_sc, r, col4, N) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-            if (j < ntok) {
-                const float d = group_sum(dot4(hv, c4[j]), lpr);
-                if (r < P && col4 == 0) s_hc[j * P + r] = d;
-            }
-        }
-    }
-    __syncthreads();
-
     const float Dh = a.D[h];
-    for (int i = tid; i < ntok * P; i += kThreads) {
-        const int j = i / P, p = i - j * P, t = pos + j;
-        float acc = s_decay[j] * s_hc[j * P + p];
-        for (int s = 0; s <= t; ++s) {
-            const float xs = (s < pos) ? to_f32(xb[(bh * cap + s) * P + p])
-                                       : to_f32(xin[((static_cast<size_t>(b) * ntok + (s - pos)) * H + h) * P + p]);
-            acc = fmaf(s_w[j][s] * s_g[j][s], xs, acc);
+    if constexpr (WIDE) {
+        // warp w owns rows r0..r0+7; lane l adds slot l's replay term to every row
+        for (int r0 = warp * 8; r0 < P; r0 += kWarps * 8) {
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                if (j < ntok) {
+                    const int t = pos + j;
+                    const float dec = s_decay[j];
+                    float part[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float4 hv = (r0 + k < P) ? tile_load4<RF>(s_tile, s_sc, r0 + k, lane, N)
+                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                        part[k] = dec * dot4(hv, c4[j]);
+                    }
+                    if (lane <= t) {
+                        const float coef = s_w[j][lane] * s_g[j][lane];
+                        const float4* xv = reinterpret_cast<const float4*>(s_x + lane * xs + r0);
+                        const float4 xa = xv[0], xc = xv[1];
+                        part[0] = fmaf(coef, xa.x, part[0]);
+                        part[1] = fmaf(coef, xa.y, part[1]);
+                        part[2] = fmaf(coef, xa.z, part[2]);
+                        part[3] = fmaf(coef, xa.w, part[3]);
+                        part[4] = fmaf(coef, xc.x, part[4]);
+                        part[5] = fmaf(coef, xc.y, part[5]);
+                        part[6] = fmaf(coef, xc.z, part[6]);
+                        part[7] = fmaf(coef, xc.w, part[7]);
+                    }
+                    const float z = warp_reduce8(part);
+                    const int r = r0 + ((lane >> 2) & 7);
+                    if ((lane & 3) == 0 && r < P) yout[j * HP + r] = fmaf(Dh, s_x[t * xs + r], z);
+                }
+            }
         }
-        const float xt = to_f32(xin[((static_cast<size_t>(b) * ntok + j) * H + h) * P + p]);
-        a.y[((static_cast<size_t>(b) * ntok + j) * H + h) * P + p] = fmaf(Dh, xt, acc);
+    } else {
+        for (int r0 = warp * rpw; r0 < P; r0 += kWarps * rpw) {
+            const int r = r0 + rsub;
+            const bool valid = r < P;
+            const float4 hv = valid ? tile_load4<RF>(s_tile, s_sc, r, col4, N) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                if (j < ntok) {
+                    const int t = pos + j;
+                    float part = s_decay[j] * dot4(hv, c4[j]);
+                    if (valid)
+                        for (int sl = col4; sl <= t; sl += lpr)
+                            part = fmaf(s_w[j][sl] * s_g[j][sl], s_x[sl * xs + r], part);
+                    const float sum = group_sum(part, lpr);
+                    if (valid && col4 == 0) yout[j * HP + r] = fmaf(Dh, s_x[t * xs + r], sum);
+                }
+            }
+        }
     }
 
-    if (!a.advance) return;
-    bool fold_now = false;
     if constexpr (RF == kF32 && NT == 1 && FUSED) {
-        fold_now = (T == a.s.L);
         if (fold_now) {
-            // fused flush: the token that fills the buffer also folds it into
-            // the checkpoint, reusing the tile already in shared memory.
-            for (int i = tid; i < T * P; i += kThreads) {
-                const int s = i / P, p = i - s * P;
-                const float xs = (s < pos) ? to_f32(xb[(bh * cap + s) * P + p])
-                                           : to_f32(xin[(static_cast<size_t>(b) * H + h) * P + p]);
-                s_xw[i] = s_w[0][s] * xs;
-            }
-            __syncthreads();
+            // fused flush: the token that fills the buffer folds it into the
+            // checkpoint from the tile, x rows and B rows already in shared memory.
             float* dst = a.ckpt_w + bh * P * N;
-            auto brow = [&](int s, int c) {
-                return (s < pos) ? load4(bb + ((static_cast<size_t>(b) * G + g) * cap + s) * N + 4 * c)
-                                 : load4(Bin + (static_cast<size_t>(b) * G + g) * N + 4 * c);
+            auto brow = [&](int sl, int c) {
+                const float w = s_w[0][sl];
+                const float4 v = reinterpret_cast<const float4*>(s_B + sl * N)[c];
+                return make_float4(w * v.x, w * v.y, w * v.z, w * v.w);
             };
             auto emit = [&](int r, int c, float4 v, bool valid) {
                 if (valid) stream_store4(dst + r * N + 4 * c, v);
             };
-            fold_rows(reinterpret_cast<float*>(s_tile), s_xw, P, N, lpr, T, s_decay[0], brow, emit);
+            fold_tile(reinterpret_cast<const float*>(s_tile), s_x, xs, P, N, lpr, T, s_decay[0], brow, emit);
         }
     }
+}
+
+// ---------------------------------------------------------------------------
+// Persistent, warp-specialised replay decode / verify for d_state 128 and
+// head_dim a multiple of 8. One CTA per SM walks the tiles
+// t = blockIdx.x + k * gridDim.x ((request, head) = (t / H, t % H)).
+// A producer warp reads each tile's position one tile ahead and brings all
+// of the tile's inputs into a ring of shared-memory stages with bulk copies
+// (the state tile, the buffered x and B rows, this call's x, B and C rows,
+// the dt row; completion on the stage's "full" mbarrier). Eight consumer
+// warps compute the outputs from shared memory only and release the stage
+// (its "empty" mbarrier). The HBM stream never waits for a tile's
+// arithmetic, and a tile's arithmetic never waits for HBM latency.
+// Every wait is bounded by %globaltimer; a timeout sets the error word.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t fdiv(uint32_t x, const FastDiv& f) { return (__umulhi(x, f.mul) + x) >> f.shr; }
+
+// Barrier of one consumer group (named barrier 1 + gi), returning the OR of v.
+__device__ __forceinline__ int group_sync_or(int gi, int v) {
+    int r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.s32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.s32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(v), "r"(1 + gi), "r"(kConsWarps * 32)
+        : "memory");
+    return r;
+}
+
+__device__ __forceinline__ void group_sync(int gi) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + gi), "r"(kConsWarps * 32) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Consumer groups of the pipelined kernel: two for decode, one for verify
+// (whose K+1 tokens need the registers).
+__host__ __device__ constexpr int pipe_groups(int nt) { return nt == 1 ? 2 : 1; }
+__host__ __device__ constexpr int pipe_threads(int nt) { return (pipe_groups(nt) * kConsWarps + 1) * 32; }
+
+template <typename TIn, int RF, int NT>
+__global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const ReplayArgs a, const PipeLayout lay) {
+    constexpr int CG = pipe_groups(NT);
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full_bar[kPipeStagesMax];
+    __shared__ __align__(8) uint64_t empty_bar[kPipeStagesMax];
+    __shared__ float s_w[CG][NT][kMaxCap];  // dt_s exp(A (S_t - S_s)) for token j; 0 for s > t
+    __shared__ float s_g[CG][NT][kMaxCap];  // B_s . C_j
+    __shared__ float s_decay[CG][NT];       // exp(A S_t)
+    __shared__ volatile int s_abort;
+
+    const int H = a.s.H, P = a.s.P, N = a.s.N, G = a.s.G, cap = a.s.cap, capr = a.s.capr;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int ntok = a.ntok, S = lay.stages;
+    const int ntiles = a.s.batch * H;
+    const size_t HP = static_cast<size_t>(H) * P, GN = static_cast<size_t>(G) * N;
+    constexpr int es = static_cast<int>(sizeof(TIn));
+    const uint32_t tb = tile_bytes(RF, P, N), sb = scale_bytes(RF, P, N);
+    (void)G;
+
+    if (tid == 0) {
+        for (int st = 0; st < S; ++st) {
+            mbar_init(smem_u32(&full_bar[st]), 1);
+            mbar_init(smem_u32(&empty_bar[st]), kConsWarps);
+        }
+        s_abort = 0;
+    }
     __syncthreads();
-    if (tid == 0) request_done(a.arrive, b, H, a.pos, fold_now ? 0 : pos + 1, a.flush_count, fold_now);
+
+    if (warp == CG * kConsWarps) {
+        // ------------------------------------------------------------ producer
+        // Lane i holds the position, dt, A and D of the i-th tile of the
+        // current batch of 32 tiles (and prefetches the next batch), so no
+        // load latency sits between two issues. Arrivals: lane 1 + k % 31
+        // adds tile k's arrival for its request and checks the returned
+        // count 31 tiles later; the request's last arrival moves pos.
+        int p0 = 0, p1 = 0;
+        float d0[NT], d1[NT], A0 = 0.f, A1 = 0.f, D0 = 0.f, D1 = 0.f;
+        auto fetch = [&](int kbase, int& pp, float (&dd)[NT], float& AA, float& DD) {
+            const uint32_t tt = blockIdx.x + static_cast<uint32_t>(kbase + lane) * gridDim.x;
+            if (tt < static_cast<uint32_t>(ntiles)) {
+                const int bb2 = fdiv(tt, lay.divH), hh2 = tt - bb2 * H;
+                pp = a.pos[bb2];
+#pragma unroll
+                for (int j = 0; j < NT; ++j)
+                    dd[j] = (j < ntok) ? a.dt[(static_cast<size_t>(bb2) * ntok + j) * H + hh2] : 0.f;
+                AA = a.A[hh2];
+                DD = a.D[hh2];
+            }
+        };
+        fetch(0, p0, d0, A0, D0);
+        fetch(32, p1, d1, A1, D1);
+        int pend_b = -1, pend_new = 0;
+        uint32_t pend_old = 0;
+        int k_issued = -1;  // last tile index issued
+        bool aborted = false;
+        for (int k = 0;; ++k) {
+            const uint32_t t = blockIdx.x + static_cast<uint32_t>(k) * gridDim.x;
+            if (t >= static_cast<uint32_t>(ntiles)) break;
+            const int b = fdiv(t, lay.divH), h = t - b * H, g = fdiv(h, lay.divHpg);
+            const bool cur = (k >> 5) & 1;
+            const int sel = k & 31;
+            if (sel == 0 && k > 0) {  // refill the other buffer with the batch after this one
+                if (cur)
+                    fetch(k + 32, p0, d0, A0, D0);
+                else
+                    fetch(k + 32, p1, d1, A1, D1);
+            }
+            // a uniform branch picks the batch, so the warp never reads the
+            // registers of the batch still being fetched
+            int pos;
+            float Ah, Dh, dtj[NT];
+            if (cur) {
+                pos = __shfl_sync(0xffffffffu, p1, sel);
+                Ah = __shfl_sync(0xffffffffu, A1, sel);
+                Dh = __shfl_sync(0xffffffffu, D1, sel);
+#pragma unroll
+                for (int j = 0; j < NT; ++j) dtj[j] = __shfl_sync(0xffffffffu, d1[j], sel);
+            } else {
+                pos = __shfl_sync(0xffffffffu, p0, sel);
+                Ah = __shfl_sync(0xffffffffu, A0, sel);
+                Dh = __shfl_sync(0xffffffffu, D0, sel);
+#pragma unroll
+                for (int j = 0; j < NT; ++j) dtj[j] = __shfl_sync(0xffffffffu, d0[j], sel);
+            }
+            const bool ok = pos >= 0 && pos + ntok <= cap;
+            if (a.advance && lane == 1 + (k % 31)) {
+                if (pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 1)) {
+                    a.arrive[pend_b] = 0u;
+                    a.pos[pend_b] = pend_new;
+                }
+                pend_b = -1;
+                if (ok) {
+                    pend_b = b;
+                    pend_new = pos + 1;
+                    pend_old = atomicAdd(&a.arrive[b], 1u);
+                }
+            }
+            const int st = k % S, use = k / S;
+            unsigned char* sp = smem + static_cast<size_t>(st) * lay.stage_bytes;
+            int live = 1;
+            if (lane == 0) {
+                if (use > 0 && !mbar_wait_bounded(smem_u32(&empty_bar[st]), (use - 1) & 1, kWaitNs)) {
+                    set_error(a.err, RSSM_DEVERR_TIMEOUT);
+                    s_abort = 1;
+                }
+                live = !s_abort;
+            }
+            live = __shfl_sync(0xffffffffu, live, 0);  // one decision for the whole warp
+            if (!live) {
+                aborted = true;
+                break;
+            }
+            const size_t bh = static_cast<size_t>(b) * H + h, bg = static_cast<size_t>(b) * G + g;
+            const uint32_t fb = smem_u32(&full_bar[st]);
+            if (lane == 0) {
+                float* meta = reinterpret_cast<float*>(sp + lay.dtnew);  // dt[8], then A, D
+#pragma unroll
+                for (int j = 0; j < NT; ++j)
+                    if (j < ntok) meta[j] = dtj[j];
+                meta[kMaxTok] = Ah;
+                meta[kMaxTok + 1] = Dh;
+                *reinterpret_cast<int*>(sp + lay.meta) = pos;
+                uint32_t bytes = tb + sb;
+                if (ok)
+                    bytes += static_cast<uint32_t>((pos + ntok) * P * es + (pos + ntok) * N * es + ntok * N * es +
+                                                   capr * 4);
+                mbar_expect_tx(fb, bytes);
+            }
+            __syncwarp();
+            // the tile's copies, one per lane, issued together:
+            // 0 tile, 1 FP4 scales, 2 buffered x rows, 3 buffered B rows, 4 dt row,
+            // then per token j: 5+3j x row, 6+3j B row, 7+3j C row
+            {
+                const void* src = nullptr;
+                uint32_t dst = 0, nb = 0;
+                if (lane == 0) {
+                    src = static_cast<const unsigned char*>(a.tile) + bh * tb;
+                    dst = smem_u32(sp + lay.tile);
+                    nb = tb;
+                } else if (lane == 1) {
+                    if (RF == kFP4) {
+                        src = a.tile_scales + bh * sb;
+                        dst = smem_u32(sp + lay.scales);
+                        nb = sb;
+                    }
+                } else if (ok) {
+                    if (lane == 2 && pos > 0) {
+                        src = static_cast<const TIn*>(a.xbuf) + bh * cap * P;
+                        dst = smem_u32(sp + lay.xrows);
+                        nb = pos * P * es;
+                    } else if (lane == 3 && pos > 0) {
+                        src = static_cast<const TIn*>(a.bbuf) + bg * cap * N;
+                        dst = smem_u32(sp + lay.brows);
+                        nb = pos * N * es;
+                    } else if (lane == 4) {
+                        src = a.dtbuf + bh * capr;
+                        dst = smem_u32(sp + lay.dtrow);
+                        nb = capr * 4;
+                    } else if (lane >= 5 && lane < 5 + 3 * ntok) {
+                        const int j = (lane - 5) / 3, w = (lane - 5) - 3 * j;
+                        const size_t bj = static_cast<size_t>(b) * ntok + j;
+                        if (w == 0) {
+                            src = static_cast<const TIn*>(a.x) + bj * HP + static_cast<size_t>(h) * P;
+                            dst = smem_u32(sp + lay.xrows + (pos + j) * P * es);
+                            nb = P * es;
+                        } else if (w == 1) {
+                            src = static_cast<const TIn*>(a.B) + bj * GN + static_cast<size_t>(g) * N;
+                            dst = smem_u32(sp + lay.brows + (pos + j) * N * es);
+                            nb = N * es;
+                        } else {
+                            src = static_cast<const TIn*>(a.C) + bj * GN + static_cast<size_t>(g) * N;
+                            dst = smem_u32(sp + lay.crows + j * N * es);
+                            nb = N * es;
+                        }
+                    }
+                }
+                if (nb > 0) bulk_g2s(dst, src, nb, fb);
+            }
+            k_issued = k;
+            __syncwarp();
+        }
+        // the arrivals still pending
+        if (a.advance && pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 1)) {
+            a.arrive[pend_b] = 0u;
+            a.pos[pend_b] = pend_new;
+        }
+        if (aborted && lane == 0) {
+            // let every copy this warp issued land before the CTA can exit:
+            // the last S tiles issued are the ones that may be in flight
+            for (int kk = k_issued; kk >= 0 && kk > k_issued - S; --kk)
+                mbar_wait_bounded(smem_u32(&full_bar[kk % S]), (kk / S) & 1, kWaitNs);
+        }
+        return;
+    }
+
+    // --------------------------------------------------------------- consumers
+    // Group gi takes tiles k = gi, gi + 2, ...; its 8 warps: warps 0..3 form
+    // the B.C products (8 slots each), warp 7 the decay weights, all of them
+    // 8 rows each of the output.
+    const int gi = warp / kConsWarps, cw = warp - gi * kConsWarps;
+    const int ctid = tid - gi * kConsWarps * 32;
+    const int hpg_shift_free = 0;
+    (void)hpg_shift_free;
+    for (int k = gi;; k += CG) {
+        const uint32_t t = blockIdx.x + static_cast<uint32_t>(k) * gridDim.x;
+        if (t >= static_cast<uint32_t>(ntiles)) break;
+        const int b = fdiv(t, lay.divH), h = t - b * H, g = fdiv(h, lay.divHpg);
+        const size_t bh = static_cast<size_t>(b) * H + h, bg = static_cast<size_t>(b) * G + g;
+        const int st = k % S, use = k / S;
+        const unsigned char* sp = smem + static_cast<size_t>(st) * lay.stage_bytes;
+        int stop = 0;
+        if (ctid == 0) {
+            stop = s_abort;
+            if (!stop && !mbar_wait_bounded(smem_u32(&full_bar[st]), use & 1, kWaitNs)) {
+                set_error(a.err, RSSM_DEVERR_TIMEOUT);
+                s_abort = 1;
+                stop = 1;
+                mbar_wait_bounded(smem_u32(&full_bar[st]), use & 1, kWaitNs);  // copies in flight
+            }
+        }
+        // the stage has landed; this group's previous readers of s_w / s_g are done
+        if (group_sync_or(gi, stop)) break;
+        const int pos = *reinterpret_cast<const int*>(sp + lay.meta);
+        const int T = pos + ntok;
+        const bool ok = pos >= 0 && T <= cap;
+        const TIn* xr = reinterpret_cast<const TIn*>(sp + lay.xrows);  // slot s row: xr + s*P
+        const TIn* br = reinterpret_cast<const TIn*>(sp + lay.brows);  // slot s row: br + s*N
+        const TIn* cr = reinterpret_cast<const TIn*>(sp + lay.crows);  // token j row: cr + j*N
+        const float* meta = reinterpret_cast<const float*>(sp + lay.dtnew);  // dt[8], A, D
+        float4 c4[NT];
+        if (!ok) {
+            if (ctid == 0) set_error(a.err, (pos < 0 || pos > cap) ? RSSM_DEVERR_POS_RANGE : RSSM_DEVERR_CAPACITY);
+        } else {
+#pragma unroll
+            for (int j = 0; j < NT; ++j)
+                c4[j] = (j < ntok) ? load4(cr + j * N + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (cw * 8 < T) {
+                // B_s . C_j for slots s0..s0+7, reduced together
+                const int s0 = cw * 8;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    if (j < ntok) {
+                        float part[8];
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            part[kk] = (s0 + kk < T) ? dot4(load4(br + (s0 + kk) * N + 4 * lane), c4[j]) : 0.f;
+                        const float z = warp_reduce8(part);
+                        const int sl = s0 + ((lane >> 2) & 7);
+                        if ((lane & 3) == 0 && sl < T) s_g[gi][j][sl] = z;
+                    }
+                }
+            }
+            if (cw == kConsWarps - 1) {
+                const float* dtrow = reinterpret_cast<const float*>(sp + lay.dtrow);
+                const float dnew = (lane >= pos && lane < T) ? meta[lane - pos] : 0.f;
+                const float dts = (lane < pos) ? dtrow[lane] : dnew;
+                if (lane >= pos && lane < T) a.dtbuf[bh * capr + lane] = dnew;
+                const float Sx = warp_prefix(dts);
+                const float Ah = meta[kMaxTok];
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    if (j < ntok) {
+                        const float St = __shfl_sync(0xffffffffu, Sx, pos + j);
+                        s_w[gi][j][lane] = (lane <= pos + j) ? dts * expf(Ah * (St - Sx)) : 0.f;
+                        if (lane == 0) s_decay[gi][j] = expf(Ah * St);
+                    }
+                }
+            }
+            if (cw == 4 || cw == 5) {
+                // append this call's x (and, for the group's first head, B) to the buffer
+                const int q0 = ctid - 4 * 32;  // 0..63
+                const int xq = (ntok * P * es) >> 4, bq = (ntok * N * es) >> 4;
+                for (int q = q0; q < xq; q += 64)
+                    reinterpret_cast<uint4*>(static_cast<TIn*>(a.xbuf) + (bh * cap + pos) * P)[q] =
+                        reinterpret_cast<const uint4*>(xr + pos * P)[q];
+                if (h == g * (H / G))
+                    for (int q = q0; q < bq; q += 64)
+                        reinterpret_cast<uint4*>(static_cast<TIn*>(a.bbuf) + (bg * cap + pos) * N)[q] =
+                            reinterpret_cast<const uint4*>(br + pos * N)[q];
+            }
+        }
+        group_sync(gi);  // s_w, s_g, s_decay ready
+        if (ok) {
+            const unsigned char* tile = sp + lay.tile;
+            const unsigned char* sc = sp + lay.scales;
+            const float Dh = meta[kMaxTok + 1];
+            float* yout = a.y + static_cast<size_t>(b) * ntok * HP + static_cast<size_t>(h) * P;
+            for (int r0 = cw * 8; r0 < P; r0 += kConsWarps * 8) {
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    if (j < ntok) {
+                        const int tt = pos + j;
+                        const float dec = s_decay[gi][j];
+                        float part[8];
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const float4 hv = (r0 + kk < P) ? tile_load4<RF>(tile, sc, r0 + kk, lane, N)
+                                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                            part[kk] = dec * dot4(hv, c4[j]);
+                        }
+                        if (lane <= tt) {
+                            const float coef = s_w[gi][j][lane] * s_g[gi][j][lane];
+                            Raw8<TIn> xv;
+                            xv.load(xr + lane * P + r0);
+                            const float4 xa = xv.lo(), xc = xv.hi();
+                            part[0] = fmaf(coef, xa.x, part[0]);
+                            part[1] = fmaf(coef, xa.y, part[1]);
+                            part[2] = fmaf(coef, xa.z, part[2]);
+                            part[3] = fmaf(coef, xa.w, part[3]);
+                            part[4] = fmaf(coef, xc.x, part[4]);
+                            part[5] = fmaf(coef, xc.y, part[5]);
+                            part[6] = fmaf(coef, xc.z, part[6]);
+                            part[7] = fmaf(coef, xc.w, part[7]);
+                        }
+                        const float z = warp_reduce8(part);
+                        const int r = r0 + ((lane >> 2) & 7);
+                        if ((lane & 3) == 0 && r < P) yout[j * HP + r] = fmaf(Dh, to_f32(xr[tt * P + r]), z);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -305,19 +853,46 @@ __global__ void __launch_bounds__(kThreads) k_replay(const ReplayArgs a) {
 // write the FP4 output copy from the fp32 result.
 // ---------------------------------------------------------------------------
 template <typename TIn, int UF, int OUT4>
-__global__ void __launch_bounds__(kThreads) k_fold(const FoldArgs a) {
+__global__ void __launch_bounds__(kThreads, 4) k_fold(const FoldArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t bar;
     __shared__ float s_cw[kMaxCap];
     __shared__ float s_alpha;
+    __shared__ int s_pos;
+    __shared__ uint32_t s_fc;
 
     const int H = a.s.H, P = a.s.P, N = a.s.N, G = a.s.G, cap = a.s.cap, lpr = a.s.lpr;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.x / H, h = blockIdx.x - b * H;
     const int g = h / (H / G);
+    const int xs = round_up8(P);
     const size_t bh = static_cast<size_t>(b) * H + h;
 
-    const int pos = a.pos[b];
+    const uint32_t tb = tile_bytes(UF, P, N), sb = scale_bytes(UF, P, N);
+    unsigned char* s_in = smem;
+    unsigned char* s_insc = smem + align16(tb);
+    unsigned char* after_in = smem + align16(tb) + align16(sb);
+    float* s32 = (UF == kF32) ? reinterpret_cast<float*>(s_in) : reinterpret_cast<float*>(after_in);
+    float* s_B = reinterpret_cast<float*>(after_in + (UF == kF32 ? 0u : 4u * P * N));  // [cap][N]
+    float* s_x = s_B + cap * N;                                                        // [cap][xs]
+    const uint32_t bar_a = smem_u32(&bar);
+
+    if (tid == 0) {
+        // the only reads of pos and flush_count: every thread uses these copies
+        const int p0 = a.pos[b];
+        s_pos = p0;
+        s_fc = a.flush_count[b];
+        const bool go0 = p0 >= 0 && p0 <= cap && ((p0 >= a.s.L) || (a.mode >= 1 && p0 > 0) || (a.mode == 2));
+        if (go0) {
+            mbar_init(bar_a, 1);
+            mbar_expect_tx(bar_a, tb + sb);
+            bulk_g2s(smem_u32(s_in), static_cast<const unsigned char*>(a.upd) + bh * tb, tb, bar_a);
+            if (UF == kFP4) bulk_g2s(smem_u32(s_insc), a.upd_scales + bh * sb, sb, bar_a);
+        }
+    }
+    __syncthreads();
+    const int pos = s_pos;
+    const uint32_t fc = s_fc;
     if (pos < 0 || pos > cap) {
         if (tid == 0) set_error(a.err, RSSM_DEVERR_POS_RANGE);
         return;
@@ -325,42 +900,51 @@ __global__ void __launch_bounds__(kThreads) k_fold(const FoldArgs a) {
     const bool go = (pos >= a.s.L) || (a.mode >= 1 && pos > 0) || (a.mode == 2);
     if (!go) return;
     const int T = pos;
-    const uint32_t fc = a.flush_count[b];
+    // past the barrier no thread of this CTA reads pos or flush_count again;
+    // once every CTA of the request has arrived, the last one resets them
+    if (tid == kThreads - 32) request_done(a.arrive, b, H, a.pos, 0, a.flush_count, true);
 
-    const uint32_t tb = tile_bytes(UF, P, N), sb = scale_bytes(UF, P, N);
-    unsigned char* s_in = smem;
-    unsigned char* s_insc = smem + align16(tb);
-    unsigned char* after_in = smem + align16(tb) + align16(sb);
-    float* s32 = (UF == kF32) ? reinterpret_cast<float*>(s_in) : reinterpret_cast<float*>(after_in);
-    float* s_xw = reinterpret_cast<float*>(after_in + (UF == kF32 ? 0u : 4u * P * N));  // [T][P]
-    const uint32_t bar_a = smem_u32(&bar);
-
-    if (tid == 0) {
-        mbar_init(bar_a, 1);
-        mbar_expect_tx(bar_a, tb + sb);
-        bulk_g2s(smem_u32(s_in), static_cast<const unsigned char*>(a.upd) + bh * tb, tb, bar_a);
-        if (UF == kFP4) bulk_g2s(smem_u32(s_insc), a.upd_scales + bh * sb, sb, bar_a);
-    }
+    const TIn* xb = static_cast<const TIn*>(a.xbuf);
+    const TIn* bb = static_cast<const TIn*>(a.bbuf);
     const float Ah = a.A[h];
+    // one round of independent loads: B rows, x rows (16-byte chunks when the
+    // rows allow it), dt
+    const TIn* bbg = bb + (static_cast<size_t>(b) * G + g) * cap * N;
+    const TIn* xbh = xb + bh * cap * P;
+    for (int q = tid; q < ((T * N) >> 3); q += kThreads) {
+        Raw8<TIn> r;
+        r.load(bbg + (q << 3));
+        reinterpret_cast<float4*>(s_B)[2 * q] = r.lo();
+        reinterpret_cast<float4*>(s_B)[2 * q + 1] = r.hi();
+    }
+    if ((P & 7) == 0) {
+        for (int q = tid; q < ((T * P) >> 3); q += kThreads) {
+            const int e = q << 3, sl = e / P, p = e - sl * P;
+            Raw8<TIn> r;
+            r.load(xbh + e);
+            float4* d = reinterpret_cast<float4*>(s_x + sl * xs + p);
+            d[0] = r.lo();
+            d[1] = r.hi();
+        }
+    } else {
+        for (int i = tid; i < T * P; i += kThreads) s_x[(i / P) * xs + (i % P)] = to_f32(xbh[i]);
+    }
     if (warp == 0) {
-        const float dts = (lane < T) ? a.dtbuf[bh * cap + lane] : 0.f;
+        const float dts = (lane < T) ? a.dtbuf[bh * a.s.capr + lane] : 0.f;
         const float Sx = warp_prefix(dts);
         const float Stot = T > 0 ? __shfl_sync(0xffffffffu, Sx, T - 1) : 0.f;
         s_cw[lane] = (lane < T) ? dts * expf(Ah * (Stot - Sx)) : 0.f;
         if (lane == 0) s_alpha = expf(Ah * Stot);
     }
-    __syncthreads();
-    const TIn* xb = static_cast<const TIn*>(a.xbuf);
-    const TIn* bb = static_cast<const TIn*>(a.bbuf);
-    for (int i = tid; i < T * P; i += kThreads) {
-        const int s = i / P, p = i - s * P;
-        s_xw[i] = s_cw[s] * to_f32(xb[(bh * cap + s) * P + p]);
-    }
 
-    const bool arrived = mbar_wait_bounded(bar_a, 0, kWaitNs);
+    // one thread waits for the tile; the barrier publishes it to the CTA
+    bool arrived = true;
+    if (tid == 0) arrived = mbar_wait_bounded(bar_a, 0, kWaitNs);
     if (__syncthreads_or(!arrived)) {
-        if (tid == 0) set_error(a.err, RSSM_DEVERR_TIMEOUT);
-        if (!arrived) mbar_wait_bounded(bar_a, 0, kWaitNs);
+        if (tid == 0) {
+            set_error(a.err, RSSM_DEVERR_TIMEOUT);
+            mbar_wait_bounded(bar_a, 0, kWaitNs);
+        }
         return;
     }
     if constexpr (UF != kF32) {
@@ -372,18 +956,22 @@ __global__ void __launch_bounds__(kThreads) k_fold(const FoldArgs a) {
         __syncthreads();
     }
 
-    auto brow = [&](int s, int c) { return load4(bb + ((static_cast<size_t>(b) * G + g) * cap + s) * N + 4 * c); };
+    auto brow = [&](int s, int c) {
+        const float w = s_cw[s];
+        const float4 v = reinterpret_cast<const float4*>(s_B + s * N)[c];
+        return make_float4(w * v.x, w * v.y, w * v.z, w * v.w);
+    };
     auto emit = [&](int r, int c, float4 v, bool valid) {
         const size_t e = (bh * P + r) * N + 4 * c;  // flat element index of v.x
         if constexpr (UF == kF32) {
             if (valid) stream_store4(static_cast<float*>(a.upd) + e, v);
         } else if constexpr (UF == kBF16 || UF == kE4M3) {
-            // Philox counter (e/4, head, request, flush_count), e within the head
-            const uint32_t e_head = static_cast<uint32_t>(r * N + 4 * c);
-            const uint4 rw = philox4x32_10(make_uint4(e_head >> 2, h, b, fc),
-                                           make_uint2(static_cast<uint32_t>(a.seed),
-                                                      static_cast<uint32_t>(a.seed >> 32)));
             if (valid) {
+                // Philox counter (e/4, head, request, flush_count), e within the head
+                const uint32_t e_head = static_cast<uint32_t>(r * N + 4 * c);
+                const uint4 rw = philox4x32_10(make_uint4(e_head >> 2, h, b, fc),
+                                               make_uint2(static_cast<uint32_t>(a.seed),
+                                                          static_cast<uint32_t>(a.seed >> 32)));
                 if constexpr (UF == kBF16) {
                     const uint2 w = make_uint2(sr_bf16(v.x, rw.x) | (sr_bf16(v.y, rw.y) << 16),
                                                sr_bf16(v.z, rw.z) | (sr_bf16(v.w, rw.w) << 16));
@@ -411,9 +999,7 @@ __global__ void __launch_bounds__(kThreads) k_fold(const FoldArgs a) {
             }
         }
     };
-    fold_rows(s32, s_xw, P, N, lpr, T, s_alpha, brow, emit);
-    __syncthreads();
-    if (tid == 0) request_done(a.arrive, b, H, a.pos, 0, a.flush_count, true);
+    fold_tile(s32, s_x, xs, P, N, lpr, T, s_alpha, brow, emit);
 }
 
 // ---------------------------------------------------------------------------
@@ -422,7 +1008,7 @@ __global__ void __launch_bounds__(kThreads) k_fold(const FoldArgs a) {
 // VERIFY: read copy cur[b], write the state after token j to copy j.
 // ---------------------------------------------------------------------------
 template <typename TIn, int NT, int VERIFY>
-__global__ void __launch_bounds__(kThreads) k_conv(const ConvArgs a) {
+__global__ void __launch_bounds__(kThreads, VERIFY ? (NT <= kMidTok ? 3 : 2) : 6) k_conv(const ConvArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t bar;
 
@@ -467,11 +1053,14 @@ __global__ void __launch_bounds__(kThreads) k_conv(const ConvArgs a) {
         aj[j] = expf(dtj[j] * Ah);
     }
     const float Dh = a.D[h];
-    __syncthreads();
-    const bool arrived = mbar_wait_bounded(bar_a, 0, kWaitNs);
+    // one thread waits for the tile; the barrier publishes it to the CTA
+    bool arrived = true;
+    if (tid == 0) arrived = mbar_wait_bounded(bar_a, 0, kWaitNs);
     if (__syncthreads_or(!arrived)) {
-        if (tid == 0) set_error(a.err, RSSM_DEVERR_TIMEOUT);
-        if (!arrived) mbar_wait_bounded(bar_a, 0, kWaitNs);
+        if (tid == 0) {
+            set_error(a.err, RSSM_DEVERR_TIMEOUT);
+            mbar_wait_bounded(bar_a, 0, kWaitNs);
+        }
         return;
     }
     const float4* s_tile = reinterpret_cast<const float4*>(smem);
@@ -523,17 +1112,21 @@ __global__ void k_accept(int batch, int K, int cap, const int32_t* n, int32_t* p
 __global__ void k_round_test(int op, int64_t n, const float* v, uint64_t seed, uint32_t c1, uint32_t c2,
                              uint32_t c3, void* out) {
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (op == 3) {
+    if (op == 3 || op == 5) {
         // one lane per 4 values; quads of lanes make one 16-value block
         const int64_t q = i;  // group of 4 values
         const bool valid = 4 * q < n;
         const float4 x = valid ? reinterpret_cast<const float4*>(v)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
         uint32_t sc;
         const uint32_t codes = fp4_quant_quad(x, &sc);
-        if (valid) {
+        if (valid && op == 3) {
             uint8_t* o = static_cast<uint8_t*>(out);
             *reinterpret_cast<uint16_t*>(o + 2 * q) = static_cast<uint16_t>(codes);
             if ((q & 3) == 0) o[n / 2 + q / 4] = static_cast<uint8_t>(sc);
+        }
+        if (valid && op == 5) {
+            // the decode the FP4-reading kernels use
+            reinterpret_cast<float4*>(out)[q] = fp4x4_val(codes, e4m3_val(sc) * 16384.0f);
         }
         return;
     }
@@ -552,16 +1145,18 @@ __global__ void k_round_test(int op, int64_t n, const float* v, uint64_t seed, u
 // ------------------------------------------------------------------ host
 
 size_t replay_smem_bytes(const Shape& s, int rf, int ntok, int fused) {
+    (void)ntok;
     size_t b = align16(tile_bytes(rf, s.P, s.N)) + align16(scale_bytes(rf, s.P, s.N));
-    b += 4u * static_cast<size_t>((ntok * s.P + 3) & ~3);
-    if (fused) b += 4u * static_cast<size_t>(s.L) * s.P;
+    b += 4u * static_cast<size_t>(s.cap) * round_up8(s.P);
+    if (fused) b += 4u * static_cast<size_t>(s.L) * s.N;
     return b;
 }
 
 size_t fold_smem_bytes(const Shape& s, int uf) {
     size_t b = align16(tile_bytes(uf, s.P, s.N)) + align16(scale_bytes(uf, s.P, s.N));
     if (uf != kF32) b += 4u * static_cast<size_t>(s.P) * s.N;
-    b += 4u * static_cast<size_t>(s.cap) * s.P;
+    b += 4u * static_cast<size_t>(s.cap) * s.N;
+    b += 4u * static_cast<size_t>(s.cap) * round_up8(s.P);
     return b;
 }
 
@@ -575,30 +1170,144 @@ static cudaError_t launch_tiles(K kernel, const Args& a, int nblk, size_t smem, 
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
+    // all of the unified L1/shared array as shared memory: the tiles are
+    // staged there and the occupancy is bounded by it
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         static_cast<int>(cudaSharedmemCarveoutMaxShared));
+    if (e != cudaSuccess) return e;
     kernel<<<nblk, kThreads, smem, st>>>(a);
     return cudaGetLastError();
 }
 
-template <typename TIn, int NT>
+template <typename K, typename... Args>
+static cudaError_t launch_grid(K kernel, const ReplayArgs& a, const PipeLayout& L, int grid, int threads,
+                               size_t smem, cudaStream_t st) {
+    if (grid <= 0) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             static_cast<int>(cudaSharedmemCarveoutMaxShared));
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, threads, smem, st>>>(a, L);
+    return cudaGetLastError();
+}
+
+template <typename TIn, int NT, int W>
 static cudaError_t replay_dispatch_fmt(const ReplayArgs& a, int rf, size_t smem, int nblk, cudaStream_t st) {
     switch (rf) {
         case kF32:
-            if (NT == 1 && a.fused) return launch_tiles(k_replay<TIn, kF32, NT, 1>, a, nblk, smem, st);
-            return launch_tiles(k_replay<TIn, kF32, NT, 0>, a, nblk, smem, st);
-        case kBF16: return launch_tiles(k_replay<TIn, kBF16, NT, 0>, a, nblk, smem, st);
-        case kE4M3: return launch_tiles(k_replay<TIn, kE4M3, NT, 0>, a, nblk, smem, st);
-        default: return launch_tiles(k_replay<TIn, kFP4, NT, 0>, a, nblk, smem, st);
+            if constexpr (NT == 1) {
+                if (a.fused) return launch_tiles(k_replay<TIn, kF32, NT, 1, W>, a, nblk, smem, st);
+            }
+            return launch_tiles(k_replay<TIn, kF32, NT, 0, W>, a, nblk, smem, st);
+        case kBF16: return launch_tiles(k_replay<TIn, kBF16, NT, 0, W>, a, nblk, smem, st);
+        case kE4M3: return launch_tiles(k_replay<TIn, kE4M3, NT, 0, W>, a, nblk, smem, st);
+        default: return launch_tiles(k_replay<TIn, kFP4, NT, 0, W>, a, nblk, smem, st);
     }
 }
 
+template <typename TIn, int NT>
+static cudaError_t replay_dispatch_wide(const ReplayArgs& a, int rf, size_t smem, int nblk, cudaStream_t st) {
+    const bool wide = a.s.N == 128 && a.s.P % 8 == 0;
+    return wide ? replay_dispatch_fmt<TIn, NT, 1>(a, rf, smem, nblk, st)
+                : replay_dispatch_fmt<TIn, NT, 0>(a, rf, smem, nblk, st);
+}
+
+// Stage layout of k_replay_pipe (16-byte aligned pieces, 128-byte aligned stages).
+PipeLayout pipe_layout(const Shape& s, int rf, int ntok, int in_bf16, size_t smem_budget) {
+    const uint32_t es = in_bf16 ? 2u : 4u;
+    PipeLayout L;
+    uint32_t off = 0;
+    L.tile = off;
+    off += align16(tile_bytes(rf, s.P, s.N));
+    L.scales = off;
+    off += align16(scale_bytes(rf, s.P, s.N));
+    L.xrows = off;
+    off += align16(static_cast<uint32_t>(s.cap * s.P) * es);
+    L.brows = off;
+    off += align16(static_cast<uint32_t>(s.cap * s.N) * es);
+    L.crows = off;
+    off += align16(static_cast<uint32_t>(ntok * s.N) * es);
+    L.dtrow = off;
+    off += align16(static_cast<uint32_t>(s.capr) * 4u);
+    L.dtnew = off;  // this call's dt [kMaxTok], then A_h and D_h
+    off += 4u * kMaxTok + 16u;
+    L.meta = off;
+    off += 16u;
+    L.stage_bytes = (off + 127u) & ~127u;
+    const size_t n = smem_budget / L.stage_bytes;
+    L.stages = static_cast<int>(n < static_cast<size_t>(kPipeStagesMax) ? n : kPipeStagesMax);
+    L.divH = make_fastdiv(static_cast<uint32_t>(s.H));
+    L.divHpg = make_fastdiv(static_cast<uint32_t>(s.H / s.G));
+    return L;
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    size_t smem_optin = 0;
+};
+
+static DeviceInfo device_info() {
+    static DeviceInfo cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DeviceInfo{};
+    if (cache[dev].sms == 0) {
+        int sms = 0, optin = 0;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        cache[dev].smem_optin = static_cast<size_t>(optin);
+        cache[dev].sms = sms;
+    }
+    return cache[dev];
+}
+
+template <typename TIn, int NT>
+static cudaError_t pipe_dispatch(const ReplayArgs& a, const PipeLayout& L, int rf, int grid, cudaStream_t st) {
+    const size_t smem = static_cast<size_t>(L.stages) * L.stage_bytes;
+    constexpr int thr = pipe_threads(NT);
+    switch (rf) {
+        case kF32: return launch_grid(k_replay_pipe<TIn, kF32, NT>, a, L, grid, thr, smem, st);
+        case kBF16: return launch_grid(k_replay_pipe<TIn, kBF16, NT>, a, L, grid, thr, smem, st);
+        case kE4M3: return launch_grid(k_replay_pipe<TIn, kE4M3, NT>, a, L, grid, thr, smem, st);
+        default: return launch_grid(k_replay_pipe<TIn, kFP4, NT>, a, L, grid, thr, smem, st);
+    }
+}
+
+static cudaError_t launch_replay_pipe(const ReplayArgs& a, int in_bf16, int rf, const PipeLayout& L, int grid,
+                                      cudaStream_t st) {
+    if (a.ntok == 1)
+        return in_bf16 ? pipe_dispatch<__nv_bfloat16, 1>(a, L, rf, grid, st) : pipe_dispatch<float, 1>(a, L, rf, grid, st);
+    if (a.ntok <= kMidTok)
+        return in_bf16 ? pipe_dispatch<__nv_bfloat16, kMidTok>(a, L, rf, grid, st)
+                       : pipe_dispatch<float, kMidTok>(a, L, rf, grid, st);
+    return in_bf16 ? pipe_dispatch<__nv_bfloat16, kMaxTok>(a, L, rf, grid, st)
+                   : pipe_dispatch<float, kMaxTok>(a, L, rf, grid, st);
+}
+
 cudaError_t launch_replay(const ReplayArgs& a, int in_bf16, int rf, cudaStream_t st) {
+    // the pipelined kernel serves d_state 128 with head_dim a multiple of 8
+    if (!a.fused && a.s.N == 128 && a.s.P % 8 == 0) {
+        const DeviceInfo di = device_info();
+        if (di.sms > 0) {
+            const size_t budget = di.smem_optin > 4096 ? di.smem_optin - 4096 : 0;
+            const PipeLayout L = pipe_layout(a.s, rf, a.ntok, in_bf16, budget);
+            if (L.stages >= 2) {
+                const int ntiles = a.s.batch * a.s.H;
+                const int grid = ntiles < di.sms ? ntiles : di.sms;
+                return launch_replay_pipe(a, in_bf16, rf, L, grid, st);
+            }
+        }
+    }
     const size_t smem = replay_smem_bytes(a.s, rf, a.ntok, a.fused);
     const int nblk = a.s.batch * a.s.H;
     if (a.ntok == 1)
-        return in_bf16 ? replay_dispatch_fmt<__nv_bfloat16, 1>(a, rf, smem, nblk, st)
-                       : replay_dispatch_fmt<float, 1>(a, rf, smem, nblk, st);
-    return in_bf16 ? replay_dispatch_fmt<__nv_bfloat16, kMaxTok>(a, rf, smem, nblk, st)
-                   : replay_dispatch_fmt<float, kMaxTok>(a, rf, smem, nblk, st);
+        return in_bf16 ? replay_dispatch_wide<__nv_bfloat16, 1>(a, rf, smem, nblk, st)
+                       : replay_dispatch_wide<float, 1>(a, rf, smem, nblk, st);
+    if (a.ntok <= kMidTok)
+        return in_bf16 ? replay_dispatch_wide<__nv_bfloat16, kMidTok>(a, rf, smem, nblk, st)
+                       : replay_dispatch_wide<float, kMidTok>(a, rf, smem, nblk, st);
+    return in_bf16 ? replay_dispatch_wide<__nv_bfloat16, kMaxTok>(a, rf, smem, nblk, st)
+                   : replay_dispatch_wide<float, kMaxTok>(a, rf, smem, nblk, st);
 }
 
 template <typename TIn>
@@ -631,6 +1340,9 @@ cudaError_t launch_conv(const ConvArgs& a, int in_bf16, int verify, cudaStream_t
     if (!verify)
         return in_bf16 ? launch_tiles(k_conv<__nv_bfloat16, 1, 0>, a, nblk, smem, st)
                        : launch_tiles(k_conv<float, 1, 0>, a, nblk, smem, st);
+    if (a.ntok <= kMidTok)
+        return in_bf16 ? launch_tiles(k_conv<__nv_bfloat16, kMidTok, 1>, a, nblk, smem, st)
+                       : launch_tiles(k_conv<float, kMidTok, 1>, a, nblk, smem, st);
     return in_bf16 ? launch_tiles(k_conv<__nv_bfloat16, kMaxTok, 1>, a, nblk, smem, st)
                    : launch_tiles(k_conv<float, kMaxTok, 1>, a, nblk, smem, st);
 }
@@ -645,7 +1357,7 @@ cudaError_t launch_accept(int batch, int K, int cap, const int32_t* n, int32_t* 
 cudaError_t launch_round_test(int op, int64_t n, const float* v, uint64_t seed, uint32_t c1, uint32_t c2,
                               uint32_t c3, void* out, cudaStream_t st) {
     if (n <= 0) return cudaSuccess;
-    const int64_t items = (op == 3) ? n / 4 : n;
+    const int64_t items = (op == 3 || op == 5) ? n / 4 : n;
     const int64_t blocks = (items + 255) / 256;
     k_round_test<<<static_cast<unsigned>(blocks), 256, 0, st>>>(op, n, v, seed, c1, c2, c3, out);
     return cudaGetLastError();

@@ -135,7 +135,8 @@ class RssmState:
 
     Views: ckpt (the update copy: float32 / bfloat16 / uint8 e4m3 / uint8 FP4
     codes, [batch][H][P][N or N/2]), ckpt_scales, out_codes, out_scales,
-    xbuf [batch][H][cap][P], bbuf [batch][G][cap][N], dtbuf [batch][H][cap],
+    xbuf [batch][H][cap][P], bbuf [batch][G][cap][N], dtbuf [batch][H][capr]
+    (capr = cap rounded up to a multiple of 4),
     pos, flush_count, arrive, err. Counters and buffers start at zero."""
 
     def __init__(self, desc, device=None):
@@ -145,6 +146,7 @@ class RssmState:
         B, H, P, N, G = desc.batch, desc.nheads, desc.head_dim, desc.d_state, desc.ngroups
         cap = desc.interval + desc.max_draft
         self.cap = cap
+        capr = (cap + 3) // 4 * 4
         in_dt = _IN_DT[desc.in_dtype]
 
         def field(f, shape, dtype):
@@ -162,7 +164,7 @@ class RssmState:
         self.out_scales = field(FIELD_OUT_SCALES, (B, H, P, N // 16), torch.uint8)
         self.xbuf = field(FIELD_XBUF, (B, H, cap, P), in_dt)
         self.bbuf = field(FIELD_BBUF, (B, G, cap, N), in_dt)
-        self.dtbuf = field(FIELD_DTBUF, (B, H, cap), torch.float32)
+        self.dtbuf = field(FIELD_DTBUF, (B, H, capr), torch.float32)
         self.pos = field(FIELD_POS, (B,), torch.int32)
         self.flush_count = field(FIELD_FLUSH_COUNT, (B,), torch.int32)
         self.arrive = field(FIELD_ARRIVE, (B,), torch.int32)
@@ -249,6 +251,8 @@ def rssm_round_test(op, v, seed=0, c1=0, c2=0, c3=0, stream=None):
         out = torch.empty(n, dtype=torch.uint8, device=v.device)
     elif op == 3:
         out = torch.empty(n // 2 + n // 16, dtype=torch.uint8, device=v.device)
+    elif op == 5:
+        out = torch.empty(n, dtype=torch.float32, device=v.device)
     else:
         out = torch.empty(n, dtype=torch.int32, device=v.device)
     _check(lib().rssm_round_test(int(op), n, _ptr(v, torch.float32, "v"), int(seed), int(c1), int(c2), int(c3),

@@ -116,7 +116,8 @@ typedef enum rssm_field {
     RSSM_FIELD_OUT_SCALES,     /* FP4 output copy: e4m3 [batch][H][P][N/16] */
     RSSM_FIELD_XBUF,           /* buffered x  [batch][H][Cap][P] in in_dtype */
     RSSM_FIELD_BBUF,           /* buffered B  [batch][G][Cap][N] in in_dtype */
-    RSSM_FIELD_DTBUF,          /* buffered dt [batch][H][Cap] float */
+    RSSM_FIELD_DTBUF,          /* buffered dt [batch][H][CapR] float, CapR = Cap rounded
+                                  up to a multiple of 4 (16-byte rows) */
     RSSM_FIELD_POS,            /* int32 [batch]: valid buffer length */
     RSSM_FIELD_FLUSH_COUNT,    /* uint32 [batch]: refreshes so far (Philox counter word) */
     RSSM_FIELD_ARRIVE,         /* uint32 [batch]: scratch, must be zero before first use;
@@ -249,7 +250,9 @@ RSSM_API rssm_status_t rssm_get_error(const rssm_desc_t *desc, const rssm_state_
  *   op 2: e4m3 nearest-even, saturating -> uint8 out[n]
  *   op 3: FP4 block copy  -> uint8 out[n/2] codes, then uint8 out[n/2 + n/16] scales
  *   op 4: Philox word e%4 at (e/4, c1, c2, c3)  -> uint32 out[n]
- * n must be a multiple of 16 for op 3. */
+ *   op 5: FP4 block copy, then decoded the way FP4-reading kernels decode it
+ *         -> float out[n]
+ * n must be a multiple of 16 for ops 3 and 5. */
 RSSM_API rssm_status_t rssm_round_test(int32_t op, int64_t n, const float *v, uint64_t seed, uint32_t c1,
                               uint32_t c2, uint32_t c3, void *out, void *stream);
 

@@ -65,6 +65,7 @@ def test_field_bytes():
     assert fb(rssm.FIELD_XBUF) == 256 * 64 * 16 * 64 * 2
     assert fb(rssm.FIELD_BBUF) == 256 * 8 * 16 * 128 * 2
     assert fb(rssm.FIELD_DTBUF) == 256 * 64 * 16 * 4
+    assert rssm.rssm_state_field_bytes(cfg(max_draft=1), rssm.FIELD_DTBUF) == 256 * 64 * 20 * 4
     assert fb(rssm.FIELD_POS) == fb(rssm.FIELD_ARRIVE) == 1024 and fb(rssm.FIELD_ERR) == 4
     s = cfg(update_dtype=rssm.RSSM_BF16, out_copy=rssm.RSSM_OUTCOPY_FP4, max_draft=4)
     fs = lambda f: rssm.rssm_state_field_bytes(s, f)

@@ -82,28 +82,30 @@ def test_refresh_at_empty_buffer_builds_fp4_copy_bit_exact(kind):
     assert rssm.rssm_get_error(st) == 0
 
 
-def neighbour_steps(got, ref, kind):
-    """Distance in representable steps between two copies' bit patterns."""
+def copy_values(bits, kind):
+    return orc.widen(UPD[kind][1], np.ascontiguousarray(bits).ravel())
+
+
+def spacing(v, kind):
+    """Distance to the next representable magnitude above |v| (bf16 or e4m3)."""
+    a = np.abs(np.asarray(v, np.float64))
     if kind == "bf16":
-        g = got.astype(np.int64)
-        r = ref.astype(np.int64)
-        gs = np.where(g & 0x8000, -(g & 0x7FFF), g)
-        rs = np.where(r & 0x8000, -(r & 0x7FFF), r)
-        return np.abs(gs - rs)
-    g = got.astype(np.int64)
-    r = ref.astype(np.int64)
-    gs = np.where(g & 0x80, -(g & 0x7F), g)
-    rs = np.where(r & 0x80, -(r & 0x7F), r)
-    return np.abs(gs - rs)
+        e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+        return np.exp2(e - 7)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -6)))
+    return np.exp2(e - 3)
 
 
 @pytest.mark.parametrize("kind", ["bf16", "e4m3"])
 def test_fp4_decode_and_refresh_match_oracle(kind):
     """One interval from a prepared split state: every output read from the
-    FP4 copy matches the oracle (fp32 vs fp64 on exact dequantised values);
-    the refreshed update copy and FP4 copy match the oracle bit for bit
-    except where the fp32 fold differs from the rounded fp64 fold right at a
-    rounding threshold, and then only by one representable step."""
+    FP4 copy matches the oracle (fp32 vs fp64 on exact dequantised values).
+    The refreshed update copy and FP4 copy match the oracle bit for bit
+    except where the fp32 fold (GPU) and the fp64 fold rounded to fp32
+    (oracle) straddle a rounding threshold: at least 99.9% of the elements
+    agree exactly, and every element of the update copy lies within one
+    spacing of the oracle's unrounded value plus the fp32 fold error
+    (1e-5 rms of the state)."""
     shape = LayerShape(4, 8, 64, 128, 2)
     L = shape.interval
     inp = make_inputs(shape, L, 31, torch.bfloat16, device="cuda")
@@ -125,11 +127,12 @@ def test_fp4_decode_and_refresh_match_oracle(kind):
         req.flush_count.value = 1
         ys = np.stack([req.decode(r["x"][t], r["B"][t], r["C"][t], r["dt"][t]) for t in range(L)])
         assert_close(to_np(y[:, b]), ys, f"FP4-copy decode, request {b}")
-        req.refresh()
-        got_upd = copy_bits(st.ckpt[b])
-        steps = neighbour_steps(got_upd.ravel(), req.upd.ravel(), kind)
-        assert steps.max() <= 1
-        mism_upd += int(np.count_nonzero(steps))
+        v32 = req.refresh(want_v32=True).astype(np.float64).ravel()
+        got_upd = copy_bits(st.ckpt[b]).ravel()
+        mism_upd += int(np.count_nonzero(got_upd != req.upd.ravel()))
+        err = np.abs(copy_values(got_upd, kind) - v32)
+        bound = spacing(v32, kind) + 1e-5 * np.sqrt(np.mean(v32 ** 2))
+        assert np.all(err <= bound), float(np.max(err - bound))
         gc = st.out_codes[b].cpu().numpy().ravel()
         mism_codes += int(np.count_nonzero(gc != req.codes.ravel()))
         total += gc.size

@@ -178,8 +178,10 @@ def small_state(shape=LayerShape(4, 4, 32, 64, 2, interval=16, max_draft=2)):
     return shape, inp, desc, st
 
 
-def test_device_error_bad_pos_is_reported_and_contained():
-    shape, inp, desc, st = small_state()
+@pytest.mark.parametrize("d_state", [64, 128])
+def test_device_error_bad_pos_is_reported_and_contained(d_state):
+    """d_state 128 runs the pipelined kernel, 64 the per-tile kernel."""
+    shape, inp, desc, st = small_state(LayerShape(4, 4, 32, d_state, 2, interval=16, max_draft=2))
     y = torch.full((4, 4, 32), 7.0, device="cuda")
     st.pos[2] = 99
     rssm.rssm_decode_step(st, inp["x"][0], inp["B"][0], inp["C"][0], inp["dt"][0], inp["A"], inp["D"], y)
@@ -191,8 +193,9 @@ def test_device_error_bad_pos_is_reported_and_contained():
     assert set(st.arrive.cpu().tolist()) == {0}
 
 
-def test_device_error_capacity_and_accept_range():
-    shape, inp, desc, st = small_state()
+@pytest.mark.parametrize("d_state", [64, 128])
+def test_device_error_capacity_and_accept_range(d_state):
+    shape, inp, desc, st = small_state(LayerShape(4, 4, 32, d_state, 2, interval=16, max_draft=2))
     K = 2
     vi = make_inputs(shape, 1, 4, torch.bfloat16, device="cuda", ntok=K + 1)
     y = torch.empty((4, K + 1, 4, 32), device="cuda")

@@ -98,3 +98,16 @@ def test_fp4_block_copy_bit_exact():
     assert np.array_equal(got[n // 2:], scales), "scales differ"
     bad = np.nonzero(got[: n // 2] != codes)[0]
     assert bad.size == 0, [(i, hex(got[i]), hex(codes[i]), v[2 * i:2 * i + 2]) for i in bad[:10]]
+
+
+def test_fp4_read_path_decodes_exactly():
+    """The FP4 decode of the replay and refresh kernels, applied to the
+    kernels' own FP4 copy, gives exactly the oracle's dequantised values."""
+    rng = np.random.default_rng(4)
+    blocks = (rng.normal(0, 1, (1 << 14, 16)) * np.exp2(rng.uniform(-12, 8, (1 << 14, 1)))).astype(np.float32)
+    v = np.concatenate([fp4_tie_blocks(), blocks.ravel()]).astype(np.float32)
+    got = rssm.rssm_round_test(5, torch.from_numpy(v).cuda()).cpu().numpy()
+    codes, scales = orc.fp4_quant(v)
+    ref = orc.widen(orc.FP4, codes, scales)
+    assert np.array_equal(got.astype(np.float64), ref)
+    assert np.array_equal(np.signbit(got), np.signbit(ref))
