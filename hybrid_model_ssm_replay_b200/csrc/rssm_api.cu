@@ -174,6 +174,29 @@ rssm_status_t rssm_decode_step(const rssm_desc_t* d, const rssm_state_t* st, con
     return replay_call(d, st, 1, 1, x, B, C, dt, A, D, y, stream);
 }
 
+rssm_status_t rssm_decode_step_noalloc(const rssm_desc_t* d, const rssm_state_t* st, const void* x, const void* B,
+                                       const void* C, const float* dt, const float* A, const float* D, float* y,
+                                       void* stream) {
+    rssm_status_t s = rssm_check_desc(d);
+    if (s != RSSM_OK) return s;
+    if (d->batch > RSSM_NOALLOC_MAX_BATCH) return RSSM_ERR_CAPACITY;
+    if (!st || !st->ckpt || !st->xbuf || !st->bbuf || !st->dtbuf || !st->pos || !st->flush_count || !st->err)
+        return RSSM_ERR_INVALID_ARG;
+    if (fp4_needs_scales(d) && !st->ckpt_scales) return RSSM_ERR_INVALID_ARG;
+    if (d->out_copy == RSSM_OUTCOPY_FP4 && (!st->out_codes || !st->out_scales)) return RSSM_ERR_INVALID_ARG;
+    if (!x || !B || !C || !dt || !A || !D || !y) return RSSM_ERR_INVALID_ARG;
+    uint32_t* scratch = noalloc_arrive_scratch();
+    if (!scratch) return RSSM_ERR_CUDA;
+    // the counters must start at zero; a previous call that stopped on a
+    // device error may have left some set
+    cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(uint32_t) * static_cast<size_t>(d->batch),
+                                    static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return RSSM_ERR_CUDA;
+    rssm_state_t view = *st;
+    view.arrive = scratch;
+    return replay_call(d, &view, 1, 1, x, B, C, dt, A, D, y, stream);
+}
+
 rssm_status_t rssm_verify(const rssm_desc_t* d, const rssm_state_t* st, int32_t K, const void* x, const void* B,
                           const void* C, const float* dt, const float* A, const float* D, float* y,
                           void* stream) {

@@ -111,6 +111,9 @@ cudaError_t launch_accept(int batch, int K, int cap, const int32_t* n, int32_t* 
 cudaError_t launch_round_test(int op, int64_t n, const float* v, uint64_t seed, uint32_t c1, uint32_t c2,
                               uint32_t c3, void* out, cudaStream_t st);
 
+// Scratch of the no-allocation decode entry point (see rssm.h).
+uint32_t* noalloc_arrive_scratch();
+
 // Dynamic shared memory of one CTA, in bytes.
 size_t replay_smem_bytes(const Shape& s, int read_fmt, int ntok, int fused);
 size_t fold_smem_bytes(const Shape& s, int upd_fmt);

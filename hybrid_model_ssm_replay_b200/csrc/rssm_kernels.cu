@@ -1142,6 +1142,25 @@ __global__ void k_round_test(int op, int64_t n, const float* v, uint64_t seed, u
     }
 }
 
+// ------------------------------------------------- no-allocation scratch
+// Arrival counters for rssm_decode_step_noalloc: one uint32 per request,
+// resident on every GPU that loads the library (256 KiB) until exit.
+static __device__ __align__(256) uint32_t g_noalloc_arrive[RSSM_NOALLOC_MAX_BATCH];
+
+// Device address of g_noalloc_arrive on the current device, looked up once
+// per device (cudaGetSymbolAddress) and cached. nullptr when the lookup fails.
+uint32_t* noalloc_arrive_scratch() {
+    static uint32_t* cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (cache[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_arrive) != cudaSuccess) return nullptr;
+        cache[dev] = static_cast<uint32_t*>(ptr);
+    }
+    return cache[dev];
+}
+
 // ------------------------------------------------------------------ host
 
 size_t replay_smem_bytes(const Shape& s, int rf, int ntok, int fused) {

@@ -67,6 +67,7 @@ def lib():
         "rssm_check_desc": ([D], ct.c_int),
         "rssm_state_field_bytes": ([D, i32], ct.c_size_t),
         "rssm_decode_step": ([D, S, vp, vp, vp, vp, vp, vp, vp, vp], ct.c_int),
+        "rssm_decode_step_noalloc": ([D, S, vp, vp, vp, vp, vp, vp, vp, vp], ct.c_int),
         "rssm_flush": ([D, S, vp, i32, vp], ct.c_int),
         "rssm_verify": ([D, S, i32, vp, vp, vp, vp, vp, vp, vp, vp], ct.c_int),
         "rssm_accept": ([D, S, vp, vp], ct.c_int),
@@ -181,6 +182,17 @@ def rssm_decode_step(state, x, B, C, dt, A, D, y, stream=None):
                                   _ptr(C, in_dt, "C"), _ptr(dt, torch.float32, "dt"), _ptr(A, torch.float32, "A"),
                                   _ptr(D, torch.float32, "D"), _ptr(y, torch.float32, "y"), _stream(stream)),
            "rssm_decode_step")
+    return y
+
+
+def rssm_decode_step_noalloc(state, x, B, C, dt, A, D, y, stream=None):
+    """rssm_decode_step without caller-allocated scratch (state.arrive unused)."""
+    d = state.desc
+    in_dt = _IN_DT[d.in_dtype]
+    _check(lib().rssm_decode_step_noalloc(ct.byref(d), ct.byref(state.struct), _ptr(x, in_dt, "x"),
+                                          _ptr(B, in_dt, "B"), _ptr(C, in_dt, "C"), _ptr(dt, torch.float32, "dt"),
+                                          _ptr(A, torch.float32, "A"), _ptr(D, torch.float32, "D"),
+                                          _ptr(y, torch.float32, "y"), _stream(stream)), "rssm_decode_step_noalloc")
     return y
 
 

@@ -180,6 +180,32 @@ RSSM_API rssm_status_t rssm_decode_step(const rssm_desc_t *desc, const rssm_stat
 RSSM_API rssm_status_t rssm_flush(const rssm_desc_t *desc, const rssm_state_t *state, const float *A,
                          int32_t force, void *stream);
 
+/* Largest batch rssm_decode_step_noalloc accepts. */
+#define RSSM_NOALLOC_MAX_BATCH 65536
+
+/* rssm_decode_step for callers that cannot allocate device memory -- for
+ * example an engine that plans all of its device memory ahead and hands each
+ * layer only the buffers it planned, or a process whose allocator is owned by
+ * another runtime. The article has no counterpart: this is an interface
+ * variant of this library, not a step of the method.
+ * Same arguments, results and errors as rssm_decode_step, except that
+ * state->arrive is not used (it may be NULL): the per-request arrival
+ * counters live in a file-scope device array of RSSM_NOALLOC_MAX_BATCH
+ * uint32 (256 KiB) that every GPU loading the library holds until the
+ * process exits. The call allocates nothing: it clears the counters it uses
+ * with cudaMemsetAsync on `stream` and launches the decode kernel.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the one array: calls whose work overlaps on the GPU
+ *    (other streams, concurrent graphs) race on it. Serialise them.
+ *  - batch > RSSM_NOALLOC_MAX_BATCH returns RSSM_ERR_CAPACITY and launches
+ *    nothing. */
+RSSM_API rssm_status_t rssm_decode_step_noalloc(const rssm_desc_t *desc, const rssm_state_t *state,
+                                                const void *x, const void *B, const void *C,
+                                                const float *dt, const float *A, const float *D,
+                                                float *y, void *stream);
+
 /* Speculative verify (s3): writes the K+1 tokens (the pending token j = 0
  * and K drafts) into slots pos..pos+K and computes their outputs from one
  * read of the checkpoint. pos is NOT advanced and no state is created.
