@@ -48,29 +48,27 @@ Shape shape_of(const rssm_desc_t* d) {
 
 rssm_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? RSSM_OK : RSSM_ERR_CUDA; }
 
-// Format and pointers of the copy that outputs read (s4: the output copy
-// when there is one, else the update copy itself).
-int read_format(const rssm_desc_t* d, const rssm_state_t* st, const void** tile, const uint8_t** scales) {
-    if (d->out_copy == RSSM_OUTCOPY_FP4) {
-        *tile = st->out_codes;
-        *scales = static_cast<const uint8_t*>(st->out_scales);
-        return kFP4;
-    }
-    *tile = st->ckpt;
-    *scales = static_cast<const uint8_t*>(st->ckpt_scales);
-    return d->update_dtype;
+// Format of the copy that outputs read (s4: the FP4 output copy when there
+// is one, else the update copy itself); it is the copy a record holds.
+int read_format(const rssm_desc_t* d) { return d->out_copy == RSSM_OUTCOPY_FP4 ? kFP4 : d->update_dtype; }
+
+RecLayout rec_of(const rssm_desc_t* d) {
+    return record_layout(shape_of(d), read_format(d), d->in_dtype == RSSM_BF16 ? 2 : 4);
 }
 
-bool fp4_needs_scales(const rssm_desc_t* d) { return d->update_dtype == RSSM_FP4; }
+// The update copy lives outside the records only beside an FP4 output copy.
+bool separate_ckpt(const rssm_desc_t* d) { return d->out_copy == RSSM_OUTCOPY_FP4; }
+
+rssm_status_t check_state_fields(const rssm_desc_t* d, const rssm_state_t* st, bool need_arrive) {
+    if (!st) return RSSM_ERR_INVALID_ARG;
+    if (!st->record || !st->bbuf || !st->pos || !st->flush_count || !st->err) return RSSM_ERR_INVALID_ARG;
+    if (need_arrive && !st->arrive) return RSSM_ERR_INVALID_ARG;
+    if (separate_ckpt(d) && !st->ckpt) return RSSM_ERR_INVALID_ARG;
+    return RSSM_OK;
+}
 
 rssm_status_t check_state_common(const rssm_desc_t* d, const rssm_state_t* st) {
-    if (!st) return RSSM_ERR_INVALID_ARG;
-    if (!st->ckpt || !st->xbuf || !st->bbuf || !st->dtbuf || !st->pos || !st->flush_count || !st->arrive ||
-        !st->err)
-        return RSSM_ERR_INVALID_ARG;
-    if (fp4_needs_scales(d) && !st->ckpt_scales) return RSSM_ERR_INVALID_ARG;
-    if (d->out_copy == RSSM_OUTCOPY_FP4 && (!st->out_codes || !st->out_scales)) return RSSM_ERR_INVALID_ARG;
-    return RSSM_OK;
+    return check_state_fields(d, st, true);
 }
 
 }  // namespace
@@ -109,6 +107,19 @@ rssm_status_t rssm_check_desc(const rssm_desc_t* d) {
     return RSSM_OK;
 }
 
+rssm_status_t rssm_record_layout(const rssm_desc_t* d, rssm_record_layout_t* out) {
+    rssm_status_t s = rssm_check_desc(d);
+    if (s != RSSM_OK) return s;
+    if (!out) return RSSM_ERR_INVALID_ARG;
+    const RecLayout r = rec_of(d);
+    out->bytes = r.bytes;
+    out->tile_bytes = r.tile;
+    out->scales_offset = r.scales;
+    out->dt_offset = r.dt;
+    out->x_offset = r.x;
+    return RSSM_OK;
+}
+
 size_t rssm_state_field_bytes(const rssm_desc_t* d, int32_t field) {
     if (rssm_check_desc(d) != RSSM_OK) return 0;
     const size_t Bz = d->batch, H = d->nheads, P = d->head_dim, N = d->d_state, G = d->ngroups;
@@ -116,19 +127,15 @@ size_t rssm_state_field_bytes(const rssm_desc_t* d, int32_t field) {
     const size_t in_el = d->in_dtype == RSSM_BF16 ? 2 : 4;
     const size_t n_state = Bz * H * P * N;
     switch (field) {
+        case RSSM_FIELD_RECORD: return Bz * H * rec_of(d).bytes;
         case RSSM_FIELD_CKPT:
+            if (!separate_ckpt(d)) return 0;
             switch (d->update_dtype) {
                 case RSSM_F32: return 4 * n_state;
                 case RSSM_BF16: return 2 * n_state;
-                case RSSM_E4M3: return n_state;
-                default: return n_state / 2;
+                default: return n_state;  // E4M3 (an FP4 update copy has no separate output copy)
             }
-        case RSSM_FIELD_CKPT_SCALES: return d->update_dtype == RSSM_FP4 ? n_state / 16 : 0;
-        case RSSM_FIELD_OUT_CODES: return d->out_copy == RSSM_OUTCOPY_FP4 ? n_state / 2 : 0;
-        case RSSM_FIELD_OUT_SCALES: return d->out_copy == RSSM_OUTCOPY_FP4 ? n_state / 16 : 0;
-        case RSSM_FIELD_XBUF: return Bz * H * cap * P * in_el;
         case RSSM_FIELD_BBUF: return Bz * G * cap * N * in_el;
-        case RSSM_FIELD_DTBUF: return Bz * H * ((cap + 3) & ~static_cast<size_t>(3)) * 4;
         case RSSM_FIELD_POS: return Bz * 4;
         case RSSM_FIELD_FLUSH_COUNT: return Bz * 4;
         case RSSM_FIELD_ARRIVE: return Bz * 4;
@@ -145,11 +152,10 @@ static rssm_status_t replay_call(const rssm_desc_t* d, const rssm_state_t* st, i
     a.ntok = ntok;
     a.advance = advance;
     a.fused = advance && (d->flags & RSSM_FLAG_FUSED_FLUSH) ? 1 : 0;
-    const int rf = read_format(d, st, &a.tile, &a.tile_scales);
-    a.ckpt_w = static_cast<float*>(st->ckpt);
-    a.xbuf = st->xbuf;
+    const int rf = read_format(d);
+    a.rec = rec_of(d);
+    a.record = static_cast<unsigned char*>(st->record);
     a.bbuf = st->bbuf;
-    a.dtbuf = st->dtbuf;
     a.pos = st->pos;
     a.flush_count = st->flush_count;
     a.arrive = st->arrive;
@@ -180,10 +186,7 @@ rssm_status_t rssm_decode_step_noalloc(const rssm_desc_t* d, const rssm_state_t*
     rssm_status_t s = rssm_check_desc(d);
     if (s != RSSM_OK) return s;
     if (d->batch > RSSM_NOALLOC_MAX_BATCH) return RSSM_ERR_CAPACITY;
-    if (!st || !st->ckpt || !st->xbuf || !st->bbuf || !st->dtbuf || !st->pos || !st->flush_count || !st->err)
-        return RSSM_ERR_INVALID_ARG;
-    if (fp4_needs_scales(d) && !st->ckpt_scales) return RSSM_ERR_INVALID_ARG;
-    if (d->out_copy == RSSM_OUTCOPY_FP4 && (!st->out_codes || !st->out_scales)) return RSSM_ERR_INVALID_ARG;
+    if ((s = check_state_fields(d, st, false)) != RSSM_OK) return s;
     if (!x || !B || !C || !dt || !A || !D || !y) return RSSM_ERR_INVALID_ARG;
     uint32_t* scratch = noalloc_arrive_scratch();
     if (!scratch) return RSSM_ERR_CUDA;
@@ -224,13 +227,16 @@ static rssm_status_t fold_launch(const rssm_desc_t* d, const rssm_state_t* st, i
     a.mode = mode;
     a.out_fp4 = d->out_copy == RSSM_OUTCOPY_FP4;
     a.seed = d->seed;
-    a.upd = st->ckpt;
-    a.upd_scales = static_cast<uint8_t*>(st->ckpt_scales);
-    a.out_codes = static_cast<uint8_t*>(st->out_codes);
-    a.out_scales = static_cast<uint8_t*>(st->out_scales);
-    a.xbuf = st->xbuf;
+    a.rec = rec_of(d);
+    a.record = static_cast<unsigned char*>(st->record);
+    if (separate_ckpt(d)) {
+        a.upd = static_cast<unsigned char*>(st->ckpt);
+        a.upd_stride = static_cast<uint32_t>(d->head_dim) * d->d_state * (d->update_dtype == RSSM_F32 ? 4 : d->update_dtype == RSSM_BF16 ? 2 : 1);
+    } else {
+        a.upd = a.record;
+        a.upd_stride = a.rec.bytes;
+    }
     a.bbuf = st->bbuf;
-    a.dtbuf = st->dtbuf;
     a.pos = st->pos;
     a.flush_count = st->flush_count;
     a.arrive = st->arrive;

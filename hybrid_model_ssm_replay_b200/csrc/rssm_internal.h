@@ -15,18 +15,25 @@ struct Shape {
     int batch, H, P, N, G, L, cap, lpr, capr;
 };
 
+// Byte geometry of one (request, head) record (rssm.h, RSSM_FIELD_RECORD):
+// [read copy values | FP4 scales | dt, capr floats | x, cap rows of P].
+struct RecLayout {
+    uint32_t bytes;   // record stride (a multiple of 128)
+    uint32_t tile;    // bytes of the read copy's values (FP4: codes)
+    uint32_t scales;  // offset of the FP4 scales
+    uint32_t dt;      // offset of the buffered dt
+    uint32_t x;       // offset of the buffered x
+};
+
 // Replay decode / verify (ReplaySSM article s1, s3).
 struct ReplayArgs {
     Shape s;
     int ntok;        // tokens per request in this call: 1 (decode) or K+1 (verify)
     int advance;     // decode: pos += 1 by the last CTA of the request
     int fused;       // decode: fold the buffer when this token fills it (fp32 state)
-    const void* tile;            // read copy: fp32 / bf16 / e4m3 values or FP4 codes
-    const uint8_t* tile_scales;  // FP4 scales of the read copy
-    float* ckpt_w;               // fused flush: fp32 checkpoint written back
-    void* xbuf;
+    RecLayout rec;
+    unsigned char* record;  // record (b, h) at record + (b*H + h) * rec.bytes
     void* bbuf;
-    float* dtbuf;
     int32_t* pos;
     uint32_t* flush_count;
     uint32_t* arrive;
@@ -56,11 +63,14 @@ inline FastDiv make_fastdiv(uint32_t d) {
     return f;
 }
 
-// Shared-memory stage of the pipelined replay kernel: byte offsets of the
-// state tile, FP4 scales, x rows [cap][P], B rows [cap][N], C rows [ntok][N],
-// dt row [capr], this call's dt [8] and the position; `stages` stages.
+// Shared-memory stage of the pipelined replay kernel: a mirror of the
+// record prefix (same offsets as RecLayout, x rows up to cap), the buffered
+// B rows [cap][N] at `brows` and this call's dt [8], A_h, D_h and the
+// position at `meta`; `stages` stages. After them, per consumer group, two
+// buffers of `newrows` bytes for the x, B and C rows of this call
+// ([ntok][P], [ntok][N], [ntok][N] at 0, nb_off, nc_off).
 struct PipeLayout {
-    uint32_t stage_bytes, tile, scales, xrows, brows, crows, dtrow, dtnew, meta;
+    uint32_t stage_bytes, brows, meta, newrows, nb_off, nc_off;
     int stages;
     FastDiv divH, divHpg;  // tile -> (request, head), head -> group
 };
@@ -69,15 +79,13 @@ struct PipeLayout {
 struct FoldArgs {
     Shape s;
     int mode;          // 0: pos >= L only; 1: also any pos > 0; 2: every request
-    int out_fp4;       // also write the FP4 output copy
+    int out_fp4;       // also write the FP4 output copy (the record's read copy)
     uint64_t seed;
-    void* upd;         // update copy (fp32 / bf16 / e4m3 values or FP4 codes)
-    uint8_t* upd_scales;
-    uint8_t* out_codes;
-    uint8_t* out_scales;
-    const void* xbuf;
+    RecLayout rec;
+    unsigned char* record;
+    unsigned char* upd;    // update copy of (b, h) at upd + (b*H + h) * upd_stride
+    uint32_t upd_stride;   // (FP4 update copy: scales at upd + ... + rec.scales)
     const void* bbuf;
-    const float* dtbuf;
     int32_t* pos;
     uint32_t* flush_count;
     uint32_t* arrive;
@@ -117,6 +125,9 @@ uint32_t* noalloc_arrive_scratch();
 // Dynamic shared memory of one CTA, in bytes.
 size_t replay_smem_bytes(const Shape& s, int read_fmt, int ntok, int fused);
 size_t fold_smem_bytes(const Shape& s, int upd_fmt);
+
+// Record geometry for the read-copy format and the input element size.
+RecLayout record_layout(const Shape& s, int read_fmt, int in_bytes);
 size_t conv_smem_bytes(const Shape& s);
 
 }  // namespace rssm

@@ -238,9 +238,10 @@ __global__ void __launch_bounds__(kThreads, replay_min_blocks(NT, FUSED)) k_repl
     const TIn* Cin = static_cast<const TIn*>(a.C) + static_cast<size_t>(b) * ntok * GN + static_cast<size_t>(g) * N;
     const float* dtin = a.dt + static_cast<size_t>(b) * ntok * H + h;
     float* yout = a.y + static_cast<size_t>(b) * ntok * HP + static_cast<size_t>(h) * P;
-    TIn* xb = static_cast<TIn*>(a.xbuf) + bh * cap * P;
+    unsigned char* rec = a.record + bh * a.rec.bytes;
+    TIn* xb = reinterpret_cast<TIn*>(rec + a.rec.x);
     TIn* bb = static_cast<TIn*>(a.bbuf) + bg * cap * N;
-    float* dtb = a.dtbuf + bh * a.s.capr;
+    float* dtb = reinterpret_cast<float*>(rec + a.rec.dt);
 
     const uint32_t tb = tile_bytes(RF, P, N), sb = scale_bytes(RF, P, N);
     unsigned char* s_tile = smem;
@@ -251,9 +252,9 @@ __global__ void __launch_bounds__(kThreads, replay_min_blocks(NT, FUSED)) k_repl
 
     if (tid == 0) {
         mbar_init(bar_a, 1);
+        // the copy's values and (FP4) scales, contiguous in the record as here
         mbar_expect_tx(bar_a, tb + sb);
-        bulk_g2s(smem_u32(s_tile), static_cast<const unsigned char*>(a.tile) + bh * tb, tb, bar_a);
-        if (RF == kFP4) bulk_g2s(smem_u32(s_sc), a.tile_scales + bh * sb, sb, bar_a);
+        bulk_g2s(smem_u32(s_tile), rec, tb + sb, bar_a);
         s_pos = a.pos[b];  // the only read of pos: every thread uses this copy
     }
 
@@ -464,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, replay_min_blocks(NT, FUSED)) k_repl
         if (fold_now) {
             // fused flush: the token that fills the buffer folds it into the
             // checkpoint from the tile, x rows and B rows already in shared memory.
-            float* dst = a.ckpt_w + bh * P * N;
+            float* dst = reinterpret_cast<float*>(rec);
             auto brow = [&](int sl, int c) {
                 const float w = s_w[0][sl];
                 const float4 v = reinterpret_cast<const float4*>(s_B + sl * N)[c];
@@ -482,14 +483,16 @@ __global__ void __launch_bounds__(kThreads, replay_min_blocks(NT, FUSED)) k_repl
 // Persistent, warp-specialised replay decode / verify for d_state 128 and
 // head_dim a multiple of 8. One CTA per SM walks the tiles
 // t = blockIdx.x + k * gridDim.x ((request, head) = (t / H, t % H)).
-// A producer warp reads each tile's position one tile ahead and brings all
-// of the tile's inputs into a ring of shared-memory stages with bulk copies
-// (the state tile, the buffered x and B rows, this call's x, B and C rows,
-// the dt row; completion on the stage's "full" mbarrier). Eight consumer
-// warps compute the outputs from shared memory only and release the stage
-// (its "empty" mbarrier). The HBM stream never waits for a tile's
-// arithmetic, and a tile's arithmetic never waits for HBM latency.
-// Every wait is bounded by %globaltimer; a timeout sets the error word.
+// A producer warp reads each tile's position one tile ahead and brings the
+// tile's state into a ring of shared-memory stages with two bulk copies (the
+// record prefix -- copy, dt row and buffered x rows -- and the buffered B
+// rows; completion on the stage's "full" mbarrier). Consumer warps compute
+// the outputs from shared memory only and release the stage (its "empty"
+// mbarrier). This call's x, B and C rows come from the consumers
+// themselves, one tile ahead (cp.async into a per-group double buffer).
+// The HBM stream never waits for a tile's arithmetic, and a tile's
+// arithmetic never waits for HBM latency. Every wait is bounded by
+// %globaltimer; a timeout sets the error word.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t fdiv(uint32_t x, const FastDiv& f) { return (__umulhi(x, f.mul) + x) >> f.shr; }
 
@@ -515,10 +518,19 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Consumer groups of the pipelined kernel: two for decode, one for verify
 // (whose K+1 tokens need the registers).
 __host__ __device__ constexpr int pipe_groups(int nt) { return nt == 1 ? 2 : 1; }
 __host__ __device__ constexpr int pipe_threads(int nt) { return (pipe_groups(nt) * kConsWarps + 1) * 32; }
+
+// Stage meta: this call's dt [kMaxTok], A_h, D_h (floats), then the position.
+constexpr int kMetaA = kMaxTok, kMetaD = kMaxTok + 1, kMetaPos = kMaxTok + 2;
 
 template <typename TIn, int RF, int NT>
 __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const ReplayArgs a, const PipeLayout lay) {
@@ -531,14 +543,12 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
     __shared__ float s_decay[CG][NT];       // exp(A S_t)
     __shared__ volatile int s_abort;
 
-    const int H = a.s.H, P = a.s.P, N = a.s.N, G = a.s.G, cap = a.s.cap, capr = a.s.capr;
+    const int H = a.s.H, P = a.s.P, N = a.s.N, G = a.s.G, cap = a.s.cap;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int ntok = a.ntok, S = lay.stages;
     const int ntiles = a.s.batch * H;
     const size_t HP = static_cast<size_t>(H) * P, GN = static_cast<size_t>(G) * N;
     constexpr int es = static_cast<int>(sizeof(TIn));
-    const uint32_t tb = tile_bytes(RF, P, N), sb = scale_bytes(RF, P, N);
-    (void)G;
 
     if (tid == 0) {
         for (int st = 0; st < S; ++st) {
@@ -633,71 +643,25 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
                 aborted = true;
                 break;
             }
-            const size_t bh = static_cast<size_t>(b) * H + h, bg = static_cast<size_t>(b) * G + g;
-            const uint32_t fb = smem_u32(&full_bar[st]);
             if (lane == 0) {
-                float* meta = reinterpret_cast<float*>(sp + lay.dtnew);  // dt[8], then A, D
+                const uint32_t fb = smem_u32(&full_bar[st]);
+                float* meta = reinterpret_cast<float*>(sp + lay.meta);
 #pragma unroll
                 for (int j = 0; j < NT; ++j)
                     if (j < ntok) meta[j] = dtj[j];
-                meta[kMaxTok] = Ah;
-                meta[kMaxTok + 1] = Dh;
-                *reinterpret_cast<int*>(sp + lay.meta) = pos;
-                uint32_t bytes = tb + sb;
-                if (ok)
-                    bytes += static_cast<uint32_t>((pos + ntok) * P * es + (pos + ntok) * N * es + ntok * N * es +
-                                                   capr * 4);
-                mbar_expect_tx(fb, bytes);
-            }
-            __syncwarp();
-            // the tile's copies, one per lane, issued together:
-            // 0 tile, 1 FP4 scales, 2 buffered x rows, 3 buffered B rows, 4 dt row,
-            // then per token j: 5+3j x row, 6+3j B row, 7+3j C row
-            {
-                const void* src = nullptr;
-                uint32_t dst = 0, nb = 0;
-                if (lane == 0) {
-                    src = static_cast<const unsigned char*>(a.tile) + bh * tb;
-                    dst = smem_u32(sp + lay.tile);
-                    nb = tb;
-                } else if (lane == 1) {
-                    if (RF == kFP4) {
-                        src = a.tile_scales + bh * sb;
-                        dst = smem_u32(sp + lay.scales);
-                        nb = sb;
-                    }
-                } else if (ok) {
-                    if (lane == 2 && pos > 0) {
-                        src = static_cast<const TIn*>(a.xbuf) + bh * cap * P;
-                        dst = smem_u32(sp + lay.xrows);
-                        nb = pos * P * es;
-                    } else if (lane == 3 && pos > 0) {
-                        src = static_cast<const TIn*>(a.bbuf) + bg * cap * N;
-                        dst = smem_u32(sp + lay.brows);
-                        nb = pos * N * es;
-                    } else if (lane == 4) {
-                        src = a.dtbuf + bh * capr;
-                        dst = smem_u32(sp + lay.dtrow);
-                        nb = capr * 4;
-                    } else if (lane >= 5 && lane < 5 + 3 * ntok) {
-                        const int j = (lane - 5) / 3, w = (lane - 5) - 3 * j;
-                        const size_t bj = static_cast<size_t>(b) * ntok + j;
-                        if (w == 0) {
-                            src = static_cast<const TIn*>(a.x) + bj * HP + static_cast<size_t>(h) * P;
-                            dst = smem_u32(sp + lay.xrows + (pos + j) * P * es);
-                            nb = P * es;
-                        } else if (w == 1) {
-                            src = static_cast<const TIn*>(a.B) + bj * GN + static_cast<size_t>(g) * N;
-                            dst = smem_u32(sp + lay.brows + (pos + j) * N * es);
-                            nb = N * es;
-                        } else {
-                            src = static_cast<const TIn*>(a.C) + bj * GN + static_cast<size_t>(g) * N;
-                            dst = smem_u32(sp + lay.crows + j * N * es);
-                            nb = N * es;
-                        }
-                    }
+                meta[kMetaA] = Ah;
+                meta[kMetaD] = Dh;
+                reinterpret_cast<int*>(meta)[kMetaPos] = pos;
+                // record prefix: copy, scales, dt row and x rows 0..pos-1
+                const uint32_t nrec = a.rec.x + static_cast<uint32_t>(pos * P * es);
+                const uint32_t nb = static_cast<uint32_t>(pos * N * es);
+                mbar_expect_tx(fb, ok ? nrec + nb : 0u);  // nothing to copy for a bad position
+                if (ok) {
+                    const size_t bh = static_cast<size_t>(b) * H + h, bg = static_cast<size_t>(b) * G + g;
+                    bulk_g2s(smem_u32(sp), a.record + bh * a.rec.bytes, nrec, fb);
+                    if (nb > 0)
+                        bulk_g2s(smem_u32(sp + lay.brows), static_cast<const TIn*>(a.bbuf) + bg * cap * N, nb, fb);
                 }
-                if (nb > 0) bulk_g2s(dst, src, nb, fb);
             }
             k_issued = k;
             __syncwarp();
@@ -717,14 +681,47 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
     }
 
     // --------------------------------------------------------------- consumers
-    // Group gi takes tiles k = gi, gi + 2, ...; its 8 warps: warps 0..3 form
-    // the B.C products (8 slots each), warp 7 the decay weights, all of them
-    // 8 rows each of the output.
+    // Group gi takes tiles k = gi, gi + CG, ...; its 8 warps: warps 0..3 form
+    // the B.C products (8 slots each), warp 7 the decay weights, warps 4..5
+    // append this call's x and B to the buffer, all of them 8 rows each of
+    // the output.
     const int gi = warp / kConsWarps, cw = warp - gi * kConsWarps;
     const int ctid = tid - gi * kConsWarps * 32;
-    const int hpg_shift_free = 0;
-    (void)hpg_shift_free;
-    for (int k = gi;; k += CG) {
+    unsigned char* nbase = smem + static_cast<size_t>(S) * lay.stage_bytes + static_cast<size_t>(gi) * 2 * lay.newrows;
+    // this call's rows of tile kk -> buf: [ntok][P] x, [ntok][N] B, [ntok][N] C, 16-byte chunks
+    const int xc = (P * es) >> 4, bc = (N * es) >> 4, per_tok = xc + 2 * bc;
+    auto prefetch = [&](int kk, unsigned char* buf) {
+        const uint32_t t = blockIdx.x + static_cast<uint32_t>(kk) * gridDim.x;
+        if (t >= static_cast<uint32_t>(ntiles)) return;
+        const int b = fdiv(t, lay.divH), h = t - b * H, g = fdiv(h, lay.divHpg);
+        for (int q = ctid; q < ntok * per_tok; q += kConsWarps * 32) {
+            const int j = q / per_tok;
+            int r = q - j * per_tok;
+            const size_t bj = static_cast<size_t>(b) * ntok + j;
+            const unsigned char* src;
+            uint32_t dst;
+            if (r < xc) {
+                src = reinterpret_cast<const unsigned char*>(static_cast<const TIn*>(a.x) + bj * HP +
+                                                             static_cast<size_t>(h) * P);
+                dst = smem_u32(buf + j * P * es);
+            } else if (r < xc + bc) {
+                r -= xc;
+                src = reinterpret_cast<const unsigned char*>(static_cast<const TIn*>(a.B) + bj * GN +
+                                                             static_cast<size_t>(g) * N);
+                dst = smem_u32(buf + lay.nb_off + j * N * es);
+            } else {
+                r -= xc + bc;
+                src = reinterpret_cast<const unsigned char*>(static_cast<const TIn*>(a.C) + bj * GN +
+                                                             static_cast<size_t>(g) * N);
+                dst = smem_u32(buf + lay.nc_off + j * N * es);
+            }
+            cp_async16(dst + 16u * r, src + 16 * r);
+        }
+        cp_async_commit();
+    };
+    prefetch(gi, nbase);
+    int it = 0;
+    for (int k = gi;; k += CG, ++it) {
         const uint32_t t = blockIdx.x + static_cast<uint32_t>(k) * gridDim.x;
         if (t >= static_cast<uint32_t>(ntiles)) break;
         const int b = fdiv(t, lay.divH), h = t - b * H, g = fdiv(h, lay.divHpg);
@@ -741,22 +738,29 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
                 mbar_wait_bounded(smem_u32(&full_bar[st]), use & 1, kWaitNs);  // copies in flight
             }
         }
-        // the stage has landed; this group's previous readers of s_w / s_g are done
+        cp_async_wait_all();  // this thread's share of this tile's rows
+        // the stage and this tile's rows have landed; this group's previous
+        // readers of s_w / s_g and of the other row buffer are done
         if (group_sync_or(gi, stop)) break;
-        const int pos = *reinterpret_cast<const int*>(sp + lay.meta);
+        const unsigned char* nr = nbase + (it & 1) * lay.newrows;
+        prefetch(k + CG, nbase + ((it + 1) & 1) * lay.newrows);
+        const float* meta = reinterpret_cast<const float*>(sp + lay.meta);  // dt[8], A, D, pos
+        const int pos = reinterpret_cast<const int*>(meta)[kMetaPos];
         const int T = pos + ntok;
         const bool ok = pos >= 0 && T <= cap;
-        const TIn* xr = reinterpret_cast<const TIn*>(sp + lay.xrows);  // slot s row: xr + s*P
-        const TIn* br = reinterpret_cast<const TIn*>(sp + lay.brows);  // slot s row: br + s*N
-        const TIn* cr = reinterpret_cast<const TIn*>(sp + lay.crows);  // token j row: cr + j*N
-        const float* meta = reinterpret_cast<const float*>(sp + lay.dtnew);  // dt[8], A, D
+        const TIn* xr = reinterpret_cast<const TIn*>(sp + a.rec.x);     // slot s < pos: xr + s*P
+        const TIn* br = reinterpret_cast<const TIn*>(sp + lay.brows);   // slot s < pos: br + s*N
+        const TIn* nx = reinterpret_cast<const TIn*>(nr);               // token j: nx + j*P
+        const TIn* nb = reinterpret_cast<const TIn*>(nr + lay.nb_off);  // token j: nb + j*N
+        const TIn* nc = reinterpret_cast<const TIn*>(nr + lay.nc_off);  // token j: nc + j*N
+        unsigned char* rec = a.record + bh * a.rec.bytes;
         float4 c4[NT];
         if (!ok) {
             if (ctid == 0) set_error(a.err, (pos < 0 || pos > cap) ? RSSM_DEVERR_POS_RANGE : RSSM_DEVERR_CAPACITY);
         } else {
 #pragma unroll
             for (int j = 0; j < NT; ++j)
-                c4[j] = (j < ntok) ? load4(cr + j * N + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+                c4[j] = (j < ntok) ? load4(nc + j * N + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
             if (cw * 8 < T) {
                 // B_s . C_j for slots s0..s0+7, reduced together
                 const int s0 = cw * 8;
@@ -765,8 +769,11 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
                     if (j < ntok) {
                         float part[8];
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            part[kk] = (s0 + kk < T) ? dot4(load4(br + (s0 + kk) * N + 4 * lane), c4[j]) : 0.f;
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const int sl = s0 + kk;
+                            const TIn* row = (sl < pos) ? br + sl * N : nb + (sl - pos) * N;
+                            part[kk] = (sl < T) ? dot4(load4(row + 4 * lane), c4[j]) : 0.f;
+                        }
                         const float z = warp_reduce8(part);
                         const int sl = s0 + ((lane >> 2) & 7);
                         if ((lane & 3) == 0 && sl < T) s_g[gi][j][sl] = z;
@@ -774,12 +781,12 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
                 }
             }
             if (cw == kConsWarps - 1) {
-                const float* dtrow = reinterpret_cast<const float*>(sp + lay.dtrow);
+                const float* dtrow = reinterpret_cast<const float*>(sp + a.rec.dt);
                 const float dnew = (lane >= pos && lane < T) ? meta[lane - pos] : 0.f;
                 const float dts = (lane < pos) ? dtrow[lane] : dnew;
-                if (lane >= pos && lane < T) a.dtbuf[bh * capr + lane] = dnew;
+                if (lane >= pos && lane < T) reinterpret_cast<float*>(rec + a.rec.dt)[lane] = dnew;
                 const float Sx = warp_prefix(dts);
-                const float Ah = meta[kMaxTok];
+                const float Ah = meta[kMetaA];
 #pragma unroll
                 for (int j = 0; j < NT; ++j) {
                     if (j < ntok) {
@@ -792,22 +799,22 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
             if (cw == 4 || cw == 5) {
                 // append this call's x (and, for the group's first head, B) to the buffer
                 const int q0 = ctid - 4 * 32;  // 0..63
-                const int xq = (ntok * P * es) >> 4, bq = (ntok * N * es) >> 4;
-                for (int q = q0; q < xq; q += 64)
-                    reinterpret_cast<uint4*>(static_cast<TIn*>(a.xbuf) + (bh * cap + pos) * P)[q] =
-                        reinterpret_cast<const uint4*>(xr + pos * P)[q];
-                if (h == g * (H / G))
-                    for (int q = q0; q < bq; q += 64)
-                        reinterpret_cast<uint4*>(static_cast<TIn*>(a.bbuf) + (bg * cap + pos) * N)[q] =
-                            reinterpret_cast<const uint4*>(br + pos * N)[q];
+                const int xq = ntok * xc, bq = ntok * bc;
+                uint4* xdst = reinterpret_cast<uint4*>(rec + a.rec.x + static_cast<size_t>(pos) * P * es);
+                for (int q = q0; q < xq; q += 64) xdst[q] = reinterpret_cast<const uint4*>(nx)[q];
+                if (h == g * (H / G)) {
+                    uint4* bdst = reinterpret_cast<uint4*>(static_cast<TIn*>(a.bbuf) + (bg * cap + pos) * N);
+                    for (int q = q0; q < bq; q += 64) bdst[q] = reinterpret_cast<const uint4*>(nb)[q];
+                }
             }
         }
         group_sync(gi);  // s_w, s_g, s_decay ready
         if (ok) {
-            const unsigned char* tile = sp + lay.tile;
-            const unsigned char* sc = sp + lay.scales;
-            const float Dh = meta[kMaxTok + 1];
+            const unsigned char* tile = sp;
+            const unsigned char* sc = sp + a.rec.scales;
+            const float Dh = meta[kMetaD];
             float* yout = a.y + static_cast<size_t>(b) * ntok * HP + static_cast<size_t>(h) * P;
+            const TIn* xrow = (lane < pos) ? xr + lane * P : nx + (lane - pos) * P;  // slot `lane`
             for (int r0 = cw * 8; r0 < P; r0 += kConsWarps * 8) {
 #pragma unroll
                 for (int j = 0; j < NT; ++j) {
@@ -824,20 +831,20 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
                         if (lane <= tt) {
                             const float coef = s_w[gi][j][lane] * s_g[gi][j][lane];
                             Raw8<TIn> xv;
-                            xv.load(xr + lane * P + r0);
-                            const float4 xa = xv.lo(), xc = xv.hi();
+                            xv.load(xrow + r0);
+                            const float4 xa = xv.lo(), xc4 = xv.hi();
                             part[0] = fmaf(coef, xa.x, part[0]);
                             part[1] = fmaf(coef, xa.y, part[1]);
                             part[2] = fmaf(coef, xa.z, part[2]);
                             part[3] = fmaf(coef, xa.w, part[3]);
-                            part[4] = fmaf(coef, xc.x, part[4]);
-                            part[5] = fmaf(coef, xc.y, part[5]);
-                            part[6] = fmaf(coef, xc.z, part[6]);
-                            part[7] = fmaf(coef, xc.w, part[7]);
+                            part[4] = fmaf(coef, xc4.x, part[4]);
+                            part[5] = fmaf(coef, xc4.y, part[5]);
+                            part[6] = fmaf(coef, xc4.z, part[6]);
+                            part[7] = fmaf(coef, xc4.w, part[7]);
                         }
                         const float z = warp_reduce8(part);
                         const int r = r0 + ((lane >> 2) & 7);
-                        if ((lane & 3) == 0 && r < P) yout[j * HP + r] = fmaf(Dh, to_f32(xr[tt * P + r]), z);
+                        if ((lane & 3) == 0 && r < P) yout[j * HP + r] = fmaf(Dh, to_f32(nx[j * P + r]), z);
                     }
                 }
             }
@@ -845,6 +852,7 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
     }
+    cp_async_wait_all();  // no copy of this thread outlives the CTA
 }
 
 // ---------------------------------------------------------------------------
@@ -884,10 +892,10 @@ __global__ void __launch_bounds__(kThreads, 4) k_fold(const FoldArgs a) {
         s_fc = a.flush_count[b];
         const bool go0 = p0 >= 0 && p0 <= cap && ((p0 >= a.s.L) || (a.mode >= 1 && p0 > 0) || (a.mode == 2));
         if (go0) {
+            // values and (FP4, in the record) scales: contiguous, as here
             mbar_init(bar_a, 1);
             mbar_expect_tx(bar_a, tb + sb);
-            bulk_g2s(smem_u32(s_in), static_cast<const unsigned char*>(a.upd) + bh * tb, tb, bar_a);
-            if (UF == kFP4) bulk_g2s(smem_u32(s_insc), a.upd_scales + bh * sb, sb, bar_a);
+            bulk_g2s(smem_u32(s_in), a.upd + bh * a.upd_stride, tb + sb, bar_a);
         }
     }
     __syncthreads();
@@ -904,13 +912,14 @@ __global__ void __launch_bounds__(kThreads, 4) k_fold(const FoldArgs a) {
     // once every CTA of the request has arrived, the last one resets them
     if (tid == kThreads - 32) request_done(a.arrive, b, H, a.pos, 0, a.flush_count, true);
 
-    const TIn* xb = static_cast<const TIn*>(a.xbuf);
+    unsigned char* rec = a.record + bh * a.rec.bytes;
+    unsigned char* upd = a.upd + bh * a.upd_stride;
     const TIn* bb = static_cast<const TIn*>(a.bbuf);
     const float Ah = a.A[h];
     // one round of independent loads: B rows, x rows (16-byte chunks when the
     // rows allow it), dt
     const TIn* bbg = bb + (static_cast<size_t>(b) * G + g) * cap * N;
-    const TIn* xbh = xb + bh * cap * P;
+    const TIn* xbh = reinterpret_cast<const TIn*>(rec + a.rec.x);
     for (int q = tid; q < ((T * N) >> 3); q += kThreads) {
         Raw8<TIn> r;
         r.load(bbg + (q << 3));
@@ -930,7 +939,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_fold(const FoldArgs a) {
         for (int i = tid; i < T * P; i += kThreads) s_x[(i / P) * xs + (i % P)] = to_f32(xbh[i]);
     }
     if (warp == 0) {
-        const float dts = (lane < T) ? a.dtbuf[bh * a.s.capr + lane] : 0.f;
+        const float dts = (lane < T) ? reinterpret_cast<const float*>(rec + a.rec.dt)[lane] : 0.f;
         const float Sx = warp_prefix(dts);
         const float Stot = T > 0 ? __shfl_sync(0xffffffffu, Sx, T - 1) : 0.f;
         s_cw[lane] = (lane < T) ? dts * expf(Ah * (Stot - Sx)) : 0.f;
@@ -962,40 +971,40 @@ __global__ void __launch_bounds__(kThreads, 4) k_fold(const FoldArgs a) {
         return make_float4(w * v.x, w * v.y, w * v.z, w * v.w);
     };
     auto emit = [&](int r, int c, float4 v, bool valid) {
-        const size_t e = (bh * P + r) * N + 4 * c;  // flat element index of v.x
+        const uint32_t e = static_cast<uint32_t>(r * N + 4 * c);  // element of v.x within the head
         if constexpr (UF == kF32) {
-            if (valid) stream_store4(static_cast<float*>(a.upd) + e, v);
+            if (valid) stream_store4(reinterpret_cast<float*>(upd) + e, v);
         } else if constexpr (UF == kBF16 || UF == kE4M3) {
             if (valid) {
-                // Philox counter (e/4, head, request, flush_count), e within the head
-                const uint32_t e_head = static_cast<uint32_t>(r * N + 4 * c);
-                const uint4 rw = philox4x32_10(make_uint4(e_head >> 2, h, b, fc),
+                // Philox counter (e/4, head, request, flush_count)
+                const uint4 rw = philox4x32_10(make_uint4(e >> 2, h, b, fc),
                                                make_uint2(static_cast<uint32_t>(a.seed),
                                                           static_cast<uint32_t>(a.seed >> 32)));
                 if constexpr (UF == kBF16) {
                     const uint2 w = make_uint2(sr_bf16(v.x, rw.x) | (sr_bf16(v.y, rw.y) << 16),
                                                sr_bf16(v.z, rw.z) | (sr_bf16(v.w, rw.w) << 16));
-                    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.upd) + e) = w;
+                    *reinterpret_cast<uint2*>(upd + 2u * e) = w;
                 } else {
                     const uint32_t w = sr_e4m3(v.x, rw.x) | (sr_e4m3(v.y, rw.y) << 8) |
                                        (sr_e4m3(v.z, rw.z) << 16) | (sr_e4m3(v.w, rw.w) << 24);
-                    *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(a.upd) + e) = w;
+                    *reinterpret_cast<uint32_t*>(upd + e) = w;
                 }
             }
         } else {
+            // the shared FP4 copy lives in the record: scales at rec.scales
             uint32_t sc;
             const uint32_t codes = fp4_quant_quad(v, &sc);
             if (valid) {
-                *reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(a.upd) + e / 2) = static_cast<uint16_t>(codes);
-                if ((c & 3) == 0) a.upd_scales[e / 16] = static_cast<uint8_t>(sc);
+                *reinterpret_cast<uint16_t*>(upd + e / 2) = static_cast<uint16_t>(codes);
+                if ((c & 3) == 0) upd[a.rec.scales + e / 16] = static_cast<uint8_t>(sc);
             }
         }
         if constexpr (OUT4 != 0) {
             uint32_t sc;
             const uint32_t codes = fp4_quant_quad(v, &sc);
             if (valid) {
-                *reinterpret_cast<uint16_t*>(a.out_codes + e / 2) = static_cast<uint16_t>(codes);
-                if ((c & 3) == 0) a.out_scales[e / 16] = static_cast<uint8_t>(sc);
+                *reinterpret_cast<uint16_t*>(rec + e / 2) = static_cast<uint16_t>(codes);
+                if ((c & 3) == 0) rec[a.rec.scales + e / 16] = static_cast<uint8_t>(sc);
             }
         }
     };
@@ -1232,29 +1241,29 @@ static cudaError_t replay_dispatch_wide(const ReplayArgs& a, int rf, size_t smem
                 : replay_dispatch_fmt<TIn, NT, 0>(a, rf, smem, nblk, st);
 }
 
-// Stage layout of k_replay_pipe (16-byte aligned pieces, 128-byte aligned stages).
-PipeLayout pipe_layout(const Shape& s, int rf, int ntok, int in_bf16, size_t smem_budget) {
+RecLayout record_layout(const Shape& s, int rf, int in_bytes) {
+    RecLayout r;
+    r.tile = tile_bytes(rf, s.P, s.N);
+    r.scales = rf == kFP4 ? align16(r.tile) : 0u;
+    r.dt = align16(align16(r.tile) + scale_bytes(rf, s.P, s.N));
+    r.x = r.dt + 4u * static_cast<uint32_t>(s.capr);
+    r.bytes = (r.x + static_cast<uint32_t>(s.cap * s.P * in_bytes) + 127u) & ~127u;
+    return r;
+}
+
+// Stage layout of k_replay_pipe (16-byte aligned pieces, 128-byte aligned
+// stages and row buffers); the stages fill what the row buffers leave.
+PipeLayout pipe_layout(const Shape& s, const RecLayout& rec, int ntok, int in_bf16, int groups, size_t smem_budget) {
     const uint32_t es = in_bf16 ? 2u : 4u;
     PipeLayout L;
-    uint32_t off = 0;
-    L.tile = off;
-    off += align16(tile_bytes(rf, s.P, s.N));
-    L.scales = off;
-    off += align16(scale_bytes(rf, s.P, s.N));
-    L.xrows = off;
-    off += align16(static_cast<uint32_t>(s.cap * s.P) * es);
-    L.brows = off;
-    off += align16(static_cast<uint32_t>(s.cap * s.N) * es);
-    L.crows = off;
-    off += align16(static_cast<uint32_t>(ntok * s.N) * es);
-    L.dtrow = off;
-    off += align16(static_cast<uint32_t>(s.capr) * 4u);
-    L.dtnew = off;  // this call's dt [kMaxTok], then A_h and D_h
-    off += 4u * kMaxTok + 16u;
-    L.meta = off;
-    off += 16u;
-    L.stage_bytes = (off + 127u) & ~127u;
-    const size_t n = smem_budget / L.stage_bytes;
+    L.brows = align16(rec.x + static_cast<uint32_t>(s.cap * s.P) * es);
+    L.meta = L.brows + align16(static_cast<uint32_t>(s.cap * s.N) * es);
+    L.stage_bytes = (L.meta + 64u + 127u) & ~127u;
+    L.nb_off = align16(static_cast<uint32_t>(ntok * s.P) * es);
+    L.nc_off = L.nb_off + align16(static_cast<uint32_t>(ntok * s.N) * es);
+    L.newrows = (L.nc_off + static_cast<uint32_t>(ntok * s.N) * es + 127u) & ~127u;
+    const size_t rows = static_cast<size_t>(groups) * 2u * L.newrows;
+    const size_t n = smem_budget > rows ? (smem_budget - rows) / L.stage_bytes : 0;
     L.stages = static_cast<int>(n < static_cast<size_t>(kPipeStagesMax) ? n : kPipeStagesMax);
     L.divH = make_fastdiv(static_cast<uint32_t>(s.H));
     L.divHpg = make_fastdiv(static_cast<uint32_t>(s.H / s.G));
@@ -1282,8 +1291,8 @@ static DeviceInfo device_info() {
 
 template <typename TIn, int NT>
 static cudaError_t pipe_dispatch(const ReplayArgs& a, const PipeLayout& L, int rf, int grid, cudaStream_t st) {
-    const size_t smem = static_cast<size_t>(L.stages) * L.stage_bytes;
     constexpr int thr = pipe_threads(NT);
+    const size_t smem = static_cast<size_t>(L.stages) * L.stage_bytes + 2u * pipe_groups(NT) * L.newrows;
     switch (rf) {
         case kF32: return launch_grid(k_replay_pipe<TIn, kF32, NT>, a, L, grid, thr, smem, st);
         case kBF16: return launch_grid(k_replay_pipe<TIn, kBF16, NT>, a, L, grid, thr, smem, st);
@@ -1309,7 +1318,8 @@ cudaError_t launch_replay(const ReplayArgs& a, int in_bf16, int rf, cudaStream_t
         const DeviceInfo di = device_info();
         if (di.sms > 0) {
             const size_t budget = di.smem_optin > 4096 ? di.smem_optin - 4096 : 0;
-            const PipeLayout L = pipe_layout(a.s, rf, a.ntok, in_bf16, budget);
+            const int groups = a.ntok == 1 ? pipe_groups(1) : pipe_groups(kMidTok);
+            const PipeLayout L = pipe_layout(a.s, a.rec, a.ntok, in_bf16, groups, budget);
             if (L.stages >= 2) {
                 const int ntiles = a.s.batch * a.s.H;
                 const int grid = ntiles < di.sms ? ntiles : di.sms;

@@ -24,8 +24,7 @@ RSSM_FLAG_FUSED_FLUSH = 1
 DEVERR = {0: "none", 1: "pos out of range", 2: "buffer capacity", 3: "accepted count out of range",
           4: "bulk copy timeout"}
 
-(FIELD_CKPT, FIELD_CKPT_SCALES, FIELD_OUT_CODES, FIELD_OUT_SCALES, FIELD_XBUF, FIELD_BBUF, FIELD_DTBUF,
- FIELD_POS, FIELD_FLUSH_COUNT, FIELD_ARRIVE, FIELD_ERR) = range(11)
+(FIELD_RECORD, FIELD_CKPT, FIELD_BBUF, FIELD_POS, FIELD_FLUSH_COUNT, FIELD_ARRIVE, FIELD_ERR) = range(7)
 
 
 class Desc(ct.Structure):
@@ -37,8 +36,11 @@ class Desc(ct.Structure):
 
 
 class StateStruct(ct.Structure):
-    _fields_ = [(n, ct.c_void_p) for n in ("ckpt", "ckpt_scales", "out_codes", "out_scales", "xbuf", "bbuf",
-                                           "dtbuf", "pos", "flush_count", "arrive", "err")]
+    _fields_ = [(n, ct.c_void_p) for n in ("record", "ckpt", "bbuf", "pos", "flush_count", "arrive", "err")]
+
+
+class RecordLayout(ct.Structure):
+    _fields_ = [(n, ct.c_uint64) for n in ("bytes", "tile_bytes", "scales_offset", "dt_offset", "x_offset")]
 
 
 class RssmError(RuntimeError):
@@ -66,6 +68,7 @@ def lib():
         "rssm_status_string": ([ct.c_int], ct.c_char_p),
         "rssm_check_desc": ([D], ct.c_int),
         "rssm_state_field_bytes": ([D, i32], ct.c_size_t),
+        "rssm_record_layout": ([D, _P(RecordLayout)], ct.c_int),
         "rssm_decode_step": ([D, S, vp, vp, vp, vp, vp, vp, vp, vp], ct.c_int),
         "rssm_decode_step_noalloc": ([D, S, vp, vp, vp, vp, vp, vp, vp, vp], ct.c_int),
         "rssm_flush": ([D, S, vp, i32, vp], ct.c_int),
@@ -128,17 +131,30 @@ def rssm_state_field_bytes(desc, field):
     return lib().rssm_state_field_bytes(ct.byref(desc), field)
 
 
+def rssm_record_layout(desc):
+    out = RecordLayout()
+    _check(lib().rssm_record_layout(ct.byref(desc), ct.byref(out)), "rssm_record_layout")
+    return out
+
+
 _IN_DT = {RSSM_F32: torch.float32, RSSM_BF16: torch.bfloat16}
 
 
 class RssmState:
     """Per-layer replay state, allocated through PyTorch on the current device.
 
-    Views: ckpt (the update copy: float32 / bfloat16 / uint8 e4m3 / uint8 FP4
-    codes, [batch][H][P][N or N/2]), ckpt_scales, out_codes, out_scales,
-    xbuf [batch][H][cap][P], bbuf [batch][G][cap][N], dtbuf [batch][H][capr]
-    (capr = cap rounded up to a multiple of 4),
-    pos, flush_count, arrive, err. Counters and buffers start at zero."""
+    `record` is the uint8 tensor [batch][H][record bytes] of rssm.h; the
+    other names are views into it or separate fields:
+      ckpt        the update copy [batch][H][P][N] (float32 / bfloat16 /
+                  uint8 e4m3; FP4 shared copy: uint8 codes [..][N/2]) --
+                  inside the records unless there is an FP4 output copy
+      ckpt_scales FP4 shared copy: e4m3 scales [batch][H][P][N/16]
+      out_codes, out_scales  FP4 output copy (inside the records)
+      xbuf [batch][H][cap][P], dtbuf [batch][H][capr] (views into the records;
+      capr = cap rounded up to a multiple of 4), bbuf [batch][G][cap][N],
+      pos, flush_count, arrive, err.
+    Views into the records are strided (not contiguous). Everything starts at
+    zero."""
 
     def __init__(self, desc, device=None):
         _check(rssm_check_desc(desc), "rssm_check_desc")
@@ -149,6 +165,7 @@ class RssmState:
         self.cap = cap
         capr = (cap + 3) // 4 * 4
         in_dt = _IN_DT[desc.in_dtype]
+        self.layout = lay = rssm_record_layout(desc)
 
         def field(f, shape, dtype):
             nbytes = rssm_state_field_bytes(desc, f)
@@ -157,22 +174,34 @@ class RssmState:
             t = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
             return t.view(dtype).view(shape)
 
+        self.record = field(FIELD_RECORD, (B, H, lay.bytes), torch.uint8)
+
+        def part(off, nbytes, dtype, shape):
+            return self.record[:, :, off:off + nbytes].view(dtype).unflatten(-1, shape)
+
         upd = {RSSM_F32: (torch.float32, N), RSSM_BF16: (torch.bfloat16, N), RSSM_E4M3: (torch.uint8, N),
                RSSM_FP4: (torch.uint8, N // 2)}[desc.update_dtype]
-        self.ckpt = field(FIELD_CKPT, (B, H, P, upd[1]), upd[0])
-        self.ckpt_scales = field(FIELD_CKPT_SCALES, (B, H, P, N // 16), torch.uint8)
-        self.out_codes = field(FIELD_OUT_CODES, (B, H, P, N // 2), torch.uint8)
-        self.out_scales = field(FIELD_OUT_SCALES, (B, H, P, N // 16), torch.uint8)
-        self.xbuf = field(FIELD_XBUF, (B, H, cap, P), in_dt)
+        fp4_scales = (lay.scales_offset, P * N // 16, torch.uint8, (P, N // 16))
+        self.ckpt_scales = self.out_codes = self.out_scales = None
+        if desc.out_copy == RSSM_OUTCOPY_FP4:
+            self.ckpt = field(FIELD_CKPT, (B, H, P, upd[1]), upd[0])
+            self.out_codes = part(0, lay.tile_bytes, torch.uint8, (P, N // 2))
+            self.out_scales = part(*fp4_scales)
+        else:
+            self.ckpt = part(0, lay.tile_bytes, upd[0], (P, upd[1]))
+            if desc.update_dtype == RSSM_FP4:
+                self.ckpt_scales = part(*fp4_scales)
+        es = torch.tensor([], dtype=in_dt).element_size()
+        self.xbuf = part(lay.x_offset, cap * P * es, in_dt, (cap, P))
+        self.dtbuf = part(lay.dt_offset, 4 * capr, torch.float32, (capr,))
         self.bbuf = field(FIELD_BBUF, (B, G, cap, N), in_dt)
-        self.dtbuf = field(FIELD_DTBUF, (B, H, capr), torch.float32)
         self.pos = field(FIELD_POS, (B,), torch.int32)
         self.flush_count = field(FIELD_FLUSH_COUNT, (B,), torch.int32)
         self.arrive = field(FIELD_ARRIVE, (B,), torch.int32)
         self.err = field(FIELD_ERR, (1,), torch.int32)
+        sep = self.ckpt if desc.out_copy == RSSM_OUTCOPY_FP4 else None
         self.struct = StateStruct(*[None if t is None else t.data_ptr() for t in (
-            self.ckpt, self.ckpt_scales, self.out_codes, self.out_scales, self.xbuf, self.bbuf, self.dtbuf,
-            self.pos, self.flush_count, self.arrive, self.err)])
+            self.record, sep, self.bbuf, self.pos, self.flush_count, self.arrive, self.err)])
 
 
 def rssm_decode_step(state, x, B, C, dt, A, D, y, stream=None):

@@ -107,17 +107,27 @@ typedef struct rssm_desc {
     uint64_t seed;        /* Philox key of the stochastic rounding */
 } rssm_desc_t;
 
-/* Fields of the per-layer state, for rssm_state_field_bytes. Cap = L + K. */
+/* Fields of the per-layer state, for rssm_state_field_bytes. Cap = L + K,
+ * CapR = Cap rounded up to a multiple of 4.
+ *
+ * RECORD: one record of rssm_record_layout().bytes per (request b, head h),
+ * record (b, h) at byte b*H*bytes + h*bytes, holding
+ *   - at 0: the copy that outputs read, P x N row-major: the fp32 checkpoint;
+ *     the bf16 / e4m3 update copy when that is also what decode reads; or FP4
+ *     codes (element 2k in the low nibble of byte k) followed, at
+ *     .scales_offset, by one e4m3 scale per 16 contiguous d_state elements --
+ *     the FP4 output copy (out_copy) or the shared FP4 copy (update FP4);
+ *   - at .dt_offset: the buffered dt, CapR floats (slots 0..Cap-1 used);
+ *   - at .x_offset: the buffered x, Cap rows of P elements of in_dtype.
+ * Keeping a head's tile, dt and x contiguous lets a decode fetch all three
+ * with one bulk copy.
+ * CKPT: the update copy, only when it is not what decode reads (out_copy
+ *   FP4 with update_dtype F32/BF16/E4M3): [batch][H][P][N] of update_dtype.
+ * BBUF: buffered B, [batch][G][Cap][N] of in_dtype. */
 typedef enum rssm_field {
-    RSSM_FIELD_CKPT = 0,       /* update copy [batch][H][P][N] in update_dtype
-                                  (FP4: codes [batch][H][P][N/2]) */
-    RSSM_FIELD_CKPT_SCALES,    /* FP4 update copy only: e4m3 [batch][H][P][N/16] */
-    RSSM_FIELD_OUT_CODES,      /* FP4 output copy: codes [batch][H][P][N/2] */
-    RSSM_FIELD_OUT_SCALES,     /* FP4 output copy: e4m3 [batch][H][P][N/16] */
-    RSSM_FIELD_XBUF,           /* buffered x  [batch][H][Cap][P] in in_dtype */
-    RSSM_FIELD_BBUF,           /* buffered B  [batch][G][Cap][N] in in_dtype */
-    RSSM_FIELD_DTBUF,          /* buffered dt [batch][H][CapR] float, CapR = Cap rounded
-                                  up to a multiple of 4 (16-byte rows) */
+    RSSM_FIELD_RECORD = 0,
+    RSSM_FIELD_CKPT,
+    RSSM_FIELD_BBUF,
     RSSM_FIELD_POS,            /* int32 [batch]: valid buffer length */
     RSSM_FIELD_FLUSH_COUNT,    /* uint32 [batch]: refreshes so far (Philox counter word) */
     RSSM_FIELD_ARRIVE,         /* uint32 [batch]: scratch, must be zero before first use;
@@ -126,16 +136,20 @@ typedef enum rssm_field {
     RSSM_NUM_FIELDS
 } rssm_field_t;
 
-/* FP4 codes: element 2k in the low nibble of byte k, 2k+1 in the high one.
- * Unused fields may be NULL. */
+/* Byte geometry of one record (see RSSM_FIELD_RECORD). */
+typedef struct rssm_record_layout {
+    uint64_t bytes;          /* record size, a multiple of 128 */
+    uint64_t tile_bytes;     /* bytes of the read copy's values (FP4: codes) */
+    uint64_t scales_offset;  /* FP4 scales (0 when the read copy is not FP4) */
+    uint64_t dt_offset;      /* buffered dt */
+    uint64_t x_offset;       /* buffered x */
+} rssm_record_layout_t;
+
+/* Unused fields may be NULL. */
 typedef struct rssm_state {
+    void *record;
     void *ckpt;
-    void *ckpt_scales;
-    void *out_codes;
-    void *out_scales;
-    void *xbuf;
     void *bbuf;
-    float *dtbuf;
     int32_t *pos;
     uint32_t *flush_count;
     uint32_t *arrive;
@@ -155,9 +169,12 @@ RSSM_API rssm_status_t rssm_check_desc(const rssm_desc_t *desc);
  * or the description is invalid. Host-only; touches no device. */
 RSSM_API size_t rssm_state_field_bytes(const rssm_desc_t *desc, int32_t field);
 
+/* Geometry of one record for this description. Host-only. */
+RSSM_API rssm_status_t rssm_record_layout(const rssm_desc_t *desc, rssm_record_layout_t *out);
+
 /* Standard decode of one token per request (s1): appends (x, B, dt) at
- * slot pos[b], writes y, advances pos[b] by one. Reads the checkpoint (or,
- * with an FP4 output copy, that copy) once; writes no state except the
+ * slot pos[b], writes y, advances pos[b] by one. Reads the record's copy
+ * (the checkpoint, or the FP4 output copy) once; writes no state except the
  * buffer slot. The caller calls rssm_flush / rssm_lowprec_refresh once
  * pos reaches the interval, unless RSSM_FLAG_FUSED_FLUSH is set, in which
  * case the token that fills the buffer also folds it and resets pos.

@@ -60,25 +60,39 @@ def test_check_desc():
 def test_field_bytes():
     d = cfg()
     fb = lambda f: rssm.rssm_state_field_bytes(d, f)
-    assert fb(rssm.FIELD_CKPT) == 256 * 64 * 64 * 128 * 4 == 512 << 20
-    assert fb(rssm.FIELD_CKPT_SCALES) == 0 and fb(rssm.FIELD_OUT_CODES) == 0
-    assert fb(rssm.FIELD_XBUF) == 256 * 64 * 16 * 64 * 2
+    # fp32 checkpoint 64 x 128, dt 16 floats, x 16 rows of 64 bf16: 34880 -> 128-byte multiple
+    lay = rssm.rssm_record_layout(d)
+    assert (lay.tile_bytes, lay.scales_offset, lay.dt_offset, lay.x_offset) == (32768, 0, 32768, 32832)
+    assert lay.bytes == 34944
+    assert fb(rssm.FIELD_RECORD) == 256 * 64 * 34944
+    assert fb(rssm.FIELD_CKPT) == 0
     assert fb(rssm.FIELD_BBUF) == 256 * 8 * 16 * 128 * 2
-    assert fb(rssm.FIELD_DTBUF) == 256 * 64 * 16 * 4
-    assert rssm.rssm_state_field_bytes(cfg(max_draft=1), rssm.FIELD_DTBUF) == 256 * 64 * 20 * 4
     assert fb(rssm.FIELD_POS) == fb(rssm.FIELD_ARRIVE) == 1024 and fb(rssm.FIELD_ERR) == 4
+    # dt rows round the capacity up to a multiple of 4
+    l1 = rssm.rssm_record_layout(cfg(max_draft=1))
+    assert l1.x_offset - l1.dt_offset == 20 * 4
+    # split precision: the record holds the FP4 output copy, the bf16 update copy is separate
     s = cfg(update_dtype=rssm.RSSM_BF16, out_copy=rssm.RSSM_OUTCOPY_FP4, max_draft=4)
     fs = lambda f: rssm.rssm_state_field_bytes(s, f)
+    ls = rssm.rssm_record_layout(s)
+    assert (ls.tile_bytes, ls.scales_offset, ls.dt_offset, ls.x_offset) == (4096, 4096, 4608, 4688)
+    assert ls.bytes == 7296  # 4688 + 20 rows x 64 x 2 = 7248 -> 7296
     assert fs(rssm.FIELD_CKPT) == 256 << 20
-    assert fs(rssm.FIELD_OUT_CODES) == 64 << 20 and fs(rssm.FIELD_OUT_SCALES) == 8 << 20
-    assert fs(rssm.FIELD_XBUF) == 256 * 64 * 20 * 64 * 2
-    assert rssm.rssm_state_field_bytes(cfg(d_state=7), rssm.FIELD_CKPT) == 0
+    assert fs(rssm.FIELD_RECORD) == 256 * 64 * 7296
+    # shared FP4: codes and scales in the record, nothing separate
+    f4 = cfg(update_dtype=rssm.RSSM_FP4, in_dtype=rssm.RSSM_F32)
+    l4 = rssm.rssm_record_layout(f4)
+    assert (l4.scales_offset, l4.dt_offset, l4.x_offset, l4.bytes) == (4096, 4608, 4672, 8832)
+    assert rssm.rssm_state_field_bytes(f4, rssm.FIELD_CKPT) == 0
+    assert rssm.rssm_state_field_bytes(cfg(d_state=7), rssm.FIELD_RECORD) == 0
     assert rssm.rssm_state_field_bytes(d, 99) == 0
+    assert rssm.lib().rssm_record_layout(ct.byref(cfg(d_state=7)), ct.byref(rssm.RecordLayout())) == 2
+    assert rssm.lib().rssm_record_layout(ct.byref(d), None) == 1
 
 
 def fake_state():
     # non-null placeholders: the calls below must fail validation before any device access
-    return rssm.StateStruct(*([0x1000] * 11))
+    return rssm.StateStruct(*([0x1000] * 7))
 
 
 def test_host_validation_needs_no_device(L):
@@ -103,10 +117,13 @@ def test_host_validation_needs_no_device(L):
     assert L.rssm_conv_step(ct.byref(bad), p, p, p, p, p, p, p, p, None) == 2
     assert L.rssm_conv_verify(ct.byref(d), p, p, 8, p, p, p, p, p, p, p, None) == 4
     assert L.rssm_conv_accept(ct.byref(d), None, p, 1, None, None) == 1
-    # missing FP4 copy pointers
+    # a split-precision state needs its separate update copy; every state needs records
     st2 = fake_state()
-    st2.out_codes = None
+    st2.ckpt = None
     assert L.rssm_lowprec_refresh(ct.byref(dl), ct.byref(st2), p, 0, None) == 1
+    st3 = fake_state()
+    st3.record = None
+    assert L.rssm_decode_step(ct.byref(d), ct.byref(st3), p, p, p, p, p, p, p, None) == 1
     assert L.rssm_get_error(ct.byref(d), None, None, None) == 1
     assert L.rssm_round_test(9, 16, p, 0, 0, 0, 0, p, None) == 1
     assert L.rssm_round_test(3, 15, p, 0, 0, 0, 0, p, None) == 2

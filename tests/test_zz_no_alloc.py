@@ -53,7 +53,7 @@ def test_noalloc_decode_matches_decode_step(shape):
 
 def test_noalloc_rejects_batch_above_its_maximum():
     d = rssm.make_desc(65537, 2, 8, 128, 1)
-    st = rssm.StateStruct(*([0x1000] * 11))
+    st = rssm.StateStruct(*([0x1000] * 7))
     p = ct.c_void_p(0x1000)
     status = rssm.lib().rssm_decode_step_noalloc(ct.byref(d), ct.byref(st), p, p, p, p, p, p, p, None)
     assert status == 4  # RSSM_ERR_CAPACITY, nothing launched
