@@ -24,7 +24,6 @@ constexpr int kMaxCap = 32;                 // buffer slots per request (interva
 constexpr int kMaxTok = 8;                  // tokens per verify call (K + 1)
 constexpr int kMidTok = 5;                  // verify kernels specialised for K <= 4
 constexpr int kPipeStagesMax = 8;           // shared-memory stages of the pipelined replay kernel
-constexpr int kConsWarps = 8;               // warps of one consumer group
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bound of one bulk-copy wait
 
 // ------------------------------------------------------------------ errors
@@ -83,6 +82,17 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity, 100000u)) {
         if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+
+// Waits until the shared-memory word *p equals v, at most about limit_ns.
+__device__ __forceinline__ bool smem_wait_eq_bounded(const volatile int* p, int v, uint64_t limit_ns) {
+    if (*p == v) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (*p != v) {
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+        __nanosleep(64);
     }
     return true;
 }

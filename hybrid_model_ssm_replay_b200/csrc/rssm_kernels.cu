@@ -496,8 +496,9 @@ __global__ void __launch_bounds__(kThreads, replay_min_blocks(NT, FUSED)) k_repl
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t fdiv(uint32_t x, const FastDiv& f) { return (__umulhi(x, f.mul) + x) >> f.shr; }
 
-// Barrier of one consumer group (named barrier 1 + gi), returning the OR of v.
-__device__ __forceinline__ int group_sync_or(int gi, int v) {
+// Barrier of one consumer group of nthr threads (named barrier 1 + gi),
+// returning the OR of v.
+__device__ __forceinline__ int group_sync_or(int gi, int nthr, int v) {
     int r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
@@ -505,13 +506,13 @@ __device__ __forceinline__ int group_sync_or(int gi, int v) {
         "bar.red.or.pred q, %2, %3, p;\n\t"
         "selp.s32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"(v), "r"(1 + gi), "r"(kConsWarps * 32)
+        : "r"(v), "r"(1 + gi), "r"(nthr)
         : "memory");
     return r;
 }
 
-__device__ __forceinline__ void group_sync(int gi) {
-    asm volatile("bar.sync %0, %1;" ::"r"(1 + gi), "r"(kConsWarps * 32) : "memory");
+__device__ __forceinline__ void group_sync(int gi, int nthr) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + gi), "r"(nthr) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
@@ -524,17 +525,23 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Consumer groups of the pipelined kernel: two for decode, one for verify
-// (whose K+1 tokens need the registers).
-__host__ __device__ constexpr int pipe_groups(int nt) { return nt == 1 ? 2 : 1; }
-__host__ __device__ constexpr int pipe_threads(int nt) { return (pipe_groups(nt) * kConsWarps + 1) * 32; }
+// Consumer groups of the pipelined kernel and warps per group: groups work
+// on different tiles at once, which hides the latency chain of one tile
+// (barriers, shared-memory loads, shuffle reductions); three for decode, two
+// for verify (whose K+1 tokens need the registers). A group has at least
+// four warps: its B.C products take 8 slots per warp, up to 32 slots.
+__host__ __device__ constexpr int pipe_groups(int nt) { return nt == 1 ? 3 : 2; }
+__host__ __device__ constexpr int pipe_cwarps(int nt) { return (void)nt, 4; }
+__host__ __device__ constexpr int pipe_threads(int nt) { return (pipe_groups(nt) * pipe_cwarps(nt) + 1) * 32; }
 
-// Stage meta: this call's dt [kMaxTok], A_h, D_h (floats), then the position.
-constexpr int kMetaA = kMaxTok, kMetaD = kMaxTok + 1, kMetaPos = kMaxTok + 2;
+// Stage meta (int words): the position and the index k of the tile the
+// stage holds (-1 before its first use).
+constexpr int kMetaPos = 0, kMetaTile = 1;
 
 template <typename TIn, int RF, int NT>
 __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const ReplayArgs a, const PipeLayout lay) {
-    constexpr int CG = pipe_groups(NT);
+    constexpr int CG = pipe_groups(NT), CW = pipe_cwarps(NT), CT = CW * 32;
+    static_assert(CW >= 4, "B.C products need 4 warps of 8 slots");
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full_bar[kPipeStagesMax];
     __shared__ __align__(8) uint64_t empty_bar[kPipeStagesMax];
@@ -553,82 +560,48 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
     if (tid == 0) {
         for (int st = 0; st < S; ++st) {
             mbar_init(smem_u32(&full_bar[st]), 1);
-            mbar_init(smem_u32(&empty_bar[st]), kConsWarps);
+            mbar_init(smem_u32(&empty_bar[st]), CW);
+            reinterpret_cast<int*>(smem + static_cast<size_t>(st) * lay.stage_bytes + lay.meta)[kMetaTile] = -1;
         }
         s_abort = 0;
     }
     __syncthreads();
 
-    if (warp == CG * kConsWarps) {
+    if (warp == CG * CW) {
         // ------------------------------------------------------------ producer
-        // Lane i holds the position, dt, A and D of the i-th tile of the
-        // current batch of 32 tiles (and prefetches the next batch), so no
-        // load latency sits between two issues. Arrivals: lane 1 + k % 31
-        // adds tile k's arrival for its request and checks the returned
-        // count 31 tiles later; the request's last arrival moves pos.
+        // Only what the copies need: the position (lane i holds that of the
+        // i-th tile of the current batch of 32 and loads the next batch, so
+        // no load latency sits between two issues), the record and B-row
+        // addresses, the stage. Everything else is the consumers' work.
         int p0 = 0, p1 = 0;
-        float d0[NT], d1[NT], A0 = 0.f, A1 = 0.f, D0 = 0.f, D1 = 0.f;
-        auto fetch = [&](int kbase, int& pp, float (&dd)[NT], float& AA, float& DD) {
+        auto fetch = [&](int kbase, int& pp) {
             const uint32_t tt = blockIdx.x + static_cast<uint32_t>(kbase + lane) * gridDim.x;
-            if (tt < static_cast<uint32_t>(ntiles)) {
-                const int bb2 = fdiv(tt, lay.divH), hh2 = tt - bb2 * H;
-                pp = a.pos[bb2];
-#pragma unroll
-                for (int j = 0; j < NT; ++j)
-                    dd[j] = (j < ntok) ? a.dt[(static_cast<size_t>(bb2) * ntok + j) * H + hh2] : 0.f;
-                AA = a.A[hh2];
-                DD = a.D[hh2];
-            }
+            if (tt < static_cast<uint32_t>(ntiles)) pp = a.pos[fdiv(tt, lay.divH)];
         };
-        fetch(0, p0, d0, A0, D0);
-        fetch(32, p1, d1, A1, D1);
-        int pend_b = -1, pend_new = 0;
-        uint32_t pend_old = 0;
+        fetch(0, p0);
+        fetch(32, p1);
+        const uint32_t step = gridDim.x;
+        const int dh = static_cast<int>(step % static_cast<uint32_t>(H)), db = static_cast<int>(step / H);
+        int b = fdiv(blockIdx.x, lay.divH), h = static_cast<int>(blockIdx.x) - b * H;
+        const unsigned char* rsrc = a.record + static_cast<size_t>(blockIdx.x) * a.rec.bytes;
+        const size_t rstep = static_cast<size_t>(step) * a.rec.bytes;
+        const size_t brow_bytes = static_cast<size_t>(cap) * N * es;
+        int st = 0, use = 0;
         int k_issued = -1;  // last tile index issued
         bool aborted = false;
-        for (int k = 0;; ++k) {
-            const uint32_t t = blockIdx.x + static_cast<uint32_t>(k) * gridDim.x;
-            if (t >= static_cast<uint32_t>(ntiles)) break;
-            const int b = fdiv(t, lay.divH), h = t - b * H, g = fdiv(h, lay.divHpg);
+        for (int k = 0; blockIdx.x + static_cast<uint32_t>(k) * step < static_cast<uint32_t>(ntiles); ++k) {
             const bool cur = (k >> 5) & 1;
             const int sel = k & 31;
             if (sel == 0 && k > 0) {  // refill the other buffer with the batch after this one
                 if (cur)
-                    fetch(k + 32, p0, d0, A0, D0);
+                    fetch(k + 32, p0);
                 else
-                    fetch(k + 32, p1, d1, A1, D1);
+                    fetch(k + 32, p1);
             }
             // a uniform branch picks the batch, so the warp never reads the
-            // registers of the batch still being fetched
-            int pos;
-            float Ah, Dh, dtj[NT];
-            if (cur) {
-                pos = __shfl_sync(0xffffffffu, p1, sel);
-                Ah = __shfl_sync(0xffffffffu, A1, sel);
-                Dh = __shfl_sync(0xffffffffu, D1, sel);
-#pragma unroll
-                for (int j = 0; j < NT; ++j) dtj[j] = __shfl_sync(0xffffffffu, d1[j], sel);
-            } else {
-                pos = __shfl_sync(0xffffffffu, p0, sel);
-                Ah = __shfl_sync(0xffffffffu, A0, sel);
-                Dh = __shfl_sync(0xffffffffu, D0, sel);
-#pragma unroll
-                for (int j = 0; j < NT; ++j) dtj[j] = __shfl_sync(0xffffffffu, d0[j], sel);
-            }
+            // registers of the batch still being loaded
+            const int pos = cur ? __shfl_sync(0xffffffffu, p1, sel) : __shfl_sync(0xffffffffu, p0, sel);
             const bool ok = pos >= 0 && pos + ntok <= cap;
-            if (a.advance && lane == 1 + (k % 31)) {
-                if (pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 1)) {
-                    a.arrive[pend_b] = 0u;
-                    a.pos[pend_b] = pend_new;
-                }
-                pend_b = -1;
-                if (ok) {
-                    pend_b = b;
-                    pend_new = pos + 1;
-                    pend_old = atomicAdd(&a.arrive[b], 1u);
-                }
-            }
-            const int st = k % S, use = k / S;
             unsigned char* sp = smem + static_cast<size_t>(st) * lay.stage_bytes;
             int live = 1;
             if (lane == 0) {
@@ -645,31 +618,35 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
             }
             if (lane == 0) {
                 const uint32_t fb = smem_u32(&full_bar[st]);
-                float* meta = reinterpret_cast<float*>(sp + lay.meta);
-#pragma unroll
-                for (int j = 0; j < NT; ++j)
-                    if (j < ntok) meta[j] = dtj[j];
-                meta[kMetaA] = Ah;
-                meta[kMetaD] = Dh;
-                reinterpret_cast<int*>(meta)[kMetaPos] = pos;
+                int* meta = reinterpret_cast<int*>(sp + lay.meta);
+                meta[kMetaPos] = pos;
+                reinterpret_cast<volatile int*>(meta)[kMetaTile] = k;
                 // record prefix: copy, scales, dt row and x rows 0..pos-1
                 const uint32_t nrec = a.rec.x + static_cast<uint32_t>(pos * P * es);
                 const uint32_t nb = static_cast<uint32_t>(pos * N * es);
                 mbar_expect_tx(fb, ok ? nrec + nb : 0u);  // nothing to copy for a bad position
                 if (ok) {
-                    const size_t bh = static_cast<size_t>(b) * H + h, bg = static_cast<size_t>(b) * G + g;
-                    bulk_g2s(smem_u32(sp), a.record + bh * a.rec.bytes, nrec, fb);
-                    if (nb > 0)
-                        bulk_g2s(smem_u32(sp + lay.brows), static_cast<const TIn*>(a.bbuf) + bg * cap * N, nb, fb);
+                    bulk_g2s(smem_u32(sp), rsrc, nrec, fb);
+                    if (nb > 0) {
+                        const size_t bg = static_cast<size_t>(b) * G + fdiv(h, lay.divHpg);
+                        bulk_g2s(smem_u32(sp + lay.brows), static_cast<const unsigned char*>(a.bbuf) + bg * brow_bytes,
+                                 nb, fb);
+                    }
                 }
             }
             k_issued = k;
+            rsrc += rstep;
+            h += dh;
+            b += db;
+            if (h >= H) {
+                h -= H;
+                ++b;
+            }
+            if (++st == S) {
+                st = 0;
+                ++use;
+            }
             __syncwarp();
-        }
-        // the arrivals still pending
-        if (a.advance && pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 1)) {
-            a.arrive[pend_b] = 0u;
-            a.pos[pend_b] = pend_new;
         }
         if (aborted && lane == 0) {
             // let every copy this warp issued land before the CTA can exit:
@@ -681,56 +658,87 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
     }
 
     // --------------------------------------------------------------- consumers
-    // Group gi takes tiles k = gi, gi + CG, ...; its 8 warps: warps 0..3 form
-    // the B.C products (8 slots each), warp 7 the decay weights, warps 4..5
-    // append this call's x and B to the buffer, all of them 8 rows each of
-    // the output.
-    const int gi = warp / kConsWarps, cw = warp - gi * kConsWarps;
-    const int ctid = tid - gi * kConsWarps * 32;
-    unsigned char* nbase = smem + static_cast<size_t>(S) * lay.stage_bytes + static_cast<size_t>(gi) * 2 * lay.newrows;
-    // this call's rows of tile kk -> buf: [ntok][P] x, [ntok][N] B, [ntok][N] C, 16-byte chunks
+    // Group gi takes tiles k = gi, gi + CG, ...; its CW warps: warps 0..3
+    // form the B.C products (8 slots each), warp CW-1 the decay weights and
+    // the request's arrival, warp 2 appends this call's x and B to the
+    // buffer, all of them 8 rows at a time of the output.
+    const int gi = warp / CW, cw = warp - gi * CW;
+    const int ctid = tid - gi * CT;
+    unsigned char* nbase = smem + static_cast<size_t>(S) * lay.stage_bytes + static_cast<size_t>(gi) * 3 * lay.newrows;
+    // this call's rows of tile kk -> buf: [ntok][P] x, [ntok][N] B, [ntok][N] C in
+    // 16-byte chunks, then the scalars dt [ntok], A_h, D_h at nd_off
     const int xc = (P * es) >> 4, bc = (N * es) >> 4, per_tok = xc + 2 * bc;
     auto prefetch = [&](int kk, unsigned char* buf) {
         const uint32_t t = blockIdx.x + static_cast<uint32_t>(kk) * gridDim.x;
-        if (t >= static_cast<uint32_t>(ntiles)) return;
-        const int b = fdiv(t, lay.divH), h = t - b * H, g = fdiv(h, lay.divHpg);
-        for (int q = ctid; q < ntok * per_tok; q += kConsWarps * 32) {
-            const int j = q / per_tok;
-            int r = q - j * per_tok;
-            const size_t bj = static_cast<size_t>(b) * ntok + j;
-            const unsigned char* src;
-            uint32_t dst;
-            if (r < xc) {
-                src = reinterpret_cast<const unsigned char*>(static_cast<const TIn*>(a.x) + bj * HP +
-                                                             static_cast<size_t>(h) * P);
-                dst = smem_u32(buf + j * P * es);
-            } else if (r < xc + bc) {
-                r -= xc;
-                src = reinterpret_cast<const unsigned char*>(static_cast<const TIn*>(a.B) + bj * GN +
-                                                             static_cast<size_t>(g) * N);
-                dst = smem_u32(buf + lay.nb_off + j * N * es);
-            } else {
-                r -= xc + bc;
-                src = reinterpret_cast<const unsigned char*>(static_cast<const TIn*>(a.C) + bj * GN +
-                                                             static_cast<size_t>(g) * N);
-                dst = smem_u32(buf + lay.nc_off + j * N * es);
+        if (t < static_cast<uint32_t>(ntiles)) {
+            const int b = fdiv(t, lay.divH), h = t - b * H, g = fdiv(h, lay.divHpg);
+            const int nq = ntok * per_tok;
+            for (int q = ctid; q < nq + ntok + 2; q += CT) {
+                if (q >= nq) {  // scalars, 4 bytes each
+                    const int i = q - nq;
+                    const float* src = i < ntok ? a.dt + (static_cast<size_t>(b) * ntok + i) * H + h
+                                                : (i == ntok ? a.A + h : a.D + h);
+                    const uint32_t dst = smem_u32(buf + lay.nd_off + 4 * (i < ntok ? i : kMaxTok + (i - ntok)));
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+                    continue;
+                }
+                const int j = q / per_tok;
+                int r = q - j * per_tok;
+                const size_t bj = static_cast<size_t>(b) * ntok + j;
+                const unsigned char* src;
+                uint32_t dst;
+                if (r < xc) {
+                    src = reinterpret_cast<const unsigned char*>(static_cast<const TIn*>(a.x) + bj * HP +
+                                                                 static_cast<size_t>(h) * P);
+                    dst = smem_u32(buf + j * P * es);
+                } else if (r < xc + bc) {
+                    r -= xc;
+                    src = reinterpret_cast<const unsigned char*>(static_cast<const TIn*>(a.B) + bj * GN +
+                                                                 static_cast<size_t>(g) * N);
+                    dst = smem_u32(buf + lay.nb_off + j * N * es);
+                } else {
+                    r -= xc + bc;
+                    src = reinterpret_cast<const unsigned char*>(static_cast<const TIn*>(a.C) + bj * GN +
+                                                                 static_cast<size_t>(g) * N);
+                    dst = smem_u32(buf + lay.nc_off + j * N * es);
+                }
+                cp_async16(dst + 16u * r, src + 16 * r);
             }
-            cp_async16(dst + 16u * r, src + 16 * r);
         }
-        cp_async_commit();
+        cp_async_commit();  // one group per tile, empty past the last tile
     };
+    // rows of this group's first two tiles; later tiles two ahead
     prefetch(gi, nbase);
+    prefetch(gi + CG, nbase + lay.newrows);
+    const uint32_t step = static_cast<uint32_t>(CG) * gridDim.x;
+    const int dh = static_cast<int>(step % static_cast<uint32_t>(H)), db = static_cast<int>(step / H);
+    const uint32_t t0 = blockIdx.x + static_cast<uint32_t>(gi) * gridDim.x;
+    int b = fdiv(t0, lay.divH), h = static_cast<int>(t0) - b * H;
+    int st = gi, use = 0;
+    while (st >= S) {
+        st -= S;
+        ++use;
+    }
+    // deferred arrival (warp CW-1, lane 0): the returned count is checked one tile later
+    int pend_b = -1, pend_new = 0;
+    uint32_t pend_old = 0;
     int it = 0;
-    for (int k = gi;; k += CG, ++it) {
-        const uint32_t t = blockIdx.x + static_cast<uint32_t>(k) * gridDim.x;
-        if (t >= static_cast<uint32_t>(ntiles)) break;
-        const int b = fdiv(t, lay.divH), h = t - b * H, g = fdiv(h, lay.divHpg);
+    for (int k = gi; t0 + static_cast<uint32_t>(it) * step < static_cast<uint32_t>(ntiles); k += CG, ++it) {
+        const int g = fdiv(h, lay.divHpg);
         const size_t bh = static_cast<size_t>(b) * H + h, bg = static_cast<size_t>(b) * G + g;
-        const int st = k % S, use = k / S;
         const unsigned char* sp = smem + static_cast<size_t>(st) * lay.stage_bytes;
         int stop = 0;
         if (ctid == 0) {
             stop = s_abort;
+            // The stage's previous use may belong to another group and still
+            // be in flight; once the producer has tagged the stage with this
+            // tile, that use has landed and the parity below names this one.
+            const volatile int* tag = reinterpret_cast<const volatile int*>(sp + lay.meta) + kMetaTile;
+            if (!stop && !smem_wait_eq_bounded(tag, k, kWaitNs)) {
+                set_error(a.err, RSSM_DEVERR_TIMEOUT);  // never tagged: nothing was issued for it
+                s_abort = 1;
+                stop = 1;
+            }
             if (!stop && !mbar_wait_bounded(smem_u32(&full_bar[st]), use & 1, kWaitNs)) {
                 set_error(a.err, RSSM_DEVERR_TIMEOUT);
                 s_abort = 1;
@@ -738,14 +746,13 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
                 mbar_wait_bounded(smem_u32(&full_bar[st]), use & 1, kWaitNs);  // copies in flight
             }
         }
-        cp_async_wait_all();  // this thread's share of this tile's rows
+        asm volatile("cp.async.wait_group 1;" ::: "memory");  // this tile's rows (the next may be in flight)
         // the stage and this tile's rows have landed; this group's previous
-        // readers of s_w / s_g and of the other row buffer are done
-        if (group_sync_or(gi, stop)) break;
-        const unsigned char* nr = nbase + (it & 1) * lay.newrows;
-        prefetch(k + CG, nbase + ((it + 1) & 1) * lay.newrows);
-        const float* meta = reinterpret_cast<const float*>(sp + lay.meta);  // dt[8], A, D, pos
-        const int pos = reinterpret_cast<const int*>(meta)[kMetaPos];
+        // readers of s_w / s_g and of the row buffers are done
+        if (group_sync_or(gi, CT, stop)) break;
+        const unsigned char* nr = nbase + (it % 3) * lay.newrows;
+        const float* sc4 = reinterpret_cast<const float*>(nr + lay.nd_off);  // dt [8], A, D
+        const int pos = reinterpret_cast<const int*>(sp + lay.meta)[kMetaPos];
         const int T = pos + ntok;
         const bool ok = pos >= 0 && T <= cap;
         const TIn* xr = reinterpret_cast<const TIn*>(sp + a.rec.x);     // slot s < pos: xr + s*P
@@ -780,13 +787,13 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
                     }
                 }
             }
-            if (cw == kConsWarps - 1) {
+            if (cw == CW - 1) {
                 const float* dtrow = reinterpret_cast<const float*>(sp + a.rec.dt);
-                const float dnew = (lane >= pos && lane < T) ? meta[lane - pos] : 0.f;
+                const float dnew = (lane >= pos && lane < T) ? sc4[lane - pos] : 0.f;
                 const float dts = (lane < pos) ? dtrow[lane] : dnew;
                 if (lane >= pos && lane < T) reinterpret_cast<float*>(rec + a.rec.dt)[lane] = dnew;
                 const float Sx = warp_prefix(dts);
-                const float Ah = meta[kMetaA];
+                const float Ah = sc4[kMaxTok];
 #pragma unroll
                 for (int j = 0; j < NT; ++j) {
                     if (j < ntok) {
@@ -795,64 +802,104 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
                         if (lane == 0) s_decay[gi][j] = expf(Ah * St);
                     }
                 }
+                if (a.advance && lane == 0) {
+                    // every CTA read pos[b] before it processed b's tiles; the
+                    // request's last arrival moves it
+                    if (pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 1)) {
+                        a.arrive[pend_b] = 0u;
+                        a.pos[pend_b] = pend_new;
+                    }
+                    pend_b = b;
+                    pend_new = pos + 1;
+                    pend_old = atomicAdd(&a.arrive[b], 1u);
+                }
             }
-            if (cw == 4 || cw == 5) {
+            if (cw == 2) {
                 // append this call's x (and, for the group's first head, B) to the buffer
-                const int q0 = ctid - 4 * 32;  // 0..63
                 const int xq = ntok * xc, bq = ntok * bc;
                 uint4* xdst = reinterpret_cast<uint4*>(rec + a.rec.x + static_cast<size_t>(pos) * P * es);
-                for (int q = q0; q < xq; q += 64) xdst[q] = reinterpret_cast<const uint4*>(nx)[q];
+                for (int q = lane; q < xq; q += 32) xdst[q] = reinterpret_cast<const uint4*>(nx)[q];
                 if (h == g * (H / G)) {
                     uint4* bdst = reinterpret_cast<uint4*>(static_cast<TIn*>(a.bbuf) + (bg * cap + pos) * N);
-                    for (int q = q0; q < bq; q += 64) bdst[q] = reinterpret_cast<const uint4*>(nb)[q];
+                    for (int q = lane; q < bq; q += 32) bdst[q] = reinterpret_cast<const uint4*>(nb)[q];
                 }
             }
         }
-        group_sync(gi);  // s_w, s_g, s_decay ready
+        group_sync(gi, CT);  // s_w, s_g, s_decay ready
         if (ok) {
             const unsigned char* tile = sp;
             const unsigned char* sc = sp + a.rec.scales;
-            const float Dh = meta[kMetaD];
+            const float Dh = sc4[kMaxTok + 1];
             float* yout = a.y + static_cast<size_t>(b) * ntok * HP + static_cast<size_t>(h) * P;
             const TIn* xrow = (lane < pos) ? xr + lane * P : nx + (lane - pos) * P;  // slot `lane`
-            for (int r0 = cw * 8; r0 < P; r0 += kConsWarps * 8) {
+            // partials of rows r0..r0+7 for token j: lane l holds columns 4l..4l+3
+            // of h.C and slot l's replay term (zeros past the last row)
+            auto partials = [&](int r0, const float4& cj, float dec, float coef, bool term, float (&part)[8]) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const float4 hv = (r0 + kk < P) ? tile_load4<RF>(tile, sc, r0 + kk, lane, N)
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                    part[kk] = dec * dot4(hv, cj);
+                }
+                if (term && r0 < P) {
+                    Raw8<TIn> xv;
+                    xv.load(xrow + r0);
+                    const float4 xa = xv.lo(), xb = xv.hi();
+                    part[0] = fmaf(coef, xa.x, part[0]);
+                    part[1] = fmaf(coef, xa.y, part[1]);
+                    part[2] = fmaf(coef, xa.z, part[2]);
+                    part[3] = fmaf(coef, xa.w, part[3]);
+                    part[4] = fmaf(coef, xb.x, part[4]);
+                    part[5] = fmaf(coef, xb.y, part[5]);
+                    part[6] = fmaf(coef, xb.z, part[6]);
+                    part[7] = fmaf(coef, xb.w, part[7]);
+                }
+            };
+            // two 8-row blocks per pass, so their reductions overlap
+            for (int r0 = cw * 8; r0 < P; r0 += 2 * CW * 8) {
+                const int r1 = r0 + CW * 8;
 #pragma unroll
                 for (int j = 0; j < NT; ++j) {
                     if (j < ntok) {
                         const int tt = pos + j;
                         const float dec = s_decay[gi][j];
-                        float part[8];
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const float4 hv = (r0 + kk < P) ? tile_load4<RF>(tile, sc, r0 + kk, lane, N)
-                                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-                            part[kk] = dec * dot4(hv, c4[j]);
+                        const bool term = lane <= tt;
+                        const float coef = term ? s_w[gi][j][lane] * s_g[gi][j][lane] : 0.f;
+                        float pa[8], pb[8];
+                        partials(r0, c4[j], dec, coef, term, pa);
+                        partials(r1, c4[j], dec, coef, term, pb);
+                        const float za = warp_reduce8(pa), zb = warp_reduce8(pb);
+                        const int ra = r0 + ((lane >> 2) & 7), rb = r1 + ((lane >> 2) & 7);
+                        if ((lane & 3) == 0) {
+                            if (ra < P) yout[j * HP + ra] = fmaf(Dh, to_f32(nx[j * P + ra]), za);
+                            if (rb < P) yout[j * HP + rb] = fmaf(Dh, to_f32(nx[j * P + rb]), zb);
                         }
-                        if (lane <= tt) {
-                            const float coef = s_w[gi][j][lane] * s_g[gi][j][lane];
-                            Raw8<TIn> xv;
-                            xv.load(xrow + r0);
-                            const float4 xa = xv.lo(), xc4 = xv.hi();
-                            part[0] = fmaf(coef, xa.x, part[0]);
-                            part[1] = fmaf(coef, xa.y, part[1]);
-                            part[2] = fmaf(coef, xa.z, part[2]);
-                            part[3] = fmaf(coef, xa.w, part[3]);
-                            part[4] = fmaf(coef, xc4.x, part[4]);
-                            part[5] = fmaf(coef, xc4.y, part[5]);
-                            part[6] = fmaf(coef, xc4.z, part[6]);
-                            part[7] = fmaf(coef, xc4.w, part[7]);
-                        }
-                        const float z = warp_reduce8(part);
-                        const int r = r0 + ((lane >> 2) & 7);
-                        if ((lane & 3) == 0 && r < P) yout[j * HP + r] = fmaf(Dh, to_f32(nx[j * P + r]), z);
                     }
                 }
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+        // rows of the tile after next, into the buffer this group's previous
+        // tile used (every reader of it passed the barrier above)
+        prefetch(k + 2 * CG, nbase + ((it + 2) % 3) * lay.newrows);
+        h += dh;
+        b += db;
+        if (h >= H) {
+            h -= H;
+            ++b;
+        }
+        st += CG;
+        while (st >= S) {
+            st -= S;
+            ++use;
+        }
     }
     cp_async_wait_all();  // no copy of this thread outlives the CTA
+    if (cw == CW - 1 && lane == 0 && pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 1)) {
+        a.arrive[pend_b] = 0u;  // the last pending arrival of this group
+        a.pos[pend_b] = pend_new;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1261,10 +1308,12 @@ PipeLayout pipe_layout(const Shape& s, const RecLayout& rec, int ntok, int in_bf
     L.stage_bytes = (L.meta + 64u + 127u) & ~127u;
     L.nb_off = align16(static_cast<uint32_t>(ntok * s.P) * es);
     L.nc_off = L.nb_off + align16(static_cast<uint32_t>(ntok * s.N) * es);
-    L.newrows = (L.nc_off + static_cast<uint32_t>(ntok * s.N) * es + 127u) & ~127u;
-    const size_t rows = static_cast<size_t>(groups) * 2u * L.newrows;
+    L.nd_off = L.nc_off + align16(static_cast<uint32_t>(ntok * s.N) * es);
+    L.newrows = (L.nd_off + 4u * (kMaxTok + 2) + 127u) & ~127u;
+    const size_t rows = static_cast<size_t>(groups) * 3u * L.newrows;
     const size_t n = smem_budget > rows ? (smem_budget - rows) / L.stage_bytes : 0;
     L.stages = static_cast<int>(n < static_cast<size_t>(kPipeStagesMax) ? n : kPipeStagesMax);
+    L.budget = smem_budget;
     L.divH = make_fastdiv(static_cast<uint32_t>(s.H));
     L.divHpg = make_fastdiv(static_cast<uint32_t>(s.H / s.G));
     return L;
@@ -1292,7 +1341,8 @@ static DeviceInfo device_info() {
 template <typename TIn, int NT>
 static cudaError_t pipe_dispatch(const ReplayArgs& a, const PipeLayout& L, int rf, int grid, cudaStream_t st) {
     constexpr int thr = pipe_threads(NT);
-    const size_t smem = static_cast<size_t>(L.stages) * L.stage_bytes + 2u * pipe_groups(NT) * L.newrows;
+    const size_t smem = static_cast<size_t>(L.stages) * L.stage_bytes + 3u * pipe_groups(NT) * L.newrows;
+    if (smem > L.budget) return cudaErrorInvalidValue;
     switch (rf) {
         case kF32: return launch_grid(k_replay_pipe<TIn, kF32, NT>, a, L, grid, thr, smem, st);
         case kBF16: return launch_grid(k_replay_pipe<TIn, kBF16, NT>, a, L, grid, thr, smem, st);
@@ -1317,7 +1367,8 @@ cudaError_t launch_replay(const ReplayArgs& a, int in_bf16, int rf, cudaStream_t
     if (!a.fused && a.s.N == 128 && a.s.P % 8 == 0) {
         const DeviceInfo di = device_info();
         if (di.sms > 0) {
-            const size_t budget = di.smem_optin > 4096 ? di.smem_optin - 4096 : 0;
+            // the kernel's static shared memory (barriers, per-group weights) stays below 8 KiB
+            const size_t budget = di.smem_optin > 8192 ? di.smem_optin - 8192 : 0;
             const int groups = a.ntok == 1 ? pipe_groups(1) : pipe_groups(kMidTok);
             const PipeLayout L = pipe_layout(a.s, a.rec, a.ntok, in_bf16, groups, budget);
             if (L.stages >= 2) {
