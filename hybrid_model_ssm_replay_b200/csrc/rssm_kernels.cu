@@ -1059,6 +1059,341 @@ __global__ void __launch_bounds__(kThreads, 4) k_fold(const FoldArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Persistent, warp-specialised fold (flush and refresh) for d_state 128 and
+// head_dim a multiple of 8. The producer warp walks the CTA's tiles, skips
+// the requests that are not due, and brings each due tile into a stage: its
+// update copy and, from the record, dt and the x rows 0..pos-1 (one bulk copy
+// when the update copy is the record's own copy), plus the group's B rows.
+// Consumer groups take the due tiles in turn (stage sequence q = gi, gi+CG,
+// ...; the producer ends each group's sequence with a tile index of -1):
+// weights, B and w_s x_s to fp32 in the group's scratch, then the rank-T
+// update 8 rows x 4 columns per thread and the format's epilogue, stored
+// straight from registers.
+// ---------------------------------------------------------------------------
+struct FoldPipeLayout {
+    uint32_t stage_bytes, st_dt, st_x, brows, meta, scratch;
+    int stages;
+    FastDiv divH, divHpg;
+};
+
+// meta words of a fold stage: tile index (-1: end), position, flush count, A_h, tag
+constexpr int kFMetaTile = 0, kFMetaPos = 1, kFMetaFc = 2, kFMetaA = 3, kFMetaTag = 4;
+
+__host__ __device__ constexpr int fold_groups() { return 3; }
+__host__ __device__ constexpr int fold_cwarps() { return 4; }
+__host__ __device__ constexpr int fold_threads() { return (fold_groups() * fold_cwarps() + 1) * 32; }
+
+template <typename TIn, int UF, int OUT4>
+__global__ void __launch_bounds__(fold_threads(), 1) k_fold_pipe(const FoldArgs a, const FoldPipeLayout lay) {
+    constexpr int CG = fold_groups(), CW = fold_cwarps(), CT = CW * 32;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full_bar[kPipeStagesMax];
+    __shared__ __align__(8) uint64_t empty_bar[kPipeStagesMax];
+    __shared__ float s_cw[CG][kMaxCap];  // dt_s exp(A (S_T - S_s))
+    __shared__ float s_alpha[CG];        // exp(A S_T)
+    __shared__ volatile int s_abort;
+
+    const int H = a.s.H, P = a.s.P, N = a.s.N, G = a.s.G, cap = a.s.cap, L = a.s.L;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int S = lay.stages;
+    const int ntiles = a.s.batch * H;
+    constexpr int es = static_cast<int>(sizeof(TIn));
+    const uint32_t tbu = tile_bytes(UF, P, N) + scale_bytes(UF, P, N);  // update copy (+ FP4 scales)
+    const bool in_record = a.upd == a.record;
+
+    if (tid == 0) {
+        for (int st = 0; st < S; ++st) {
+            mbar_init(smem_u32(&full_bar[st]), 1);
+            mbar_init(smem_u32(&empty_bar[st]), CW);
+            reinterpret_cast<int*>(smem + static_cast<size_t>(st) * lay.stage_bytes + lay.meta)[kFMetaTag] = -1;
+        }
+        s_abort = 0;
+    }
+    __syncthreads();
+
+    if (warp == CG * CW) {
+        // ------------------------------------------------------------ producer
+        int p0 = 0, p1 = 0;
+        uint32_t f0 = 0, f1 = 0;
+        float A0 = 0.f, A1 = 0.f;
+        auto fetch = [&](int kbase, int& pp, uint32_t& ff, float& AA) {
+            const uint32_t tt = blockIdx.x + static_cast<uint32_t>(kbase + lane) * gridDim.x;
+            if (tt < static_cast<uint32_t>(ntiles)) {
+                const int bb = fdiv(tt, lay.divH);
+                pp = a.pos[bb];
+                ff = a.flush_count[bb];
+                AA = a.A[tt - bb * H];
+            }
+        };
+        fetch(0, p0, f0, A0);
+        fetch(32, p1, f1, A1);
+        int q = 0, st = 0, use = 0;  // stage sequence of the due tiles
+        int q_issued = -1;
+        bool aborted = false;
+        // takes the next stage; false when the kernel is aborting
+        auto take_stage = [&]() {
+            int live = 1;
+            if (lane == 0) {
+                if (use > 0 && !mbar_wait_bounded(smem_u32(&empty_bar[st]), (use - 1) & 1, kWaitNs)) {
+                    set_error(a.err, RSSM_DEVERR_TIMEOUT);
+                    s_abort = 1;
+                }
+                live = !s_abort;
+            }
+            return __shfl_sync(0xffffffffu, live, 0) != 0;
+        };
+        auto next_stage = [&]() {
+            q_issued = q;
+            ++q;
+            if (++st == S) {
+                st = 0;
+                ++use;
+            }
+        };
+        for (int k = 0; blockIdx.x + static_cast<uint32_t>(k) * gridDim.x < static_cast<uint32_t>(ntiles); ++k) {
+            const uint32_t t = blockIdx.x + static_cast<uint32_t>(k) * gridDim.x;
+            const bool cur = (k >> 5) & 1;
+            const int sel = k & 31;
+            if (sel == 0 && k > 0) {
+                if (cur)
+                    fetch(k + 32, p0, f0, A0);
+                else
+                    fetch(k + 32, p1, f1, A1);
+            }
+            int pos;
+            uint32_t fc;
+            float Ah;
+            if (cur) {
+                pos = __shfl_sync(0xffffffffu, p1, sel);
+                fc = __shfl_sync(0xffffffffu, f1, sel);
+                Ah = __shfl_sync(0xffffffffu, A1, sel);
+            } else {
+                pos = __shfl_sync(0xffffffffu, p0, sel);
+                fc = __shfl_sync(0xffffffffu, f0, sel);
+                Ah = __shfl_sync(0xffffffffu, A0, sel);
+            }
+            if (pos < 0 || pos > cap) {
+                if (lane == 0) set_error(a.err, RSSM_DEVERR_POS_RANGE);
+                continue;
+            }
+            if (!((pos >= L) || (a.mode >= 1 && pos > 0) || (a.mode == 2))) continue;  // not due
+            if (!take_stage()) {
+                aborted = true;
+                break;
+            }
+            if (lane == 0) {
+                unsigned char* sp = smem + static_cast<size_t>(st) * lay.stage_bytes;
+                const uint32_t fb = smem_u32(&full_bar[st]);
+                int* meta = reinterpret_cast<int*>(sp + lay.meta);
+                meta[kFMetaTile] = static_cast<int>(t);
+                meta[kFMetaPos] = pos;
+                meta[kFMetaFc] = static_cast<int>(fc);
+                reinterpret_cast<float*>(meta)[kFMetaA] = Ah;
+                reinterpret_cast<volatile int*>(meta)[kFMetaTag] = q;
+                const int b = fdiv(t, lay.divH), h = static_cast<int>(t) - b * H;
+                const unsigned char* rec = a.record + static_cast<size_t>(t) * a.rec.bytes;
+                const uint32_t nx = static_cast<uint32_t>(pos * P * es), nb = static_cast<uint32_t>(pos * N * es);
+                const uint32_t ndx = (a.rec.x - a.rec.dt) + nx;  // dt row and x rows, contiguous in the record
+                mbar_expect_tx(fb, (in_record ? a.rec.x + nx : tbu + ndx) + nb);
+                if (in_record) {
+                    bulk_g2s(smem_u32(sp), rec, a.rec.x + nx, fb);
+                } else {
+                    bulk_g2s(smem_u32(sp), a.upd + static_cast<size_t>(t) * a.upd_stride, tbu, fb);
+                    bulk_g2s(smem_u32(sp + lay.st_dt), rec + a.rec.dt, ndx, fb);
+                }
+                if (nb > 0) {
+                    const size_t bg = static_cast<size_t>(b) * G + fdiv(h, lay.divHpg);
+                    bulk_g2s(smem_u32(sp + lay.brows),
+                             static_cast<const unsigned char*>(a.bbuf) + bg * static_cast<size_t>(cap) * N * es, nb,
+                             fb);
+                }
+            }
+            next_stage();
+            __syncwarp();
+        }
+        // one end marker per consumer group
+        for (int e = 0; e < CG && !aborted; ++e) {
+            if (!take_stage()) {
+                aborted = true;
+                break;
+            }
+            if (lane == 0) {
+                unsigned char* sp = smem + static_cast<size_t>(st) * lay.stage_bytes;
+                int* meta = reinterpret_cast<int*>(sp + lay.meta);
+                meta[kFMetaTile] = -1;
+                reinterpret_cast<volatile int*>(meta)[kFMetaTag] = q;
+                mbar_expect_tx(smem_u32(&full_bar[st]), 0u);
+            }
+            next_stage();
+            __syncwarp();
+        }
+        if (aborted && lane == 0) {
+            for (int qq = q_issued; qq >= 0 && qq > q_issued - S; --qq)
+                mbar_wait_bounded(smem_u32(&full_bar[qq % S]), (qq / S) & 1, kWaitNs);
+        }
+        return;
+    }
+
+    // --------------------------------------------------------------- consumers
+    const int gi = warp / CW, cw = warp - gi * CW;
+    const int ctid = tid - gi * CT;
+    float* s_Bf = reinterpret_cast<float*>(smem + static_cast<size_t>(S) * lay.stage_bytes +
+                                           static_cast<size_t>(gi) * lay.scratch);  // [T][N]
+    float* s_xw = s_Bf + cap * N;                                                    // [T][P]
+    const int bq = N / 8, xq = P / 8;  // 8-element chunks per B row / x row
+    int st = gi, use = 0;
+    while (st >= S) {
+        st -= S;
+        ++use;
+    }
+    int pend_b = -1;
+    uint32_t pend_old = 0;
+    for (int q = gi;; q += CG) {
+        const unsigned char* sp = smem + static_cast<size_t>(st) * lay.stage_bytes;
+        const int* meta = reinterpret_cast<const int*>(sp + lay.meta);
+        int stop = 0;
+        if (ctid == 0) {
+            stop = s_abort;
+            const volatile int* tag = reinterpret_cast<const volatile int*>(meta) + kFMetaTag;
+            if (!stop && !smem_wait_eq_bounded(tag, q, kWaitNs)) {
+                set_error(a.err, RSSM_DEVERR_TIMEOUT);
+                s_abort = 1;
+                stop = 1;
+            }
+            if (!stop && !mbar_wait_bounded(smem_u32(&full_bar[st]), use & 1, kWaitNs)) {
+                set_error(a.err, RSSM_DEVERR_TIMEOUT);
+                s_abort = 1;
+                stop = 1;
+                mbar_wait_bounded(smem_u32(&full_bar[st]), use & 1, kWaitNs);
+            }
+        }
+        if (group_sync_or(gi, CT, stop)) break;
+        const int t = meta[kFMetaTile];
+        if (t < 0) {  // end of this group's sequence: hand the stage back and stop
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+            break;
+        }
+        const int T = meta[kFMetaPos];
+        const uint32_t fc = static_cast<uint32_t>(meta[kFMetaFc]);
+        const float Ah = reinterpret_cast<const float*>(meta)[kFMetaA];
+        const int b = fdiv(static_cast<uint32_t>(t), lay.divH), h = t - b * H;
+        const TIn* xr = reinterpret_cast<const TIn*>(sp + lay.st_x);
+        const TIn* br = reinterpret_cast<const TIn*>(sp + lay.brows);
+        if (cw == CW - 1) {
+            const float dts = (lane < T) ? reinterpret_cast<const float*>(sp + lay.st_dt)[lane] : 0.f;
+            const float Sx = warp_prefix(dts);
+            const float Stot = T > 0 ? __shfl_sync(0xffffffffu, Sx, T - 1) : 0.f;
+            s_cw[gi][lane] = (lane < T) ? dts * expf(Ah * (Stot - Sx)) : 0.f;
+            if (lane == 0) s_alpha[gi] = expf(Ah * Stot);
+            if (lane == 0) {
+                // every CTA read pos[b] before processing b's tiles; the last arrival resets it
+                if (pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 1)) {
+                    a.arrive[pend_b] = 0u;
+                    a.pos[pend_b] = 0;
+                    a.flush_count[pend_b] += 1u;
+                }
+                pend_b = b;
+                pend_old = atomicAdd(&a.arrive[b], 1u);
+            }
+        } else {
+            // B rows to fp32
+            for (int c = ctid; c < T * bq; c += (CW - 1) * 32) {
+                Raw8<TIn> r;
+                r.load(br + c * 8);
+                reinterpret_cast<float4*>(s_Bf)[2 * c] = r.lo();
+                reinterpret_cast<float4*>(s_Bf)[2 * c + 1] = r.hi();
+            }
+        }
+        group_sync(gi, CT);  // weights and B ready
+        const float alpha = s_alpha[gi];
+        for (int c = ctid; c < T * xq; c += CT) {
+            const int sl = c / xq;
+            const float w = s_cw[gi][sl];
+            Raw8<TIn> r;
+            r.load(xr + c * 8);
+            const float4 lo = r.lo(), hi = r.hi();
+            reinterpret_cast<float4*>(s_xw)[2 * c] = make_float4(w * lo.x, w * lo.y, w * lo.z, w * lo.w);
+            reinterpret_cast<float4*>(s_xw)[2 * c + 1] = make_float4(w * hi.x, w * hi.y, w * hi.z, w * hi.w);
+        }
+        group_sync(gi, CT);  // w_s x_s ready
+        const unsigned char* tile = sp;
+        const unsigned char* tsc = sp + (in_record ? a.rec.scales : align16(tile_bytes(UF, P, N)));
+        unsigned char* upd = a.upd + static_cast<size_t>(t) * a.upd_stride;
+        unsigned char* rec = a.record + static_cast<size_t>(t) * a.rec.bytes;
+        for (int r0 = cw * kRB; r0 < P; r0 += CW * kRB) {
+            float4 acc[kRB];
+#pragma unroll
+            for (int kk = 0; kk < kRB; ++kk) acc[kk] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+            for (int sl = 0; sl < T; ++sl) {
+                const float4 bv = reinterpret_cast<const float4*>(s_Bf + sl * N)[lane];
+                const float4* xw4 = reinterpret_cast<const float4*>(s_xw + sl * P + r0);
+                const float4 xa = xw4[0], xb = xw4[1];
+                const float w[kRB] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+                for (int kk = 0; kk < kRB; ++kk) {
+                    acc[kk].x = fmaf(w[kk], bv.x, acc[kk].x);
+                    acc[kk].y = fmaf(w[kk], bv.y, acc[kk].y);
+                    acc[kk].z = fmaf(w[kk], bv.z, acc[kk].z);
+                    acc[kk].w = fmaf(w[kk], bv.w, acc[kk].w);
+                }
+            }
+#pragma unroll
+            for (int kk = 0; kk < kRB; ++kk) {
+                const int r = r0 + kk;
+                const float4 hv = tile_load4<UF>(tile, tsc, r, lane, N);
+                float4 v;
+                v.x = fmaf(alpha, hv.x, acc[kk].x);
+                v.y = fmaf(alpha, hv.y, acc[kk].y);
+                v.z = fmaf(alpha, hv.z, acc[kk].z);
+                v.w = fmaf(alpha, hv.w, acc[kk].w);
+                const uint32_t e = static_cast<uint32_t>(r * N + 4 * lane);  // element of v.x within the head
+                if constexpr (UF == kF32) {
+                    stream_store4(reinterpret_cast<float*>(upd) + e, v);
+                } else if constexpr (UF == kBF16 || UF == kE4M3) {
+                    const uint4 rw = philox4x32_10(make_uint4(e >> 2, h, b, fc),
+                                                   make_uint2(static_cast<uint32_t>(a.seed),
+                                                              static_cast<uint32_t>(a.seed >> 32)));
+                    if constexpr (UF == kBF16) {
+                        const uint2 wv = make_uint2(sr_bf16(v.x, rw.x) | (sr_bf16(v.y, rw.y) << 16),
+                                                    sr_bf16(v.z, rw.z) | (sr_bf16(v.w, rw.w) << 16));
+                        *reinterpret_cast<uint2*>(upd + 2u * e) = wv;
+                    } else {
+                        const uint32_t wv = sr_e4m3(v.x, rw.x) | (sr_e4m3(v.y, rw.y) << 8) |
+                                            (sr_e4m3(v.z, rw.z) << 16) | (sr_e4m3(v.w, rw.w) << 24);
+                        *reinterpret_cast<uint32_t*>(upd + e) = wv;
+                    }
+                } else {
+                    uint32_t scv;
+                    const uint32_t codes = fp4_quant_quad(v, &scv);
+                    *reinterpret_cast<uint16_t*>(upd + e / 2) = static_cast<uint16_t>(codes);
+                    if ((lane & 3) == 0) upd[a.rec.scales + e / 16] = static_cast<uint8_t>(scv);
+                }
+                if constexpr (OUT4 != 0) {
+                    uint32_t scv;
+                    const uint32_t codes = fp4_quant_quad(v, &scv);
+                    *reinterpret_cast<uint16_t*>(rec + e / 2) = static_cast<uint16_t>(codes);
+                    if ((lane & 3) == 0) rec[a.rec.scales + e / 16] = static_cast<uint8_t>(scv);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+        st += CG;
+        while (st >= S) {
+            st -= S;
+            ++use;
+        }
+    }
+    if (cw == CW - 1 && lane == 0 && pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 1)) {
+        a.arrive[pend_b] = 0u;  // the last pending arrival of this group
+        a.pos[pend_b] = 0;
+        a.flush_count[pend_b] += 1u;
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Conventional scheme (in-run comparison, s1/s3): per token
 //   h <- exp(dt A) h + dt x B^T, write h, y = h C + D x.
 // VERIFY: read copy cur[b], write the state after token j to copy j.
@@ -1408,7 +1743,76 @@ static cudaError_t fold_dispatch(const FoldArgs& a, int uf, size_t smem, int nbl
     }
 }
 
+template <typename TIn>
+static cudaError_t fold_pipe_dispatch(const FoldArgs& a, const FoldPipeLayout& L, int uf, int grid, size_t smem,
+                                      cudaStream_t st) {
+    auto go = [&](auto kernel) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 static_cast<int>(cudaSharedmemCarveoutMaxShared));
+        if (e != cudaSuccess) return e;
+        kernel<<<grid, fold_threads(), smem, st>>>(a, L);
+        return cudaGetLastError();
+    };
+    if (a.out_fp4) {
+        switch (uf) {
+            case kF32: return go(k_fold_pipe<TIn, kF32, 1>);
+            case kBF16: return go(k_fold_pipe<TIn, kBF16, 1>);
+            case kE4M3: return go(k_fold_pipe<TIn, kE4M3, 1>);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    switch (uf) {
+        case kF32: return go(k_fold_pipe<TIn, kF32, 0>);
+        case kBF16: return go(k_fold_pipe<TIn, kBF16, 0>);
+        case kE4M3: return go(k_fold_pipe<TIn, kE4M3, 0>);
+        default: return go(k_fold_pipe<TIn, kFP4, 0>);
+    }
+}
+
+// Stage layout of k_fold_pipe: update copy (+ scales), dt row and x rows
+// (at the record's offsets when the update copy is the record's own copy),
+// B rows, meta; per consumer group a scratch of fp32 B and w x rows.
+static FoldPipeLayout fold_pipe_layout(const FoldArgs& a, int uf, int in_bf16, size_t budget) {
+    const Shape& s = a.s;
+    const uint32_t es = in_bf16 ? 2u : 4u;
+    FoldPipeLayout L;
+    if (a.upd == a.record) {
+        L.st_dt = a.rec.dt;
+        L.st_x = a.rec.x;
+    } else {
+        L.st_dt = align16(align16(tile_bytes(uf, s.P, s.N)) + scale_bytes(uf, s.P, s.N));
+        L.st_x = L.st_dt + (a.rec.x - a.rec.dt);
+    }
+    L.brows = align16(L.st_x + static_cast<uint32_t>(s.cap * s.P) * es);
+    L.meta = L.brows + align16(static_cast<uint32_t>(s.cap * s.N) * es);
+    L.stage_bytes = (L.meta + 64u + 127u) & ~127u;
+    L.scratch = (4u * static_cast<uint32_t>(s.cap) * (s.N + s.P) + 127u) & ~127u;
+    const size_t rows = static_cast<size_t>(fold_groups()) * L.scratch;
+    const size_t n = budget > rows ? (budget - rows) / L.stage_bytes : 0;
+    L.stages = static_cast<int>(n < static_cast<size_t>(kPipeStagesMax) ? n : kPipeStagesMax);
+    L.divH = make_fastdiv(static_cast<uint32_t>(s.H));
+    L.divHpg = make_fastdiv(static_cast<uint32_t>(s.H / s.G));
+    return L;
+}
+
 cudaError_t launch_fold(const FoldArgs& a, int in_bf16, int uf, cudaStream_t st) {
+    if (a.s.N == 128 && a.s.P % 8 == 0) {
+        const DeviceInfo di = device_info();
+        if (di.sms > 0) {
+            const size_t budget = di.smem_optin > 8192 ? di.smem_optin - 8192 : 0;
+            const FoldPipeLayout L = fold_pipe_layout(a, uf, in_bf16, budget);
+            if (L.stages >= 2) {
+                const int ntiles = a.s.batch * a.s.H;
+                const int grid = ntiles < di.sms ? ntiles : di.sms;
+                const size_t smem = static_cast<size_t>(L.stages) * L.stage_bytes +
+                                    static_cast<size_t>(fold_groups()) * L.scratch;
+                return in_bf16 ? fold_pipe_dispatch<__nv_bfloat16>(a, L, uf, grid, smem, st)
+                               : fold_pipe_dispatch<float>(a, L, uf, grid, smem, st);
+            }
+        }
+    }
     const size_t smem = fold_smem_bytes(a.s, uf);
     const int nblk = a.s.batch * a.s.H;
     return in_bf16 ? fold_dispatch<__nv_bfloat16>(a, uf, smem, nblk, st) : fold_dispatch<float>(a, uf, smem, nblk, st);

@@ -67,9 +67,13 @@ def fp4_control_state(shape, inp, seed):
     return desc, st
 
 
+# d_state 64 runs the one-CTA-per-tile fold, d_state 128 the persistent pipelined one
+SHAPES = [LayerShape(3, 4, 32, 64, 2), LayerShape(3, 4, 32, 128, 2)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=["dstate64", "dstate128"])
 @pytest.mark.parametrize("kind", ["bf16", "e4m3", "f32"])
-def test_refresh_at_empty_buffer_builds_fp4_copy_bit_exact(kind):
-    shape = LayerShape(3, 4, 32, 64, 2)
+def test_refresh_at_empty_buffer_builds_fp4_copy_bit_exact(kind, shape):
     inp = make_inputs(shape, 1, 30, torch.bfloat16, device="cuda")
     desc, st = split_state(shape, inp, kind, 99)
     upd0 = copy_bits(initial_update_copy(inp["ckpt"], kind))
@@ -142,8 +146,8 @@ def test_fp4_decode_and_refresh_match_oracle(kind):
     assert st.flush_count.cpu().tolist() == [2] * 4
 
 
-def test_shared_fp4_control_decode_matches_oracle():
-    shape = LayerShape(3, 4, 32, 64, 2)
+@pytest.mark.parametrize("shape", SHAPES, ids=["dstate64", "dstate128"])
+def test_shared_fp4_control_decode_matches_oracle(shape):
     L = shape.interval
     inp = make_inputs(shape, L, 32, torch.bfloat16, device="cuda")
     desc, st = fp4_control_state(shape, inp, 5)
@@ -152,6 +156,7 @@ def test_shared_fp4_control_decode_matches_oracle():
     for t in range(L):
         rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"], y[t])
     rssm.rssm_lowprec_refresh(st, inp["A"])
+    assert rssm.rssm_get_error(st) == 0
     for b in range(3):
         r = request_inputs(inp, b)
         req = orc.LowPrecRequest(orc.FP4, False, None, codes0[b], scales0[b], 2, L, r["A"], r["D"], 5, b)
