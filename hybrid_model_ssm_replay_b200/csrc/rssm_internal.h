@@ -71,6 +71,7 @@ inline FastDiv make_fastdiv(uint32_t d) {
 // [ntok][N] at 0, nb_off, nc_off) and its dt [8], A_h, D_h (at nd_off).
 struct PipeLayout {
     uint32_t stage_bytes, brows, meta, newrows, nb_off, nc_off, nd_off;
+    uint32_t xw_bytes;  // fused fold: per-group fp32 w_s x_s scratch (0 otherwise)
     int stages;
     size_t budget;  // dynamic shared memory the layout may use
     FastDiv divH, divHpg;  // tile -> (request, head), head -> group

@@ -538,9 +538,10 @@ __host__ __device__ constexpr int pipe_threads(int nt) { return (pipe_groups(nt)
 // stage holds (-1 before its first use).
 constexpr int kMetaPos = 0, kMetaTile = 1;
 
-template <typename TIn, int RF, int NT>
+template <typename TIn, int RF, int NT, int FUSED>
 __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const ReplayArgs a, const PipeLayout lay) {
     constexpr int CG = pipe_groups(NT), CW = pipe_cwarps(NT), CT = CW * 32;
+    static_assert(!FUSED || (RF == kF32 && NT == 1), "the fused fold is for fp32 decode");
     static_assert(CW >= 4, "B.C products need 4 warps of 8 slots");
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full_bar[kPipeStagesMax];
@@ -665,6 +666,10 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
     const int gi = warp / CW, cw = warp - gi * CW;
     const int ctid = tid - gi * CT;
     unsigned char* nbase = smem + static_cast<size_t>(S) * lay.stage_bytes + static_cast<size_t>(gi) * 3 * lay.newrows;
+    // fused fold: w_s x_s in fp32, [cap][P], per group after the row buffers
+    float* s_xw = reinterpret_cast<float*>(smem + static_cast<size_t>(S) * lay.stage_bytes +
+                                           static_cast<size_t>(CG) * 3 * lay.newrows +
+                                           static_cast<size_t>(gi) * lay.xw_bytes);
     // this call's rows of tile kk -> buf: [ntok][P] x, [ntok][N] B, [ntok][N] C in
     // 16-byte chunks, then the scalars dt [ntok], A_h, D_h at nd_off
     const int xc = (P * es) >> 4, bc = (N * es) >> 4, per_tok = xc + 2 * bc;
@@ -721,6 +726,7 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
     }
     // deferred arrival (warp CW-1, lane 0): the returned count is checked one tile later
     int pend_b = -1, pend_new = 0;
+    bool pend_bump = false;
     uint32_t pend_old = 0;
     int it = 0;
     for (int k = gi; t0 + static_cast<uint32_t>(it) * step < static_cast<uint32_t>(ntiles); k += CG, ++it) {
@@ -804,13 +810,15 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
                 }
                 if (a.advance && lane == 0) {
                     // every CTA read pos[b] before it processed b's tiles; the
-                    // request's last arrival moves it
+                    // request's last arrival moves it (to 0 after a fused fold)
                     if (pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 1)) {
                         a.arrive[pend_b] = 0u;
                         a.pos[pend_b] = pend_new;
+                        if (pend_bump) a.flush_count[pend_b] += 1u;
                     }
                     pend_b = b;
-                    pend_new = pos + 1;
+                    pend_bump = FUSED && T == a.s.L;
+                    pend_new = pend_bump ? 0 : pos + 1;
                     pend_old = atomicAdd(&a.arrive[b], 1u);
                 }
             }
@@ -878,6 +886,51 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
                 }
             }
         }
+        if constexpr (FUSED != 0) {
+            if (ok && T == a.s.L) {  // uniform over the group: the token that fills the buffer folds it
+                // h <- exp(A S_T) h + sum_s w_s x_s B_s^T with w_s = s_w[gi][0][s]
+                // (t = pos = T - 1), written over the checkpoint in the record
+                const int x8 = P >> 3;
+                for (int c = ctid; c < T * x8; c += CT) {
+                    const int sl = c / x8, p8 = (c - sl * x8) << 3;
+                    Raw8<TIn> r;
+                    r.load((sl < pos ? xr + sl * P : nx) + p8);
+                    const float w = s_w[gi][0][sl];
+                    const float4 lo = r.lo(), hi = r.hi();
+                    float4* d = reinterpret_cast<float4*>(s_xw + sl * P + p8);
+                    d[0] = make_float4(w * lo.x, w * lo.y, w * lo.z, w * lo.w);
+                    d[1] = make_float4(w * hi.x, w * hi.y, w * hi.z, w * hi.w);
+                }
+                group_sync(gi, CT);
+                const float alpha = s_decay[gi][0];
+                float* ck = reinterpret_cast<float*>(rec);
+                for (int r0 = cw * kRB; r0 < P; r0 += CW * kRB) {
+                    // acc = alpha h, then the slots in order (as the flush kernels)
+                    float4 acc[kRB];
+#pragma unroll
+                    for (int kk = 0; kk < kRB; ++kk) {
+                        const float4 hv = reinterpret_cast<const float4*>(sp)[(r0 + kk) * (N >> 2) + lane];
+                        acc[kk] = make_float4(alpha * hv.x, alpha * hv.y, alpha * hv.z, alpha * hv.w);
+                    }
+#pragma unroll 2
+                    for (int sl = 0; sl < T; ++sl) {
+                        const float4 bv = load4((sl < pos ? br + sl * N : nb) + 4 * lane);
+                        const float4* xw4 = reinterpret_cast<const float4*>(s_xw + sl * P + r0);
+                        const float4 xa = xw4[0], xb = xw4[1];
+                        const float w[kRB] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+                        for (int kk = 0; kk < kRB; ++kk) {
+                            acc[kk].x = fmaf(w[kk], bv.x, acc[kk].x);
+                            acc[kk].y = fmaf(w[kk], bv.y, acc[kk].y);
+                            acc[kk].z = fmaf(w[kk], bv.z, acc[kk].z);
+                            acc[kk].w = fmaf(w[kk], bv.w, acc[kk].w);
+                        }
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < kRB; ++kk) stream_store4(ck + (r0 + kk) * N + 4 * lane, acc[kk]);
+                }
+            }
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
         // rows of the tile after next, into the buffer this group's previous
@@ -899,6 +952,7 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
     if (cw == CW - 1 && lane == 0 && pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 1)) {
         a.arrive[pend_b] = 0u;  // the last pending arrival of this group
         a.pos[pend_b] = pend_new;
+        if (pend_bump) a.flush_count[pend_b] += 1u;
     }
 }
 
@@ -1322,9 +1376,13 @@ __global__ void __launch_bounds__(fold_threads(), 1) k_fold_pipe(const FoldArgs 
         unsigned char* upd = a.upd + static_cast<size_t>(t) * a.upd_stride;
         unsigned char* rec = a.record + static_cast<size_t>(t) * a.rec.bytes;
         for (int r0 = cw * kRB; r0 < P; r0 += CW * kRB) {
+            // acc = alpha h, then the slots in order (the one-CTA fold's order)
             float4 acc[kRB];
 #pragma unroll
-            for (int kk = 0; kk < kRB; ++kk) acc[kk] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int kk = 0; kk < kRB; ++kk) {
+                const float4 hv = tile_load4<UF>(tile, tsc, r0 + kk, lane, N);
+                acc[kk] = make_float4(alpha * hv.x, alpha * hv.y, alpha * hv.z, alpha * hv.w);
+            }
 #pragma unroll 2
             for (int sl = 0; sl < T; ++sl) {
                 const float4 bv = reinterpret_cast<const float4*>(s_Bf + sl * N)[lane];
@@ -1342,12 +1400,7 @@ __global__ void __launch_bounds__(fold_threads(), 1) k_fold_pipe(const FoldArgs 
 #pragma unroll
             for (int kk = 0; kk < kRB; ++kk) {
                 const int r = r0 + kk;
-                const float4 hv = tile_load4<UF>(tile, tsc, r, lane, N);
-                float4 v;
-                v.x = fmaf(alpha, hv.x, acc[kk].x);
-                v.y = fmaf(alpha, hv.y, acc[kk].y);
-                v.z = fmaf(alpha, hv.z, acc[kk].z);
-                v.w = fmaf(alpha, hv.w, acc[kk].w);
+                const float4 v = acc[kk];
                 const uint32_t e = static_cast<uint32_t>(r * N + 4 * lane);  // element of v.x within the head
                 if constexpr (UF == kF32) {
                     stream_store4(reinterpret_cast<float*>(upd) + e, v);
@@ -1635,7 +1688,8 @@ RecLayout record_layout(const Shape& s, int rf, int in_bytes) {
 
 // Stage layout of k_replay_pipe (16-byte aligned pieces, 128-byte aligned
 // stages and row buffers); the stages fill what the row buffers leave.
-PipeLayout pipe_layout(const Shape& s, const RecLayout& rec, int ntok, int in_bf16, int groups, size_t smem_budget) {
+PipeLayout pipe_layout(const Shape& s, const RecLayout& rec, int ntok, int in_bf16, int groups, int fused,
+                       size_t smem_budget) {
     const uint32_t es = in_bf16 ? 2u : 4u;
     PipeLayout L;
     L.brows = align16(rec.x + static_cast<uint32_t>(s.cap * s.P) * es);
@@ -1645,7 +1699,8 @@ PipeLayout pipe_layout(const Shape& s, const RecLayout& rec, int ntok, int in_bf
     L.nc_off = L.nb_off + align16(static_cast<uint32_t>(ntok * s.N) * es);
     L.nd_off = L.nc_off + align16(static_cast<uint32_t>(ntok * s.N) * es);
     L.newrows = (L.nd_off + 4u * (kMaxTok + 2) + 127u) & ~127u;
-    const size_t rows = static_cast<size_t>(groups) * 3u * L.newrows;
+    L.xw_bytes = fused ? (4u * static_cast<uint32_t>(s.cap * s.P) + 127u) & ~127u : 0u;
+    const size_t rows = static_cast<size_t>(groups) * (3u * L.newrows + L.xw_bytes);
     const size_t n = smem_budget > rows ? (smem_budget - rows) / L.stage_bytes : 0;
     L.stages = static_cast<int>(n < static_cast<size_t>(kPipeStagesMax) ? n : kPipeStagesMax);
     L.budget = smem_budget;
@@ -1676,13 +1731,20 @@ static DeviceInfo device_info() {
 template <typename TIn, int NT>
 static cudaError_t pipe_dispatch(const ReplayArgs& a, const PipeLayout& L, int rf, int grid, cudaStream_t st) {
     constexpr int thr = pipe_threads(NT);
-    const size_t smem = static_cast<size_t>(L.stages) * L.stage_bytes + 3u * pipe_groups(NT) * L.newrows;
+    const size_t smem = static_cast<size_t>(L.stages) * L.stage_bytes +
+                        static_cast<size_t>(pipe_groups(NT)) * (3u * L.newrows + L.xw_bytes);
     if (smem > L.budget) return cudaErrorInvalidValue;
+    if constexpr (NT == 1) {
+        if (a.fused) {
+            if (rf != kF32) return cudaErrorInvalidValue;
+            return launch_grid(k_replay_pipe<TIn, kF32, NT, 1>, a, L, grid, thr, smem, st);
+        }
+    }
     switch (rf) {
-        case kF32: return launch_grid(k_replay_pipe<TIn, kF32, NT>, a, L, grid, thr, smem, st);
-        case kBF16: return launch_grid(k_replay_pipe<TIn, kBF16, NT>, a, L, grid, thr, smem, st);
-        case kE4M3: return launch_grid(k_replay_pipe<TIn, kE4M3, NT>, a, L, grid, thr, smem, st);
-        default: return launch_grid(k_replay_pipe<TIn, kFP4, NT>, a, L, grid, thr, smem, st);
+        case kF32: return launch_grid(k_replay_pipe<TIn, kF32, NT, 0>, a, L, grid, thr, smem, st);
+        case kBF16: return launch_grid(k_replay_pipe<TIn, kBF16, NT, 0>, a, L, grid, thr, smem, st);
+        case kE4M3: return launch_grid(k_replay_pipe<TIn, kE4M3, NT, 0>, a, L, grid, thr, smem, st);
+        default: return launch_grid(k_replay_pipe<TIn, kFP4, NT, 0>, a, L, grid, thr, smem, st);
     }
 }
 
@@ -1699,13 +1761,13 @@ static cudaError_t launch_replay_pipe(const ReplayArgs& a, int in_bf16, int rf, 
 
 cudaError_t launch_replay(const ReplayArgs& a, int in_bf16, int rf, cudaStream_t st) {
     // the pipelined kernel serves d_state 128 with head_dim a multiple of 8
-    if (!a.fused && a.s.N == 128 && a.s.P % 8 == 0) {
+    if (a.s.N == 128 && a.s.P % 8 == 0 && (!a.fused || (rf == kF32 && a.ntok == 1))) {
         const DeviceInfo di = device_info();
         if (di.sms > 0) {
             // the kernel's static shared memory (barriers, per-group weights) stays below 8 KiB
             const size_t budget = di.smem_optin > 8192 ? di.smem_optin - 8192 : 0;
             const int groups = a.ntok == 1 ? pipe_groups(1) : pipe_groups(kMidTok);
-            const PipeLayout L = pipe_layout(a.s, a.rec, a.ntok, in_bf16, groups, budget);
+            const PipeLayout L = pipe_layout(a.s, a.rec, a.ntok, in_bf16, groups, a.fused, budget);
             if (L.stages >= 2) {
                 const int ntiles = a.s.batch * a.s.H;
                 const int grid = ntiles < di.sms ? ntiles : di.sms;
