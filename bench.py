@@ -327,6 +327,12 @@ def run_ours(args):
         torch.cuda.empty_cache()
         out["large_b512"] = large_leg(rssm, torch, WORKLOADS["large_b512"], max(2, min(K, 50)), W, dev, barrier,
                                       max_over_ranks, world, peak, args.fused)
+        torch.cuda.empty_cache()
+        out["spec_b512_k4"] = spec_leg(rssm, torch, WORKLOADS["spec_b512_k4"], max(2, min(K, 32)), W, dev, barrier,
+                                       max_over_ranks, world, peak)
+        torch.cuda.empty_cache()
+        out["split_b256"] = split_leg(rssm, torch, WORKLOADS["split_b256"], max(2, min(K, 50)), W, dev, barrier,
+                                      max_over_ranks, world, peak)
     if rank == 0 and world == 1 and not args.no_extra:
         out["cpu_baseline"] = cpu_baseline()
     if world > 1:
@@ -457,6 +463,169 @@ def large_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak, 
             "conventional_gbs": conv_bytes_per_request(shape) * shape.batch * L / (ms_c / K / 1e3) / 1e9}
 
 
+def spec_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
+    """Speculative decoding (s3) on the large layer with K = 4 drafts: per
+    step, replay verify of the pending token and 4 drafts + accept(n) + the
+    masked flush, against the conventional verify that writes one state copy
+    per token + accept (copy index). n ~ U{0..4} per request and step, the
+    same table for both. Metric: accepted tokens/s = sum(n + 1) / time."""
+    from hybrid_model_ssm_replay_b200.inputs import accept_lengths, make_inputs
+    shape = wl["shape"]
+    L, Kd = shape.interval, shape.max_draft
+    WIN = 8
+    inp = make_inputs(shape, WIN, wl["seed"], wl["in_dtype"], device=dev, ntok=Kd + 1)
+    n_tab = accept_lengths(W + K, shape.batch, Kd, wl["seed"], device=dev)
+    n_host = n_tab.cpu()
+    desc = rssm.make_desc(shape.batch, shape.nheads, shape.head_dim, shape.d_state, shape.ngroups, interval=L,
+                          max_draft=Kd)
+    ys = torch.empty((shape.batch, Kd + 1, shape.nheads, shape.head_dim), device=dev)
+    st = rssm.RssmState(desc, dev)
+    st.ckpt.copy_(inp["ckpt"])
+    ev_v = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+
+    def rstep(s, ev=None):
+        w = s % WIN
+        if ev is not None:
+            ev[0].record()
+        rssm.rssm_verify(st, Kd, inp["x"][w], inp["B"][w], inp["C"][w], inp["dt"][w], inp["A"], inp["D"], ys)
+        if ev is not None:
+            ev[1].record()
+        rssm.rssm_accept(st, n_tab[s])
+        rssm.rssm_flush(st, inp["A"])
+
+    def timed(fn, with_events):
+        for s in range(W):
+            fn(s)
+        torch.cuda.synchronize()
+        barrier()
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(K):
+            if with_events:
+                fn(W + i, ev_v[i])
+            else:
+                fn(W + i)
+        e.record()
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(a.elapsed_time(e))
+
+    ms_r = timed(rstep, True)
+    if rssm.rssm_get_error(st) != 0:
+        raise RuntimeError("device error in the speculative leg")
+    # verify bytes from the positions the accept table implies (pos += n + 1, folded at >= L)
+    b = shape_bytes(shape)
+    pos = torch.zeros(shape.batch, dtype=torch.int64)
+    vbytes = []
+    for s in range(W + K):
+        if s >= W:
+            vbytes.append(int((b["state"] + pos * b["entry"] + (Kd + 1) * (b["entry"] + b["inputs"] + b["y"])).sum()))
+        pos += n_host[s].long() + 1
+        pos = torch.where(pos >= L, torch.zeros_like(pos), pos)
+    v_ms = [x.elapsed_time(y) for x, y in ev_v]
+    v_gbs = [vb / (m / 1e3) / 1e9 for vb, m in zip(vbytes, v_ms)]
+    del st
+    torch.cuda.empty_cache()
+    copies = torch.empty((Kd + 1,) + tuple(inp["ckpt"].shape), device=dev)
+    copies[0].copy_(inp["ckpt"])
+    cur = torch.zeros(shape.batch, dtype=torch.int32, device=dev)
+
+    def cstep(s):
+        w = s % WIN
+        rssm.rssm_conv_verify(desc, copies, cur, Kd, inp["x"][w], inp["B"][w], inp["C"][w], inp["dt"][w], inp["A"],
+                              inp["D"], ys)
+        rssm.rssm_conv_accept(desc, n_tab[s], cur, Kd)
+
+    ms_c = timed(cstep, False)
+    del copies
+    acc = world * int((n_host[W:W + K].long() + 1).sum())
+    return {"workload": "spec_b512_k4: batch 512, 128 heads, 64 x 128, 8 groups, interval 16, K = 4 drafts, "
+                        "accepted n ~ U{0..4}", "steps": K,
+            "replay_accepted_tokens_per_s": acc / (ms_r / 1e3),
+            "conventional_accepted_tokens_per_s": acc / (ms_c / 1e3), "speedup": ms_c / ms_r,
+            "replay_step_us": ms_r / K * 1e3, "conventional_step_us": ms_c / K * 1e3,
+            "verify_avg_launch_us": sum(v_ms) / len(v_ms) * 1e3,
+            "verify_gbs": statistics.mean(v_gbs), "verify_frac": statistics.mean(v_gbs) / peak}
+
+
+def split_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
+    """Precision split (s4) on the small layer: 16 decodes reading the FP4
+    output copy + one refresh of the bf16 (or e4m3) update copy with Philox
+    SR, and the shared-FP4 control (one FP4 copy read and updated)."""
+    from hybrid_model_ssm_replay_b200.inputs import make_inputs
+    shape = wl["shape"]
+    L = shape.interval
+    H, P, N = shape.nheads, shape.head_dim, shape.d_state
+    inp = make_inputs(shape, L, wl["seed"], wl["in_dtype"], device=dev)
+    y = torch.empty((shape.batch, H, P), device=dev)
+    b = shape_bytes(shape)
+    fp4 = H * P * N // 2 + H * P * N // 16
+    tok_other = sum(i * b["entry"] for i in range(L)) / L + b["entry"] + b["inputs"] + b["y"]
+    out = {"workload": "split_b256: batch 256, 64 heads, 64 x 128, 8 groups, interval 16; decode reads the FP4 "
+                       "copy, refresh every 16 tokens", "steps": K}
+    modes = [("bf16_fp4", rssm.RSSM_BF16, rssm.RSSM_OUTCOPY_FP4, 2),
+             ("e4m3_fp4", rssm.RSSM_E4M3, rssm.RSSM_OUTCOPY_FP4, 1),
+             ("shared_fp4", rssm.RSSM_FP4, rssm.RSSM_OUTCOPY_NONE, 0)]
+    for name, upd, oc, eu in modes:
+        desc = rssm.make_desc(shape.batch, H, P, N, shape.ngroups, interval=L, update_dtype=upd, out_copy=oc,
+                              seed=wl["seed"])
+        st = rssm.RssmState(desc, dev)
+        if upd == rssm.RSSM_FP4:
+            d0 = rssm.make_desc(shape.batch, H, P, N, shape.ngroups, interval=L, out_copy=rssm.RSSM_OUTCOPY_FP4)
+            s0 = rssm.RssmState(d0, dev)
+            s0.ckpt.copy_(inp["ckpt"])
+            rssm.rssm_lowprec_refresh(s0, inp["A"], force=True)
+            st.ckpt.copy_(s0.out_codes)
+            st.ckpt_scales.copy_(s0.out_scales)
+            del s0
+        else:
+            st.ckpt.copy_(inp["ckpt"].to(torch.bfloat16 if upd == rssm.RSSM_BF16 else torch.float8_e4m3fn)
+                          .view(st.ckpt.dtype))
+            rssm.rssm_lowprec_refresh(st, inp["A"], force=True)
+        ev_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K * L)]
+        ev_r = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+
+        def step(k, timed):
+            for i in range(L):
+                if timed:
+                    ev_d[k * L + i][0].record()
+                rssm.rssm_decode_step(st, inp["x"][i], inp["B"][i], inp["C"][i], inp["dt"][i], inp["A"], inp["D"], y)
+                if timed:
+                    ev_d[k * L + i][1].record()
+            if timed:
+                ev_r[k][0].record()
+            rssm.rssm_lowprec_refresh(st, inp["A"])
+            if timed:
+                ev_r[k][1].record()
+
+        for k in range(W):
+            step(k, False)
+        torch.cuda.synchronize()
+        barrier()
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for k in range(K):
+            step(k, True)
+        e.record()
+        torch.cuda.synchronize()
+        barrier()
+        ms = max_over_ranks(a.elapsed_time(e))
+        if rssm.rssm_get_error(st) != 0:
+            raise RuntimeError("device error in the precision-split leg")
+        d_us = statistics.mean(x.elapsed_time(z) for x, z in ev_d) * 1e3
+        r_us = statistics.mean(x.elapsed_time(z) for x, z in ev_r) * 1e3
+        dec_bytes = (fp4 + tok_other) * shape.batch
+        upd_bytes = H * P * N * eu if eu else fp4
+        ref_bytes = (2 * upd_bytes + (fp4 if eu else 0) + L * b["entry"]) * shape.batch
+        out[name] = {"tokens_per_s": world * shape.batch * L * K / (ms / 1e3), "decode_avg_launch_us": d_us,
+                     "decode_gbs": dec_bytes / (d_us / 1e6) / 1e9, "decode_frac": dec_bytes / (d_us / 1e6) / 1e9 / peak,
+                     "refresh_avg_launch_us": r_us, "refresh_gbs": ref_bytes / (r_us / 1e6) / 1e9,
+                     "step_bytes_per_token": (dec_bytes * L + ref_bytes) / (shape.batch * L)}
+        del st
+        torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------- the CPU oracle arm
 
 def oracle_interval_sample(n_requests, seed=5):
@@ -478,7 +647,29 @@ def oracle_interval(orc, f, b, L):
     return L
 
 
+def _oracle_worker(job):
+    """One host core's share of the sharded oracle run (spawned process)."""
+    f, L, target_s = job
+    from oracle import oracle as orc
+    nb = f["ckpt"].shape[0]
+    oracle_interval(orc, f, 0, L)  # warm (loads the library)
+    tok, b, t0 = 0, 0, time.perf_counter()
+    while time.perf_counter() - t0 < target_s:
+        tok += oracle_interval(orc, f, b % nb, L)
+        b += 1
+    return tok, time.perf_counter() - t0, b
+
+
+def request_slice(f, reqs):
+    """The sampled inputs of some requests: ckpt [b], per-token arrays [t][b]."""
+    return {k: (v[reqs] if k == "ckpt" else (v[:, reqs] if v.ndim >= 2 else v)) for k, v in f.items()}
+
+
 def cpu_baseline(target_s=10.0):
+    """The fp64 oracle on the host: single thread, then sharded by request
+    over the host's cores (one spawned process per core, each on its own
+    requests). Reported: the sharded run, with the single-thread figure."""
+    import multiprocessing as mp
     from oracle import oracle as orc
     f, shape = oracle_interval_sample(8)
     L = shape.interval
@@ -489,9 +680,31 @@ def cpu_baseline(target_s=10.0):
         tok += oracle_interval(orc, f, b % shape.batch, L)
         b += 1
     dt = time.perf_counter() - t0
-    return {"value": tok / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{b} request-intervals of the small_b256 layer (16 replay decodes + 1 flush each, "
-                      f"fp64, single thread), {dt:.1f} s"}
+    single = tok / dt
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    cores = max(1, min(cores, 64))
+    jobs = [(request_slice(f, [(2 * i) % 8, (2 * i + 1) % 8]), L, target_s) for i in range(cores)]
+    try:
+        # spawned workers (no CUDA state is inherited); a worker that fails to
+        # start breaks the executor instead of hanging it
+        from concurrent.futures import ProcessPoolExecutor
+        with ProcessPoolExecutor(max_workers=cores, mp_context=mp.get_context("spawn")) as ex:
+            res = list(ex.map(_oracle_worker, jobs, timeout=target_s + 120))
+        s_tok = sum(r[0] for r in res)
+        s_dt = max(r[1] for r in res)
+        s_int = sum(r[2] for r in res)
+        return {"value": s_tok / s_dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"{s_int} request-intervals of the small_b256 layer (16 replay decodes + 1 flush each, "
+                          f"fp64), sharded by request over {cores} processes, {s_dt:.1f} s",
+                "single_thread": {"value": single, "cores": 1,
+                                  "sample": f"{b} request-intervals, one thread, {dt:.1f} s"}}
+    except Exception as e:  # a host that cannot spawn: the single-thread figure
+        return {"value": single, "unit": UNIT, "cores": 1, "kind": "oracle",
+                "sample": f"{b} request-intervals of the small_b256 layer (16 replay decodes + 1 flush each, "
+                          f"fp64, single thread), {dt:.1f} s; sharded run failed: {type(e).__name__}"}
 
 
 def run_reference(args):
