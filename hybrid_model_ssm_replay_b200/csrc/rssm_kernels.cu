@@ -527,10 +527,10 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 
 // Consumer groups of the pipelined kernel and warps per group: groups work
 // on different tiles at once, which hides the latency chain of one tile
-// (barriers, shared-memory loads, shuffle reductions); three for decode, two
-// for verify (whose K+1 tokens need the registers). A group has at least
-// four warps: its B.C products take 8 slots per warp, up to 32 slots.
-__host__ __device__ constexpr int pipe_groups(int nt) { return nt == 1 ? 3 : 2; }
+// (barriers, shared-memory loads, shuffle reductions); three, or two for
+// verify of more than kMidTok tokens (whose registers would spill). A group
+// has at least four warps: its B.C products take 8 slots per warp, up to 32.
+__host__ __device__ constexpr int pipe_groups(int nt) { return nt <= kMidTok ? 3 : 2; }
 __host__ __device__ constexpr int pipe_cwarps(int nt) { return (void)nt, 4; }
 __host__ __device__ constexpr int pipe_threads(int nt) { return (pipe_groups(nt) * pipe_cwarps(nt) + 1) * 32; }
 
@@ -775,18 +775,22 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
             for (int j = 0; j < NT; ++j)
                 c4[j] = (j < ntok) ? load4(nc + j * N + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
             if (cw * 8 < T) {
-                // B_s . C_j for slots s0..s0+7, reduced together
+                // B_s . C_j for slots s0..s0+7, reduced together; the 8 B rows
+                // are read once for all tokens
                 const int s0 = cw * 8;
+                float4 bv[8];
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const int sl = s0 + kk;
+                    const TIn* row = (sl < pos) ? br + sl * N : nb + (sl - pos) * N;
+                    bv[kk] = (sl < T) ? load4(row + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
 #pragma unroll
                 for (int j = 0; j < NT; ++j) {
                     if (j < ntok) {
                         float part[8];
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const int sl = s0 + kk;
-                            const TIn* row = (sl < pos) ? br + sl * N : nb + (sl - pos) * N;
-                            part[kk] = (sl < T) ? dot4(load4(row + 4 * lane), c4[j]) : 0.f;
-                        }
+                        for (int kk = 0; kk < 8; ++kk) part[kk] = dot4(bv[kk], c4[j]);
                         const float z = warp_reduce8(part);
                         const int sl = s0 + ((lane >> 2) & 7);
                         if ((lane & 3) == 0 && sl < T) s_g[gi][j][sl] = z;
@@ -863,8 +867,39 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
                     part[7] = fmaf(coef, xb.w, part[7]);
                 }
             };
-            // two 8-row blocks per pass, so their reductions overlap
-            for (int r0 = cw * 8; r0 < P; r0 += 2 * CW * 8) {
+            if constexpr (NT > 1) {
+                // verify: one 8-row block at a time; its tile rows and x
+                // values are read once for all tokens
+                for (int r0 = cw * 8; r0 < P; r0 += CW * 8) {
+                    float4 hv[8];
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) hv[kk] = tile_load4<RF>(tile, sc, r0 + kk, lane, N);
+                    float xv8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    if (lane < T) {  // slot `lane` exists (its row lies in the stage or this call's rows)
+                        Raw8<TIn> xv;
+                        xv.load(xrow + r0);
+                        const float4 xa = xv.lo(), xb = xv.hi();
+                        xv8[0] = xa.x; xv8[1] = xa.y; xv8[2] = xa.z; xv8[3] = xa.w;
+                        xv8[4] = xb.x; xv8[5] = xb.y; xv8[6] = xb.z; xv8[7] = xb.w;
+                    }
+                    const int rr = r0 + ((lane >> 2) & 7);
+#pragma unroll
+                    for (int j = 0; j < NT; ++j) {
+                        if (j < ntok) {
+                            const int tt = pos + j;
+                            const float dec = s_decay[gi][j];
+                            const float coef = (lane <= tt) ? s_w[gi][j][lane] * s_g[gi][j][lane] : 0.f;
+                            float part[8];
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk) part[kk] = fmaf(coef, xv8[kk], dec * dot4(hv[kk], c4[j]));
+                            const float z = warp_reduce8(part);
+                            if ((lane & 3) == 0) yout[j * HP + rr] = fmaf(Dh, to_f32(nx[j * P + rr]), z);
+                        }
+                    }
+                }
+            }
+            // decode: two 8-row blocks per pass, so their reductions overlap
+            for (int r0 = cw * 8; NT == 1 && r0 < P; r0 += 2 * CW * 8) {
                 const int r1 = r0 + CW * 8;
 #pragma unroll
                 for (int j = 0; j < NT; ++j) {
@@ -1766,7 +1801,8 @@ cudaError_t launch_replay(const ReplayArgs& a, int in_bf16, int rf, cudaStream_t
         if (di.sms > 0) {
             // the kernel's static shared memory (barriers, per-group weights) stays below 8 KiB
             const size_t budget = di.smem_optin > 8192 ? di.smem_optin - 8192 : 0;
-            const int groups = a.ntok == 1 ? pipe_groups(1) : pipe_groups(kMidTok);
+            const int nt = a.ntok == 1 ? 1 : (a.ntok <= kMidTok ? kMidTok : kMaxTok);  // the kernel's token bound
+            const int groups = pipe_groups(nt);
             const PipeLayout L = pipe_layout(a.s, a.rec, a.ntok, in_bf16, groups, a.fused, budget);
             if (L.stages >= 2) {
                 const int ntiles = a.s.batch * a.s.H;
