@@ -23,7 +23,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kMaxCap = 32;                 // buffer slots per request (interval + drafts)
 constexpr int kMaxTok = 8;                  // tokens per verify call (K + 1)
 constexpr int kMidTok = 5;                  // verify kernels specialised for K <= 4
-constexpr int kPipeStagesMax = 8;           // shared-memory stages of the pipelined replay kernel
+constexpr int kPipeStagesMax = 16;          // shared-memory stages of the pipelined kernels
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bound of one bulk-copy wait
 
 // ------------------------------------------------------------------ errors
@@ -199,32 +199,44 @@ __device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
     return out & 0xFFu;
 }
 
-__device__ __forceinline__ float e4m3_val(uint32_t c) {
-    const uint32_t e = (c >> 3) & 15u, m = c & 7u;
-    const float mag = (e == 0u) ? static_cast<float>(m) * 0x1p-9f : __uint_as_float(((e + 120u) << 23) | (m << 20));
-    return (c & 0x80u) ? -mag : mag;
+// Two e4m3 codes (16 bits, element 0 in the low byte) as an fp16 pair
+// (hardware conversion; every e4m3 value is exact in fp16).
+__device__ __forceinline__ uint32_t e4m3x2_h2(uint32_t codes16) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<unsigned short>(codes16)));
+    return h;
 }
+
+__device__ __forceinline__ float2 h2_f2(uint32_t h) { return __half22float2(*reinterpret_cast<const __half2*>(&h)); }
+
+__device__ __forceinline__ float e4m3_val(uint32_t c) { return h2_f2(e4m3x2_h2(c & 0xFFu)).x; }
 
 __device__ __forceinline__ float bf16_val(uint32_t bits) { return __uint_as_float(bits << 16); }
 
-// Four e2m1 codes (16 bits, element 0 in the low nibble) times a scale, exactly.
-// Each nibble's magnitude bits go to bits 11..9 of an fp16 (the low exponent
-// bits and the top mantissa bit) and its sign to bit 15: the fp16 then holds
-// the e2m1 value times 2^-14 (e2m1's subnormal 0.5 lands on an fp16
-// subnormal), so scale2p14 = scale * 2^14 restores it. Products are exact.
-__device__ __forceinline__ float4 fp4x4_val(uint32_t codes16, float scale2p14) {
-    const uint32_t c0 = codes16 & 0xFFu, c1 = (codes16 >> 8) & 0xFFu;
-    const uint32_t w01 = ((c0 & 0x7u) << 9) | ((c0 & 0x8u) << 12) | ((c0 & 0x70u) << 21) | ((c0 & 0x80u) << 24);
-    const uint32_t w23 = ((c1 & 0x7u) << 9) | ((c1 & 0x8u) << 12) | ((c1 & 0x70u) << 21) | ((c1 & 0x80u) << 24);
-    const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&w01));
-    const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&w23));
-    return make_float4(f01.x * scale2p14, f01.y * scale2p14, f23.x * scale2p14, f23.y * scale2p14);
+// Four e2m1 codes (16 bits, element 0 in the low nibble) as floats, exactly
+// (hardware conversion of each byte to an fp16 pair, low nibble first).
+__device__ __forceinline__ float4 e2m1x4_val(uint32_t codes16) {
+    uint32_t h01, h23;
+    asm("{\n\t.reg .b8 b0, b1;\n\t"
+        "mov.b16 {b0, b1}, %2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t}"
+        : "=r"(h01), "=r"(h23)
+        : "h"(static_cast<unsigned short>(codes16)));
+    const float2 a = h2_f2(h01), b = h2_f2(h23);
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// Four FP4 values: codes times their block scale (products are exact).
+__device__ __forceinline__ float4 fp4x4_val(uint32_t codes16, float scale) {
+    const float4 v = e2m1x4_val(codes16);
+    return make_float4(v.x * scale, v.y * scale, v.z * scale, v.w * scale);
 }
 
 // Four e4m3 codes (32 bits, element 0 in the low byte) to floats.
 __device__ __forceinline__ float4 e4m3x4_val(uint32_t w) {
-    return make_float4(e4m3_val(w & 0xFFu), e4m3_val((w >> 8) & 0xFFu), e4m3_val((w >> 16) & 0xFFu),
-                       e4m3_val(w >> 24));
+    const float2 a = h2_f2(e4m3x2_h2(w & 0xFFFFu)), b = h2_f2(e4m3x2_h2(w >> 16));
+    return make_float4(a.x, a.y, b.x, b.y);
 }
 
 // Four bf16 (two 32-bit words, element 0 in the low half) to floats.

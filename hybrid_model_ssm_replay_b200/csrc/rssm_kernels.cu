@@ -44,7 +44,7 @@ __device__ __forceinline__ float4 tile_load4(const unsigned char* t, const unsig
     } else if constexpr (F == kE4M3) {
         return e4m3x4_val(reinterpret_cast<const uint32_t*>(t)[q]);
     } else {
-        return fp4x4_val(reinterpret_cast<const uint16_t*>(t)[q], e4m3_val(sc[q >> 2]) * 16384.0f);
+        return fp4x4_val(reinterpret_cast<const uint16_t*>(t)[q], e4m3_val(sc[q >> 2]));
     }
 }
 
@@ -525,24 +525,28 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Consumer groups of the pipelined kernel and warps per group: groups work
+// Consumer groups of the pipelined kernel and warps per group. Groups work
 // on different tiles at once, which hides the latency chain of one tile
-// (barriers, shared-memory loads, shuffle reductions); three, or two for
-// verify of more than kMidTok tokens (whose registers would spill). A group
-// has at least four warps: its B.C products take 8 slots per warp, up to 32.
-__host__ __device__ constexpr int pipe_groups(int nt) { return nt <= kMidTok ? 3 : 2; }
-__host__ __device__ constexpr int pipe_cwarps(int nt) { return (void)nt, 4; }
-__host__ __device__ constexpr int pipe_threads(int nt) { return (pipe_groups(nt) * pipe_cwarps(nt) + 1) * 32; }
+// (barriers, shared-memory loads, shuffle reductions). The fp32 copy fills a
+// 39 KB stage per tile at the shapes served, so few tiles fit in shared
+// memory: three groups of four warps (two groups for verify of more than
+// kMidTok tokens, whose registers would spill). The smaller bf16 / e4m3 /
+// FP4 copies leave room for many tiles: six groups of two warps, with fewer
+// barrier waits per tile.
+__host__ __device__ constexpr int pipe_groups(int nt, int rf) { return rf == kF32 ? (nt <= kMidTok ? 3 : 2) : 6; }
+__host__ __device__ constexpr int pipe_cwarps(int nt, int rf) { return rf == kF32 ? 4 : (nt <= kMidTok ? 2 : 1); }
+__host__ __device__ constexpr int pipe_threads(int nt, int rf) {
+    return (pipe_groups(nt, rf) * pipe_cwarps(nt, rf) + 1) * 32;
+}
 
 // Stage meta (int words): the position and the index k of the tile the
 // stage holds (-1 before its first use).
 constexpr int kMetaPos = 0, kMetaTile = 1;
 
 template <typename TIn, int RF, int NT, int FUSED>
-__global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const ReplayArgs a, const PipeLayout lay) {
-    constexpr int CG = pipe_groups(NT), CW = pipe_cwarps(NT), CT = CW * 32;
+__global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const ReplayArgs a, const PipeLayout lay) {
+    constexpr int CG = pipe_groups(NT, RF), CW = pipe_cwarps(NT, RF), CT = CW * 32;
     static_assert(!FUSED || (RF == kF32 && NT == 1), "the fused fold is for fp32 decode");
-    static_assert(CW >= 4, "B.C products need 4 warps of 8 slots");
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full_bar[kPipeStagesMax];
     __shared__ __align__(8) uint64_t empty_bar[kPipeStagesMax];
@@ -774,10 +778,9 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
 #pragma unroll
             for (int j = 0; j < NT; ++j)
                 c4[j] = (j < ntok) ? load4(nc + j * N + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-            if (cw * 8 < T) {
+            for (int s0 = cw * 8; s0 < T; s0 += CW * 8) {
                 // B_s . C_j for slots s0..s0+7, reduced together; the 8 B rows
                 // are read once for all tokens
-                const int s0 = cw * 8;
                 float4 bv[8];
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -826,7 +829,7 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
                     pend_old = atomicAdd(&a.arrive[b], 1u);
                 }
             }
-            if (cw == 2) {
+            if (cw == (CW >= 3 ? 2 : 0)) {
                 // append this call's x (and, for the group's first head, B) to the buffer
                 const int xq = ntok * xc, bq = ntok * bc;
                 uint4* xdst = reinterpret_cast<uint4*>(rec + a.rec.x + static_cast<size_t>(pos) * P * es);
@@ -849,9 +852,17 @@ __global__ void __launch_bounds__(pipe_threads(NT), 1) k_replay_pipe(const Repla
             auto partials = [&](int r0, const float4& cj, float dec, float coef, bool term, float (&part)[8]) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const float4 hv = (r0 + kk < P) ? tile_load4<RF>(tile, sc, r0 + kk, lane, N)
-                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-                    part[kk] = dec * dot4(hv, cj);
+                    if constexpr (RF == kFP4) {
+                        // codes . C first, then one multiply by the block scale
+                        const int q = (r0 + kk) * (N >> 2) + lane;
+                        part[kk] = (r0 + kk < P) ? (dec * e4m3_val(sc[q >> 2])) *
+                                                       dot4(e2m1x4_val(reinterpret_cast<const uint16_t*>(tile)[q]), cj)
+                                                 : 0.f;
+                    } else {
+                        const float4 hv = (r0 + kk < P) ? tile_load4<RF>(tile, sc, r0 + kk, lane, N)
+                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                        part[kk] = dec * dot4(hv, cj);
+                    }
                 }
                 if (term && r0 < P) {
                     Raw8<TIn> xv;
@@ -1605,7 +1616,7 @@ __global__ void k_round_test(int op, int64_t n, const float* v, uint64_t seed, u
         }
         if (valid && op == 5) {
             // the decode the FP4-reading kernels use
-            reinterpret_cast<float4*>(out)[q] = fp4x4_val(codes, e4m3_val(sc) * 16384.0f);
+            reinterpret_cast<float4*>(out)[q] = fp4x4_val(codes, e4m3_val(sc));
         }
         return;
     }
@@ -1765,21 +1776,24 @@ static DeviceInfo device_info() {
 
 template <typename TIn, int NT>
 static cudaError_t pipe_dispatch(const ReplayArgs& a, const PipeLayout& L, int rf, int grid, cudaStream_t st) {
-    constexpr int thr = pipe_threads(NT);
     const size_t smem = static_cast<size_t>(L.stages) * L.stage_bytes +
-                        static_cast<size_t>(pipe_groups(NT)) * (3u * L.newrows + L.xw_bytes);
+                        static_cast<size_t>(pipe_groups(NT, rf)) * (3u * L.newrows + L.xw_bytes);
     if (smem > L.budget) return cudaErrorInvalidValue;
     if constexpr (NT == 1) {
         if (a.fused) {
             if (rf != kF32) return cudaErrorInvalidValue;
-            return launch_grid(k_replay_pipe<TIn, kF32, NT, 1>, a, L, grid, thr, smem, st);
+            return launch_grid(k_replay_pipe<TIn, kF32, NT, 1>, a, L, grid, pipe_threads(NT, kF32), smem, st);
         }
     }
     switch (rf) {
-        case kF32: return launch_grid(k_replay_pipe<TIn, kF32, NT, 0>, a, L, grid, thr, smem, st);
-        case kBF16: return launch_grid(k_replay_pipe<TIn, kBF16, NT, 0>, a, L, grid, thr, smem, st);
-        case kE4M3: return launch_grid(k_replay_pipe<TIn, kE4M3, NT, 0>, a, L, grid, thr, smem, st);
-        default: return launch_grid(k_replay_pipe<TIn, kFP4, NT, 0>, a, L, grid, thr, smem, st);
+        case kF32:
+            return launch_grid(k_replay_pipe<TIn, kF32, NT, 0>, a, L, grid, pipe_threads(NT, kF32), smem, st);
+        case kBF16:
+            return launch_grid(k_replay_pipe<TIn, kBF16, NT, 0>, a, L, grid, pipe_threads(NT, kBF16), smem, st);
+        case kE4M3:
+            return launch_grid(k_replay_pipe<TIn, kE4M3, NT, 0>, a, L, grid, pipe_threads(NT, kE4M3), smem, st);
+        default:
+            return launch_grid(k_replay_pipe<TIn, kFP4, NT, 0>, a, L, grid, pipe_threads(NT, kFP4), smem, st);
     }
 }
 
@@ -1802,7 +1816,7 @@ cudaError_t launch_replay(const ReplayArgs& a, int in_bf16, int rf, cudaStream_t
             // the kernel's static shared memory (barriers, per-group weights) stays below 8 KiB
             const size_t budget = di.smem_optin > 8192 ? di.smem_optin - 8192 : 0;
             const int nt = a.ntok == 1 ? 1 : (a.ntok <= kMidTok ? kMidTok : kMaxTok);  // the kernel's token bound
-            const int groups = pipe_groups(nt);
+            const int groups = pipe_groups(nt, rf);
             const PipeLayout L = pipe_layout(a.s, a.rec, a.ntok, in_bf16, groups, a.fused, budget);
             if (L.stages >= 2) {
                 const int ntiles = a.s.batch * a.s.H;
