@@ -227,6 +227,33 @@ __device__ __forceinline__ float4 e2m1x4_val(uint32_t codes16) {
     return make_float4(a.x, a.y, b.x, b.y);
 }
 
+// Dot product of eight e2m1 codes (32 bits, element 0 in the low nibble)
+// with c[0..7], unscaled, added to acc in element order.
+__device__ __forceinline__ float e2m1x8_dot(uint32_t w, const float* c, float acc) {
+    uint32_t h0, h1, h2, h3;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+        : "r"(w));
+    float2 f = h2_f2(h0);
+    acc = fmaf(f.x, c[0], acc);
+    acc = fmaf(f.y, c[1], acc);
+    f = h2_f2(h1);
+    acc = fmaf(f.x, c[2], acc);
+    acc = fmaf(f.y, c[3], acc);
+    f = h2_f2(h2);
+    acc = fmaf(f.x, c[4], acc);
+    acc = fmaf(f.y, c[5], acc);
+    f = h2_f2(h3);
+    acc = fmaf(f.x, c[6], acc);
+    acc = fmaf(f.y, c[7], acc);
+    return acc;
+}
+
 // Four FP4 values: codes times their block scale (products are exact).
 __device__ __forceinline__ float4 fp4x4_val(uint32_t codes16, float scale) {
     const float4 v = e2m1x4_val(codes16);

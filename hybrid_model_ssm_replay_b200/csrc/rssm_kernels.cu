@@ -530,11 +530,16 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // (barriers, shared-memory loads, shuffle reductions). The fp32 copy fills a
 // 39 KB stage per tile at the shapes served, so few tiles fit in shared
 // memory: three groups of four warps (two groups for verify of more than
-// kMidTok tokens, whose registers would spill). The smaller bf16 / e4m3 /
-// FP4 copies leave room for many tiles: six groups of two warps, with fewer
-// barrier waits per tile.
-__host__ __device__ constexpr int pipe_groups(int nt, int rf) { return rf == kF32 ? (nt <= kMidTok ? 3 : 2) : 6; }
-__host__ __device__ constexpr int pipe_cwarps(int nt, int rf) { return rf == kF32 ? 4 : (nt <= kMidTok ? 2 : 1); }
+// kMidTok tokens, whose registers would spill). The smaller copies leave room
+// for many tiles: bf16 six groups of two warps; e4m3 and FP4 twelve groups of
+// one warp, each tile worked by one warp without group barriers (measured on
+// B200: FP4 decode 102 us with 6 x 2, 93 us with 12 x 1, 114 us with 8 x 1).
+__host__ __device__ constexpr int pipe_groups(int nt, int rf) {
+    return rf == kF32 ? (nt <= kMidTok ? 3 : 2) : (rf == kBF16 || nt > kMidTok ? 6 : 12);
+}
+__host__ __device__ constexpr int pipe_cwarps(int nt, int rf) {
+    return rf == kF32 ? 4 : (rf == kBF16 && nt <= kMidTok ? 2 : 1);
+}
 __host__ __device__ constexpr int pipe_threads(int nt, int rf) {
     return (pipe_groups(nt, rf) * pipe_cwarps(nt, rf) + 1) * 32;
 }
@@ -878,7 +883,53 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                     part[7] = fmaf(coef, xb.w, part[7]);
                 }
             };
-            if constexpr (NT > 1) {
+            if constexpr (RF == kFP4 && NT == 1) {
+                // FP4 decode: lane l takes row r0 + l/4 and columns 32 (l % 4) ..
+                // +31 of an 8-row block: one 16-byte load of codes and one of
+                // two scales per row, codes.C per 16 columns times the block
+                // scale, and the replay terms of slots l % 4, l % 4 + 4, ...;
+                // the row's 4 lanes then add up with two shuffles
+                const int sg = lane & 3, rl = lane >> 2;
+                float cv[32];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    Raw8<TIn> r8;
+                    r8.load(nc + 32 * sg + 8 * i);
+                    const float4 lo = r8.lo(), hi = r8.hi();
+                    cv[8 * i + 0] = lo.x;
+                    cv[8 * i + 1] = lo.y;
+                    cv[8 * i + 2] = lo.z;
+                    cv[8 * i + 3] = lo.w;
+                    cv[8 * i + 4] = hi.x;
+                    cv[8 * i + 5] = hi.y;
+                    cv[8 * i + 6] = hi.z;
+                    cv[8 * i + 7] = hi.w;
+                }
+                const float dec = s_decay[gi][0];
+                float cf[kMaxCap / 4];
+#pragma unroll
+                for (int m = 0; m < kMaxCap / 4; ++m) {
+                    const int sl = sg + 4 * m;
+                    cf[m] = (sl <= pos) ? s_w[gi][0][sl] * s_g[gi][0][sl] : 0.f;
+                }
+                for (int r0 = cw * 8; r0 < P; r0 += CW * 8) {
+                    const int r = r0 + rl;
+                    const uint4 q4 = *reinterpret_cast<const uint4*>(tile + r * (N >> 1) + 16 * sg);
+                    const float2 s2 =
+                        h2_f2(e4m3x2_h2(*reinterpret_cast<const uint16_t*>(sc + r * (N >> 4) + 2 * sg)));
+                    const float a0 = e2m1x8_dot(q4.x, cv, 0.f) + e2m1x8_dot(q4.y, cv + 8, 0.f);
+                    const float a1 = e2m1x8_dot(q4.z, cv + 16, 0.f) + e2m1x8_dot(q4.w, cv + 24, 0.f);
+                    float part = dec * fmaf(s2.x, a0, s2.y * a1);
+#pragma unroll
+                    for (int m = 0; m < kMaxCap / 4; ++m) {
+                        const int sl = sg + 4 * m;
+                        if (sl <= pos) part = fmaf(cf[m], to_f32((sl < pos ? xr + sl * P : nx)[r]), part);
+                    }
+                    part += __shfl_xor_sync(0xffffffffu, part, 1);
+                    part += __shfl_xor_sync(0xffffffffu, part, 2);
+                    if (sg == 0) yout[r] = fmaf(Dh, to_f32(nx[r]), part);
+                }
+            } else if constexpr (NT > 1) {
                 // verify: one 8-row block at a time; its tile rows and x
                 // values are read once for all tokens
                 for (int r0 = cw * 8; r0 < P; r0 += CW * 8) {
@@ -910,7 +961,7 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                 }
             }
             // decode: two 8-row blocks per pass, so their reductions overlap
-            for (int r0 = cw * 8; NT == 1 && r0 < P; r0 += 2 * CW * 8) {
+            for (int r0 = cw * 8; NT == 1 && RF != kFP4 && r0 < P; r0 += 2 * CW * 8) {
                 const int r1 = r0 + CW * 8;
 #pragma unroll
                 for (int j = 0; j < NT; ++j) {
