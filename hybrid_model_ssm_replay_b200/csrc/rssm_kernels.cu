@@ -543,6 +543,12 @@ __host__ __device__ constexpr int pipe_cwarps(int nt, int rf) {
 __host__ __device__ constexpr int pipe_threads(int nt, int rf) {
     return (pipe_groups(nt, rf) * pipe_cwarps(nt, rf) + 1) * 32;
 }
+// Static shared memory of k_replay_pipe<*, rf, nt, *>: per-group weights,
+// B.C products and decays, the stage barriers, the abort flag (plus slack for
+// what the compiler adds); the dynamic stages get the rest.
+__host__ __device__ constexpr size_t pipe_static_smem(int nt, int rf) {
+    return static_cast<size_t>(pipe_groups(nt, rf)) * nt * (2 * kMaxCap + 1) * 4 + 2 * kPipeStagesMax * 8 + 1024;
+}
 
 // Stage meta (int words): the position and the index k of the tile the
 // stage holds (-1 before its first use).
@@ -1864,9 +1870,9 @@ cudaError_t launch_replay(const ReplayArgs& a, int in_bf16, int rf, cudaStream_t
     if (a.s.N == 128 && a.s.P % 8 == 0 && (!a.fused || (rf == kF32 && a.ntok == 1))) {
         const DeviceInfo di = device_info();
         if (di.sms > 0) {
-            // the kernel's static shared memory (barriers, per-group weights) stays below 8 KiB
-            const size_t budget = di.smem_optin > 8192 ? di.smem_optin - 8192 : 0;
             const int nt = a.ntok == 1 ? 1 : (a.ntok <= kMidTok ? kMidTok : kMaxTok);  // the kernel's token bound
+            const size_t stat = pipe_static_smem(nt, rf);
+            const size_t budget = di.smem_optin > stat ? di.smem_optin - stat : 0;
             const int groups = pipe_groups(nt, rf);
             const PipeLayout L = pipe_layout(a.s, a.rec, a.ntok, in_bf16, groups, a.fused, budget);
             if (L.stages >= 2) {

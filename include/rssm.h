@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define RSSM_ABI_VERSION 1
+#define RSSM_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define RSSM_API __attribute__((visibility("default")))

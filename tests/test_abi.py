@@ -29,7 +29,7 @@ def test_exports_every_declared_symbol(L):
     assert len(names) >= 14
     for n in names:
         assert hasattr(L, n), n
-    assert L.rssm_abi_version() == 1
+    assert L.rssm_abi_version() == 2
 
 
 def cfg(**kw):

@@ -146,6 +146,54 @@ def test_fp4_decode_and_refresh_match_oracle(kind):
     assert st.flush_count.cpu().tolist() == [2] * 4
 
 
+@pytest.mark.parametrize("kind", ["bf16", "e4m3"])
+def test_speculative_verify_on_split_state_matches_oracle(kind):
+    """Speculative decoding (s3) on a split-precision state (s4): verify of
+    the pending token and K = 4 drafts reads the FP4 output copy, accept(n)
+    advances pos, and the refresh after accept folds the requests whose
+    buffer reached the interval. Four steps, so every verify reads the
+    initial FP4 copy (pos <= 15 before the last accept); the outputs match
+    the oracle within the fp32 tolerance, and each refreshed request's update
+    and FP4 copies match it bit for bit except at fp32 rounding straddles."""
+    shape = LayerShape(4, 8, 64, 128, 2, interval=16, max_draft=4)
+    K, steps, L = 4, 4, 16
+    inp = make_inputs(shape, steps, 34, torch.bfloat16, device="cuda", ntok=K + 1)
+    # accepted drafts per step and request: three requests reach the interval
+    # on the last step (pos 20, 19, 19), one does not (pos 10)
+    n_host = np.array([[4, 3, 0, 4], [4, 4, 1, 4], [4, 4, 2, 3], [4, 4, 3, 4]], np.int32)
+    n_acc = torch.from_numpy(n_host).cuda()
+    seed = 0x5EED
+    desc, st = split_state(shape, inp, kind, seed)
+    upd0 = copy_bits(initial_update_copy(inp["ckpt"], kind))
+    codes0, scales0 = orc.fp4_quant(orc.widen(UPD[kind][1], upd0, None, upd0.shape).astype(np.float32))
+    y = torch.empty((steps, shape.batch, K + 1, shape.nheads, shape.head_dim), device="cuda")
+    for s in range(steps):
+        rssm.rssm_verify(st, K, inp["x"][s], inp["B"][s], inp["C"][s], inp["dt"][s], inp["A"], inp["D"], y[s])
+        rssm.rssm_accept(st, n_acc[s])
+        rssm.rssm_lowprec_refresh(st, inp["A"])
+    assert rssm.rssm_get_error(st) == 0
+    mism = total = folded = 0
+    for b in range(shape.batch):
+        r = request_inputs(inp, b)
+        req = orc.LowPrecRequest(UPD[kind][1], True, upd0[b], codes0[b], scales0[b], shape.ngroups, L + K,
+                                 r["A"], r["D"], seed, b)
+        req.flush_count.value = 1
+        for s in range(steps):
+            ys = req.verify(r["x"][s], r["B"][s], r["C"][s], r["dt"][s])
+            assert_close(to_np(y[s, b]), ys, f"verify on the FP4 copy, step {s}, request {b}")
+            req.accept(int(n_host[s, b]))
+            if req.pos >= L:
+                req.refresh()
+                folded += 1
+        assert st.pos[b].item() == req.pos and st.flush_count[b].item() == req.flush_count.value
+        got = copy_bits(st.ckpt[b]).ravel()
+        mism += int(np.count_nonzero(got != req.upd.ravel()))
+        mism += int(np.count_nonzero(st.out_codes[b].cpu().numpy().ravel() != req.codes.ravel()))
+        total += got.size
+    assert folded == 3
+    assert mism <= 3e-3 * total, mism
+
+
 @pytest.mark.parametrize("shape", SHAPES, ids=["dstate64", "dstate128"])
 def test_shared_fp4_control_decode_matches_oracle(shape):
     L = shape.interval
