@@ -158,23 +158,19 @@ __device__ __forceinline__ uint32_t sr_e4m3(float v, uint32_t r) {
     const uint32_t a = u & 0x7FFFFFFFu;
     if (a > 0x7F800000u) return 0x7Fu;
     if (a >= 0x43E00000u) return sign | 0x7Eu;
-    const int E = static_cast<int>(a >> 23) - 127;
     uint32_t code, F;
-    if (E >= -6) {
-        code = (static_cast<uint32_t>(E + 7) << 3) | ((a >> 20) & 7u);
+    if (a >= 0x3C800000u) {
+        // normal: the exponent and top 3 mantissa bits re-biased (127 -> 7);
+        // the 20 bits below them are the fraction
+        code = (a >> 20) - (120u << 3);
         F = (a & 0xFFFFFu) << 12;
     } else {
-        // below 2^-6: count steps of 2^-9 in the 24-bit significand M * 2^(E-23)
-        const uint32_t M = (E == -127) ? (a & 0x7FFFFFu) : ((a & 0x7FFFFFu) | 0x800000u);
-        const int sh = 14 - ((E == -127) ? -126 : E);   // >= 21
-        if (sh >= 56) {
-            code = 0u;
-            F = 0u;
-        } else {
-            code = (sh >= 32) ? 0u : (M >> sh);
-            const uint64_t frac = static_cast<uint64_t>(M) & ((1ull << sh) - 1ull);
-            F = (sh <= 32) ? static_cast<uint32_t>(frac << (32 - sh)) : static_cast<uint32_t>(frac >> (sh - 32));
-        }
+        // below 2^-6: t = |v| 2^9 < 8 is exact, code = floor(t), and the
+        // fraction scaled by 2^32 is exact too
+        const float t = __uint_as_float(a) * 512.0f;
+        const float m = truncf(t);
+        code = static_cast<uint32_t>(m);
+        F = __float2uint_rz((t - m) * 4294967296.0f);
     }
     return sign | (code + (r < F ? 1u : 0u));
 }

@@ -789,7 +789,10 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
 #pragma unroll
             for (int j = 0; j < NT; ++j)
                 c4[j] = (j < ntok) ? load4(nc + j * N + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int s0 = cw * 8; s0 < T; s0 += CW * 8) {
+            // a tile that folds (fused flush) needs neither the B.C products nor
+            // the replay rows: its output comes from the folded state
+            const bool fold_now = FUSED && T == a.s.L;
+            for (int s0 = cw * 8; !fold_now && s0 < T; s0 += CW * 8) {
                 // B_s . C_j for slots s0..s0+7, reduced together; the 8 B rows
                 // are read once for all tokens
                 float4 bv[8];
@@ -840,7 +843,7 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                     pend_old = atomicAdd(&a.arrive[b], 1u);
                 }
             }
-            if (cw == (CW >= 3 ? 2 : 0)) {
+            if (!fold_now && cw == (CW >= 3 ? 2 : 0)) {
                 // append this call's x (and, for the group's first head, B) to the buffer
                 const int xq = ntok * xc, bq = ntok * bc;
                 uint4* xdst = reinterpret_cast<uint4*>(rec + a.rec.x + static_cast<size_t>(pos) * P * es);
@@ -852,7 +855,7 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
             }
         }
         group_sync(gi, CT);  // s_w, s_g, s_decay ready
-        if (ok) {
+        if (ok && !(FUSED && T == a.s.L)) {
             const unsigned char* tile = sp;
             const unsigned char* sc = sp + a.rec.scales;
             const float Dh = sc4[kMaxTok + 1];
@@ -992,7 +995,8 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
         if constexpr (FUSED != 0) {
             if (ok && T == a.s.L) {  // uniform over the group: the token that fills the buffer folds it
                 // h <- exp(A S_T) h + sum_s w_s x_s B_s^T with w_s = s_w[gi][0][s]
-                // (t = pos = T - 1), written over the checkpoint in the record
+                // (t = pos = T - 1), written over the checkpoint in the record.
+                // The folded state is h_t itself, so y_t = h_t C_t + D x_t.
                 const int x8 = P >> 3;
                 for (int c = ctid; c < T * x8; c += CT) {
                     const int sl = c / x8, p8 = (c - sl * x8) << 3;
@@ -1029,8 +1033,17 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                             acc[kk].w = fmaf(w[kk], bv.w, acc[kk].w);
                         }
                     }
+                    float part[kRB];
 #pragma unroll
-                    for (int kk = 0; kk < kRB; ++kk) stream_store4(ck + (r0 + kk) * N + 4 * lane, acc[kk]);
+                    for (int kk = 0; kk < kRB; ++kk) {
+                        stream_store4(ck + (r0 + kk) * N + 4 * lane, acc[kk]);
+                        part[kk] = dot4(acc[kk], c4[0]);
+                    }
+                    const float z = warp_reduce8(part);
+                    const int r = r0 + ((lane >> 2) & 7);
+                    if ((lane & 3) == 0)
+                        a.y[static_cast<size_t>(b) * HP + static_cast<size_t>(h) * P + r] =
+                            fmaf(sc4[kMaxTok + 1], to_f32(nx[r]), z);
                 }
             }
         }
