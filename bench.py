@@ -41,6 +41,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "SSM decode tokens/s at batch 256/512; achieved HBM GB/s vs B200 peak"
+WORKLOAD = ("small_b256: replay decode, batch 256, 64 heads, head_dim 64, d_state 128, 8 groups, fp32 checkpoint, "
+            "bf16 x/B/C, interval 16")
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -317,8 +319,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "small_b256: replay decode, batch 256, 64 heads, head_dim 64, d_state 128, "
-                               "8 groups, fp32 checkpoint, bf16 x/B/C, interval 16",
+        "config": {"workload": WORKLOAD,
                    "batch_per_gpu": shape.batch, "tokens_per_step": shape.batch * L * world,
                    "step": "16 x rssm_decode_step + " + ("fused fold" if args.fused else "1 x rssm_flush") +
                            ", replayed as a CUDA graph of the same launches",
@@ -745,9 +746,9 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "small_b256: replay decode, batch 256, 64 heads, head_dim 64, d_state 128, "
-                               "8 groups, interval 16",
-                   "step": "one request-interval (16 replay decodes + 1 flush) of the fp64 CPU oracle"},
+        "config": {"workload": WORKLOAD,
+                   "step": "one request-interval (16 replay decodes + 1 flush) of the fp64 CPU oracle, "
+                           "on requests of the same layer"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": f"{args.steps} request-intervals, single thread"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
