@@ -513,7 +513,7 @@ def spec_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
         rssm.rssm_accept(st, n_tab[s])
         rssm.rssm_flush(st, inp["A"])
 
-    def timed(fn, with_events):
+    def timed(fn, evs=None):
         for s in range(W):
             fn(s)
         torch.cuda.synchronize()
@@ -521,8 +521,8 @@ def spec_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
         a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         for i in range(K):
-            if with_events:
-                fn(W + i, ev_v[i])
+            if evs is not None:
+                fn(W + i, evs[i])
             else:
                 fn(W + i)
         e.record()
@@ -530,7 +530,7 @@ def spec_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
         barrier()
         return max_over_ranks(a.elapsed_time(e))
 
-    ms_r = timed(rstep, True)
+    ms_r = timed(rstep, ev_v)
     if rssm.rssm_get_error(st) != 0:
         raise RuntimeError("device error in the speculative leg")
     # verify bytes from the positions the accept table implies (pos += n + 1, folded at >= L)
@@ -546,6 +546,31 @@ def spec_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
     v_gbs = [vb / (m / 1e3) / 1e9 for vb, m in zip(vbytes, v_ms)]
     del st
     torch.cuda.empty_cache()
+    # the same speculative run on a split-precision state: verify reads the
+    # FP4 output copy, the refresh after accept updates the bf16 copy with SR
+    dsp = rssm.make_desc(shape.batch, shape.nheads, shape.head_dim, shape.d_state, shape.ngroups, interval=L,
+                         max_draft=Kd, update_dtype=rssm.RSSM_BF16, out_copy=rssm.RSSM_OUTCOPY_FP4, seed=wl["seed"])
+    st = rssm.RssmState(dsp, dev)
+    st.ckpt.copy_(inp["ckpt"].to(torch.bfloat16))
+    rssm.rssm_lowprec_refresh(st, inp["A"], force=True)
+    ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+
+    def sstep(s, ev=None):
+        w = s % WIN
+        if ev is not None:
+            ev[0].record()
+        rssm.rssm_verify(st, Kd, inp["x"][w], inp["B"][w], inp["C"][w], inp["dt"][w], inp["A"], inp["D"], ys)
+        if ev is not None:
+            ev[1].record()
+        rssm.rssm_accept(st, n_tab[s])
+        rssm.rssm_lowprec_refresh(st, inp["A"])
+
+    ms_s = timed(sstep, ev_s)
+    if rssm.rssm_get_error(st) != 0:
+        raise RuntimeError("device error in the split-precision speculative leg")
+    s_ms = [x.elapsed_time(y) for x, y in ev_s]
+    del st
+    torch.cuda.empty_cache()
     copies = torch.empty((Kd + 1,) + tuple(inp["ckpt"].shape), device=dev)
     copies[0].copy_(inp["ckpt"])
     cur = torch.zeros(shape.batch, dtype=torch.int32, device=dev)
@@ -556,7 +581,7 @@ def spec_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
                               inp["D"], ys)
         rssm.rssm_conv_accept(desc, n_tab[s], cur, Kd)
 
-    ms_c = timed(cstep, False)
+    ms_c = timed(cstep)
     del copies
     acc = world * int((n_host[W:W + K].long() + 1).sum())
     return {"workload": "spec_b512_k4: batch 512, 128 heads, 64 x 128, 8 groups, interval 16, K = 4 drafts, "
@@ -565,7 +590,10 @@ def spec_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
             "conventional_accepted_tokens_per_s": acc / (ms_c / 1e3), "speedup": ms_c / ms_r,
             "replay_step_us": ms_r / K * 1e3, "conventional_step_us": ms_c / K * 1e3,
             "verify_avg_launch_us": sum(v_ms) / len(v_ms) * 1e3,
-            "verify_gbs": statistics.mean(v_gbs), "verify_frac": statistics.mean(v_gbs) / peak}
+            "verify_gbs": statistics.mean(v_gbs), "verify_frac": statistics.mean(v_gbs) / peak,
+            "split_bf16_fp4": {"replay_accepted_tokens_per_s": acc / (ms_s / 1e3),
+                               "speedup_vs_conventional": ms_c / ms_s, "step_us": ms_s / K * 1e3,
+                               "verify_avg_launch_us": sum(s_ms) / len(s_ms) * 1e3}}
 
 
 def split_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):

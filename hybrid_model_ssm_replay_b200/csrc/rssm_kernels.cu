@@ -496,6 +496,16 @@ __global__ void __launch_bounds__(kThreads, replay_min_blocks(NT, FUSED)) k_repl
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t fdiv(uint32_t x, const FastDiv& f) { return (__umulhi(x, f.mul) + x) >> f.shr; }
 
+// Programmatic dependent launch (the persistent kernels are launched with
+// programmatic stream serialization): let the next kernel on the stream start
+// launching now -- its CTAs take an SM once this kernel's CTA there exits --
+// and wait until the previous kernel's writes are visible before reading any
+// global memory. Both are no-ops for a plain launch.
+__device__ __forceinline__ void pdl_prologue() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Barrier of one consumer group of nthr threads (named barrier 1 + gi),
 // returning the OR of v.
 __device__ __forceinline__ int group_sync_or(int gi, int nthr, int v) {
@@ -573,6 +583,7 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
     const size_t HP = static_cast<size_t>(H) * P, GN = static_cast<size_t>(G) * N;
     constexpr int es = static_cast<int>(sizeof(TIn));
 
+    pdl_prologue();
     if (tid == 0) {
         for (int st = 0; st < S; ++st) {
             mbar_init(smem_u32(&full_bar[st]), 1);
@@ -1271,6 +1282,7 @@ __global__ void __launch_bounds__(fold_threads(), 1) k_fold_pipe(const FoldArgs 
     const uint32_t tbu = tile_bytes(UF, P, N) + scale_bytes(UF, P, N);  // update copy (+ FP4 scales)
     const bool in_record = a.upd == a.record;
 
+    pdl_prologue();
     if (tid == 0) {
         for (int st = 0; st < S; ++st) {
             mbar_init(smem_u32(&full_bar[st]), 1);
@@ -1758,6 +1770,24 @@ static cudaError_t launch_tiles(K kernel, const Args& a, int nblk, size_t smem, 
     return cudaGetLastError();
 }
 
+// Launch with programmatic stream serialization (see pdl_prologue).
+template <typename K, typename A1, typename A2>
+static cudaError_t launch_pdl(K kernel, int grid, int threads, size_t smem, cudaStream_t st, const A1& a1,
+                              const A2& a2) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, a1, a2);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <typename K, typename... Args>
 static cudaError_t launch_grid(K kernel, const ReplayArgs& a, const PipeLayout& L, int grid, int threads,
                                size_t smem, cudaStream_t st) {
@@ -1767,8 +1797,7 @@ static cudaError_t launch_grid(K kernel, const ReplayArgs& a, const PipeLayout& 
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              static_cast<int>(cudaSharedmemCarveoutMaxShared));
     if (e != cudaSuccess) return e;
-    kernel<<<grid, threads, smem, st>>>(a, L);
-    return cudaGetLastError();
+    return launch_pdl(kernel, grid, threads, smem, st, a, L);
 }
 
 template <typename TIn, int NT, int W>
@@ -1934,8 +1963,7 @@ static cudaError_t fold_pipe_dispatch(const FoldArgs& a, const FoldPipeLayout& L
         e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  static_cast<int>(cudaSharedmemCarveoutMaxShared));
         if (e != cudaSuccess) return e;
-        kernel<<<grid, fold_threads(), smem, st>>>(a, L);
-        return cudaGetLastError();
+        return launch_pdl(kernel, grid, fold_threads(), smem, st, a, L);
     };
     if (a.out_fp4) {
         switch (uf) {
