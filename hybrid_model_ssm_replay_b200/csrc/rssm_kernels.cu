@@ -539,16 +539,18 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // on different tiles at once, which hides the latency chain of one tile
 // (barriers, shared-memory loads, shuffle reductions). The fp32 copy fills a
 // 39 KB stage per tile at the shapes served, so few tiles fit in shared
-// memory: three groups of four warps (two groups for verify of more than
-// kMidTok tokens, whose registers would spill). The smaller copies leave room
+// memory: three groups of four warps. Verify (K+1 tokens per tile) takes
+// three groups of four warps for every copy (two groups for more than kMidTok
+// tokens, whose registers would spill). Decode of the smaller copies has room
 // for many tiles: bf16 six groups of two warps; e4m3 and FP4 twelve groups of
-// one warp, each tile worked by one warp without group barriers (measured on
-// B200: FP4 decode 102 us with 6 x 2, 93 us with 12 x 1, 114 us with 8 x 1).
+// one warp, each tile worked by one warp without group barriers. (B200: FP4
+// decode 102 us with 6 x 2, 93 us with 12 x 1, 114 us with 8 x 1; FP4 verify
+// 1163 us with 12 x 1, 934 us with 3 x 4.)
 __host__ __device__ constexpr int pipe_groups(int nt, int rf) {
-    return rf == kF32 ? (nt <= kMidTok ? 3 : 2) : (rf == kBF16 || nt > kMidTok ? 6 : 12);
+    return nt > 1 ? (nt <= kMidTok ? 3 : 2) : (rf == kF32 ? 3 : (rf == kBF16 ? 6 : 12));
 }
 __host__ __device__ constexpr int pipe_cwarps(int nt, int rf) {
-    return rf == kF32 ? 4 : (rf == kBF16 && nt <= kMidTok ? 2 : 1);
+    return nt > 1 ? 4 : (rf == kF32 ? 4 : (rf == kBF16 ? 2 : 1));
 }
 __host__ __device__ constexpr int pipe_threads(int nt, int rf) {
     return (pipe_groups(nt, rf) * pipe_cwarps(nt, rf) + 1) * 32;
@@ -970,10 +972,11 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                         if (j < ntok) {
                             const int tt = pos + j;
                             const float dec = s_decay[gi][j];
+                            const float4 cd = make_float4(dec * c4[j].x, dec * c4[j].y, dec * c4[j].z, dec * c4[j].w);
                             const float coef = (lane <= tt) ? s_w[gi][j][lane] * s_g[gi][j][lane] : 0.f;
                             float part[8];
 #pragma unroll
-                            for (int kk = 0; kk < 8; ++kk) part[kk] = fmaf(coef, xv8[kk], dec * dot4(hv[kk], c4[j]));
+                            for (int kk = 0; kk < 8; ++kk) part[kk] = fmaf(coef, xv8[kk], dot4(hv[kk], cd));
                             const float z = warp_reduce8(part);
                             if ((lane & 3) == 0) yout[j * HP + rr] = fmaf(Dh, to_f32(nx[j * P + rr]), z);
                         }
