@@ -146,21 +146,29 @@ def test_fp4_decode_and_refresh_match_oracle(kind):
     assert st.flush_count.cpu().tolist() == [2] * 4
 
 
+# accepted drafts per step and request (steps x batch) for K = 4 and K = 6:
+# three requests reach the interval on the last step, one does not
+SPLIT_SPEC = {
+    4: np.array([[4, 3, 0, 4], [4, 4, 1, 4], [4, 4, 2, 3], [4, 4, 3, 4]], np.int32),   # pos 20 19 10 19
+    6: np.array([[6, 6, 0, 5], [6, 5, 1, 6], [2, 3, 2, 3]], np.int32),                 # pos 17 17 6 17
+}
+
+
+@pytest.mark.parametrize("K", [4, 6])
 @pytest.mark.parametrize("kind", ["bf16", "e4m3"])
-def test_speculative_verify_on_split_state_matches_oracle(kind):
+def test_speculative_verify_on_split_state_matches_oracle(kind, K):
     """Speculative decoding (s3) on a split-precision state (s4): verify of
-    the pending token and K = 4 drafts reads the FP4 output copy, accept(n)
-    advances pos, and the refresh after accept folds the requests whose
-    buffer reached the interval. Four steps, so every verify reads the
-    initial FP4 copy (pos <= 15 before the last accept); the outputs match
-    the oracle within the fp32 tolerance, and each refreshed request's update
-    and FP4 copies match it bit for bit except at fp32 rounding straddles."""
-    shape = LayerShape(4, 8, 64, 128, 2, interval=16, max_draft=4)
-    K, steps, L = 4, 4, 16
+    the pending token and K drafts (K = 4 and 6: the pipelined kernel's 5-
+    and 8-token bounds) reads the FP4 output copy, accept(n) advances pos,
+    and the refresh after accept folds the requests whose buffer reached the
+    interval. No request reaches the interval before the last accept, so
+    every verify reads the initial FP4 copy; the outputs match the oracle
+    within the fp32 tolerance, and each refreshed request's update and FP4
+    copies match it bit for bit except at fp32 rounding straddles."""
+    shape = LayerShape(4, 8, 64, 128, 2, interval=16, max_draft=K)
+    n_host = SPLIT_SPEC[K]
+    steps, L = n_host.shape[0], 16
     inp = make_inputs(shape, steps, 34, torch.bfloat16, device="cuda", ntok=K + 1)
-    # accepted drafts per step and request: three requests reach the interval
-    # on the last step (pos 20, 19, 19), one does not (pos 10)
-    n_host = np.array([[4, 3, 0, 4], [4, 4, 1, 4], [4, 4, 2, 3], [4, 4, 3, 4]], np.int32)
     n_acc = torch.from_numpy(n_host).cuda()
     seed = 0x5EED
     desc, st = split_state(shape, inp, kind, seed)

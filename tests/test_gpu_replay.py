@@ -129,6 +129,18 @@ def test_spec_b512_k4_sampled():
     check_spec_case(w["shape"], w["steps"], w["seed"], sample_requests(w["shape"].batch, 4), conv=True)
 
 
+@pytest.mark.parametrize("shape", [LayerShape(5, 4, 32, 128, 2, interval=16, max_draft=1),
+                                   LayerShape(5, 4, 32, 128, 2, interval=16, max_draft=6),
+                                   LayerShape(3, 4, 32, 128, 2, interval=27, max_draft=5)],
+                         ids=["k1", "k6", "cap32"])
+def test_spec_pipelined_drafts_and_capacity(shape):
+    """The pipelined verify at other draft counts (2 and 7 tokens per call,
+    under the kernel's 5- and 8-token bounds) and with the largest buffer
+    (interval 27 + 5 drafts = 32 slots: four 8-slot B.C blocks), every
+    request against the oracle, the conventional verify beside it."""
+    check_spec_case(shape, 40, 13, list(range(shape.batch)))
+
+
 def test_spec_rollback_leaves_no_trace():
     """verify K+1 then accept(n) gives the same later outputs and checkpoint as
     decoding only the n+1 accepted tokens (s3), on the GPU itself."""
