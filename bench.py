@@ -353,6 +353,8 @@ def run_ours(args):
         torch.cuda.empty_cache()
         out["split_b256"] = split_leg(rssm, torch, WORKLOADS["split_b256"], max(2, min(K, 50)), W, dev, barrier,
                                       max_over_ranks, world, peak)
+        torch.cuda.empty_cache()
+        out["prefill_b256"] = prefill_leg(rssm, torch, WORKLOADS["small_b256"], dev, barrier, max_over_ranks, world)
     if rank == 0 and world == 1 and not args.no_extra:
         out["cpu_baseline"] = cpu_baseline()
     if world > 1:
@@ -672,6 +674,38 @@ def split_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
         del st
         torch.cuda.empty_cache()
     return out
+
+
+def prefill_leg(rssm, torch, wl, dev, barrier, max_over_ranks, world, T0=512, reps=5):
+    """Prefill of a 512-token prompt into the fp32 checkpoint of the small
+    layer (rssm_prefill): prompt tokens/s and the fold's FMA rate against the
+    fp32 CUDA-core peak (148 SMs x 128 lanes x 2 flop x SM clock)."""
+    from hybrid_model_ssm_replay_b200.inputs import make_inputs
+    shape = wl["shape"]
+    inp = make_inputs(shape, T0, wl["seed"] + 11, wl["in_dtype"], device=dev)
+    desc = rssm.make_desc(shape.batch, shape.nheads, shape.head_dim, shape.d_state, shape.ngroups,
+                          interval=shape.interval)
+    st = rssm.RssmState(desc, dev)
+    st.ckpt.copy_(inp["ckpt"])
+    rssm.rssm_prefill(st, inp["x"], inp["B"], inp["dt"], inp["A"])
+    torch.cuda.synchronize()
+    barrier()
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        rssm.rssm_prefill(st, inp["x"], inp["B"], inp["dt"], inp["A"])
+    e.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(a.elapsed_time(e)) / reps
+    if rssm.rssm_get_error(st) != 0:
+        raise RuntimeError("device error in the prefill leg")
+    flops = 2.0 * shape.nheads * shape.head_dim * shape.d_state * T0 * shape.batch
+    peak_tf = 148 * 128 * 2 * 1.965e9 / 1e12
+    return {"workload": f"small_b256 shapes, prompt of {T0} tokens per request", "prompt_tokens_per_s":
+            world * shape.batch * T0 / (ms / 1e3), "ms_per_prefill": ms, "fold_tflops": flops / (ms / 1e3) / 1e12,
+            "bound": "alu", "peak_tflops": peak_tf, "frac": flops / (ms / 1e3) / 1e12 / peak_tf,
+            "peak_source": "148 SMs x 128 fp32 lanes x 2 flop x 1.965 GHz (nominal max SM clock)"}
 
 
 # ---------------------------------------------------- the CPU oracle arm

@@ -265,6 +265,28 @@ rssm_status_t rssm_lowprec_refresh(const rssm_desc_t* d, const rssm_state_t* st,
     return fold_launch(d, st, force ? 2 : 0, A, stream);
 }
 
+rssm_status_t rssm_prefill(const rssm_desc_t* d, const rssm_state_t* st, int32_t T0, const void* x, const void* B,
+                           const float* dt, const float* A, void* stream) {
+    rssm_status_t s = rssm_check_desc(d);
+    if (s != RSSM_OK) return s;
+    if (d->update_dtype != RSSM_F32 || d->out_copy != RSSM_OUTCOPY_NONE) return RSSM_ERR_UNSUPPORTED;
+    if (!st || !st->record || !st->pos || !st->err) return RSSM_ERR_INVALID_ARG;
+    if (T0 < 0) return RSSM_ERR_INVALID_ARG;
+    if (T0 > 0 && (!x || !B || !dt || !A)) return RSSM_ERR_INVALID_ARG;
+    PrefillArgs a;
+    a.s = shape_of(d);
+    a.T0 = T0;
+    a.rec = rec_of(d);
+    a.record = static_cast<unsigned char*>(st->record);
+    a.pos = st->pos;
+    a.err = st->err;
+    a.x = x;
+    a.B = B;
+    a.dt = dt;
+    a.A = A;
+    return cuda_status(launch_prefill(a, d->in_dtype == RSSM_BF16, static_cast<cudaStream_t>(stream)));
+}
+
 static rssm_status_t conv_launch(const rssm_desc_t* d, float* h, const int32_t* cur, int ntok, int32_t* err,
                                  const void* x, const void* B, const void* C, const float* dt, const float* A,
                                  const float* D, float* y, void* stream) {

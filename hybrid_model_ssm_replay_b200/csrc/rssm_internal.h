@@ -95,6 +95,20 @@ struct FoldArgs {
     const float* A;
 };
 
+// Prefill of T0 prompt tokens into the fp32 checkpoint (empty buffer).
+struct PrefillArgs {
+    Shape s;
+    int T0;
+    RecLayout rec;
+    unsigned char* record;
+    int32_t* pos;
+    int32_t* err;
+    const void* x;
+    const void* B;
+    const float* dt;
+    const float* A;
+};
+
 // Conventional step / verify (s1, s3: the scheme ReplaySSM replaces).
 struct ConvArgs {
     Shape s;
@@ -115,6 +129,7 @@ struct ConvArgs {
 // input element type.
 cudaError_t launch_replay(const ReplayArgs& a, int in_bf16, int read_fmt, cudaStream_t st);
 cudaError_t launch_fold(const FoldArgs& a, int in_bf16, int upd_fmt, cudaStream_t st);
+cudaError_t launch_prefill(const PrefillArgs& a, int in_bf16, cudaStream_t st);
 cudaError_t launch_conv(const ConvArgs& a, int in_bf16, int verify, cudaStream_t st);
 cudaError_t launch_accept(int batch, int K, int cap, const int32_t* n, int32_t* pos, int32_t* err, int add_one,
                           cudaStream_t st);

@@ -1578,6 +1578,107 @@ __global__ void __launch_bounds__(fold_threads(), 1) k_fold_pipe(const FoldArgs 
 }
 
 // ---------------------------------------------------------------------------
+// Prefill: the prompt folded into the fp32 checkpoint, kPrefillChunk tokens
+// at a time, with the fold of s1 (an interval flush of each chunk). One CTA
+// per tile keeps the tile in shared memory across chunks: per chunk the B
+// rows (fp32), the x rows and the weights dt_s exp(A (S_chunk - S_s)) are
+// staged, then the register-blocked rank-T update writes the tile back (the
+// last chunk writes the record).
+// ---------------------------------------------------------------------------
+constexpr int kPrefillChunk = 16;
+
+template <typename TIn>
+__global__ void __launch_bounds__(kThreads, 2) k_prefill(const PrefillArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ float s_cw[kPrefillChunk];
+    __shared__ float s_alpha;
+    __shared__ int s_pos;
+
+    const int H = a.s.H, P = a.s.P, N = a.s.N, G = a.s.G, lpr = a.s.lpr, batch = a.s.batch;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.x / H, h = blockIdx.x - b * H;
+    const int g = h / (H / G);
+    const int xs = round_up8(P);
+    const size_t bh = static_cast<size_t>(b) * H + h;
+    float* s32 = reinterpret_cast<float*>(smem);  // [P][N]
+    float* s_B = s32 + P * N;                      // [chunk][N]
+    float* s_x = s_B + kPrefillChunk * N;          // [chunk][xs]
+    unsigned char* rec = a.record + bh * a.rec.bytes;
+    const uint32_t tb = 4u * static_cast<uint32_t>(P * N);
+    const uint32_t bar_a = smem_u32(&bar);
+
+    if (tid == 0) {
+        const int p0 = a.pos[b];  // the only read of pos
+        s_pos = p0;
+        if (p0 == 0 && a.T0 > 0) {
+            mbar_init(bar_a, 1);
+            mbar_expect_tx(bar_a, tb);
+            bulk_g2s(smem_u32(s32), rec, tb, bar_a);
+        }
+    }
+    __syncthreads();
+    if (s_pos != 0) {
+        if (tid == 0) set_error(a.err, RSSM_DEVERR_POS_RANGE);
+        return;
+    }
+    if (a.T0 <= 0) return;
+    bool arrived = true;
+    if (tid == 0) arrived = mbar_wait_bounded(bar_a, 0, kWaitNs);
+    if (__syncthreads_or(!arrived)) {
+        if (tid == 0) {
+            set_error(a.err, RSSM_DEVERR_TIMEOUT);
+            mbar_wait_bounded(bar_a, 0, kWaitNs);
+        }
+        return;
+    }
+    const float Ah = a.A[h];
+    const size_t HP = static_cast<size_t>(H) * P, GN = static_cast<size_t>(G) * N;
+    const TIn* xin = static_cast<const TIn*>(a.x) + static_cast<size_t>(b) * HP + static_cast<size_t>(h) * P;
+    const TIn* Bin = static_cast<const TIn*>(a.B) + static_cast<size_t>(b) * GN + static_cast<size_t>(g) * N;
+    const size_t xstep = static_cast<size_t>(batch) * HP, bstep = static_cast<size_t>(batch) * GN;
+    const int n8 = N >> 3;
+    for (int t0 = 0; t0 < a.T0; t0 += kPrefillChunk) {
+        const int T = a.T0 - t0 < kPrefillChunk ? a.T0 - t0 : kPrefillChunk;
+        for (int q = tid; q < T * n8; q += kThreads) {
+            const int sl = q / n8, c8 = (q - sl * n8) << 3;
+            Raw8<TIn> r;
+            r.load(Bin + static_cast<size_t>(t0 + sl) * bstep + c8);
+            float4* d = reinterpret_cast<float4*>(s_B + sl * N + c8);
+            d[0] = r.lo();
+            d[1] = r.hi();
+        }
+        for (int i = tid; i < T * P; i += kThreads) {
+            const int sl = i / P, p = i - sl * P;
+            s_x[sl * xs + p] = to_f32(xin[static_cast<size_t>(t0 + sl) * xstep + p]);
+        }
+        if (warp == 0) {
+            const float dts = (lane < T) ? a.dt[(static_cast<size_t>(t0 + lane) * batch + b) * H + h] : 0.f;
+            const float Sx = warp_prefix(dts);
+            const float Stot = __shfl_sync(0xffffffffu, Sx, T - 1);
+            if (lane < kPrefillChunk) s_cw[lane] = (lane < T) ? dts * expf(Ah * (Stot - Sx)) : 0.f;
+            if (lane == 0) s_alpha = expf(Ah * Stot);
+        }
+        __syncthreads();  // chunk staged; the previous chunk's tile writes are visible
+        const bool last = t0 + kPrefillChunk >= a.T0;
+        auto brow = [&](int sl, int c) {
+            const float w = s_cw[sl];
+            const float4 v = reinterpret_cast<const float4*>(s_B + sl * N)[c];
+            return make_float4(w * v.x, w * v.y, w * v.z, w * v.w);
+        };
+        auto emit = [&](int r, int c, float4 v, bool valid) {
+            if (!valid) return;
+            if (last)
+                stream_store4(reinterpret_cast<float*>(rec) + r * N + 4 * c, v);
+            else
+                reinterpret_cast<float4*>(s32)[r * (N >> 2) + c] = v;
+        };
+        fold_tile(s32, s_x, xs, P, N, lpr, T, s_alpha, brow, emit);
+        __syncthreads();  // every reader of this chunk's staging is done
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Conventional scheme (in-run comparison, s1/s3): per token
 //   h <- exp(dt A) h + dt x B^T, write h, y = h C + D x.
 // VERIFY: read copy cur[b], write the state after token j to copy j.
@@ -2029,6 +2130,14 @@ cudaError_t launch_fold(const FoldArgs& a, int in_bf16, int uf, cudaStream_t st)
     const size_t smem = fold_smem_bytes(a.s, uf);
     const int nblk = a.s.batch * a.s.H;
     return in_bf16 ? fold_dispatch<__nv_bfloat16>(a, uf, smem, nblk, st) : fold_dispatch<float>(a, uf, smem, nblk, st);
+}
+
+cudaError_t launch_prefill(const PrefillArgs& a, int in_bf16, cudaStream_t st) {
+    const size_t smem = 4u * (static_cast<size_t>(a.s.P) * a.s.N + static_cast<size_t>(kPrefillChunk) * a.s.N +
+                              static_cast<size_t>(kPrefillChunk) * round_up8(a.s.P));
+    const int nblk = a.s.batch * a.s.H;
+    return in_bf16 ? launch_tiles(k_prefill<__nv_bfloat16>, a, nblk, smem, st)
+                   : launch_tiles(k_prefill<float>, a, nblk, smem, st);
 }
 
 cudaError_t launch_conv(const ConvArgs& a, int in_bf16, int verify, cudaStream_t st) {

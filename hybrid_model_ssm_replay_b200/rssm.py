@@ -75,6 +75,7 @@ def lib():
         "rssm_verify": ([D, S, i32, vp, vp, vp, vp, vp, vp, vp, vp], ct.c_int),
         "rssm_accept": ([D, S, vp, vp], ct.c_int),
         "rssm_lowprec_refresh": ([D, S, vp, i32, vp], ct.c_int),
+        "rssm_prefill": ([D, S, i32, vp, vp, vp, vp, vp], ct.c_int),
         "rssm_conv_step": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp], ct.c_int),
         "rssm_conv_verify": ([D, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp], ct.c_int),
         "rssm_conv_accept": ([D, vp, vp, i32, vp, vp], ct.c_int),
@@ -248,6 +249,16 @@ def rssm_accept(state, n_accepted, stream=None):
 def rssm_lowprec_refresh(state, A, force=False, stream=None):
     _check(lib().rssm_lowprec_refresh(ct.byref(state.desc), ct.byref(state.struct), _ptr(A, torch.float32, "A"),
                                       int(bool(force)), _stream(stream)), "rssm_lowprec_refresh")
+
+
+def rssm_prefill(state, x, B, dt, A, stream=None):
+    """Fold a prompt of T0 = x.shape[0] tokens into the fp32 checkpoint (pos must be 0)."""
+    d = state.desc
+    in_dt = _IN_DT[d.in_dtype]
+    T0 = int(x.shape[0])
+    _check(lib().rssm_prefill(ct.byref(d), ct.byref(state.struct), T0, _ptr(x, in_dt, "x"), _ptr(B, in_dt, "B"),
+                              _ptr(dt, torch.float32, "dt"), _ptr(A, torch.float32, "A"), _stream(stream)),
+           "rssm_prefill")
 
 
 def rssm_conv_step(desc, h, x, B, C, dt, A, D, y, stream=None):

@@ -257,6 +257,21 @@ RSSM_API rssm_status_t rssm_accept(const rssm_desc_t *desc, const rssm_state_t *
 RSSM_API rssm_status_t rssm_lowprec_refresh(const rssm_desc_t *desc, const rssm_state_t *state,
                                    const float *A, int32_t force, void *stream);
 
+/* Prefill of a prompt into the checkpoint -- the step before the decode path,
+ * on which the article is silent: for every request, folds T0 prompt tokens
+ * into the fp32 checkpoint with an empty buffer, chunk by chunk,
+ *     h <- exp(A S) h + sum_{t<T0} dt_t exp(A (S - S_t)) x_t B_t^T,  S = sum of the T0 dt,
+ * which is the conventional recurrence over the prompt, started from the
+ * current checkpoint (zero it first for a fresh request). pos stays 0,
+ * flush_count is unchanged; no outputs are produced.
+ *   x [T0][batch][H][P], B [T0][batch][G][N] (in_dtype); dt [T0][batch][H]
+ *   float (softplus-ed); A [H] float.
+ * Requires an fp32 state (update_dtype F32, no output copy), else
+ * RSSM_ERR_UNSUPPORTED; T0 >= 0. Device error: pos[b] != 0 (request untouched). */
+RSSM_API rssm_status_t rssm_prefill(const rssm_desc_t *desc, const rssm_state_t *state, int32_t T0,
+                                    const void *x, const void *B, const float *dt, const float *A,
+                                    void *stream);
+
 /* Conventional decode step, the in-run comparison (s1: read and write the
  * whole state every token): h <- a h + dt x B^T; y = h C + D x.
  * h [batch][H][P][N] float, updated in place; other arguments as in

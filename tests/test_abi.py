@@ -127,6 +127,11 @@ def test_host_validation_needs_no_device(L):
     assert L.rssm_get_error(ct.byref(d), None, None, None) == 1
     assert L.rssm_round_test(9, 16, p, 0, 0, 0, 0, p, None) == 1
     assert L.rssm_round_test(3, 15, p, 0, 0, 0, 0, p, None) == 2
+    # prefill: fp32 state only, T0 >= 0, inputs needed when T0 > 0
+    assert L.rssm_prefill(ct.byref(dl), ct.byref(st), 4, p, p, p, p, None) == 3
+    assert L.rssm_prefill(ct.byref(d), ct.byref(st), -1, p, p, p, p, None) == 1
+    assert L.rssm_prefill(ct.byref(d), ct.byref(st), 4, null, p, p, p, None) == 1
+    assert L.rssm_prefill(ct.byref(bad), ct.byref(st), 4, p, p, p, p, None) == 2
     assert rssm.status_string(4) == "more tokens than the buffer capacity"
 
 
