@@ -1263,13 +1263,17 @@ struct FoldPipeLayout {
 // meta words of a fold stage: tile index (-1: end), position, flush count, A_h, tag
 constexpr int kFMetaTile = 0, kFMetaPos = 1, kFMetaFc = 2, kFMetaA = 3, kFMetaTag = 4;
 
-__host__ __device__ constexpr int fold_groups() { return 3; }
-__host__ __device__ constexpr int fold_cwarps() { return 4; }
-__host__ __device__ constexpr int fold_threads() { return (fold_groups() * fold_cwarps() + 1) * 32; }
+// Consumer groups of four warps: three for the fp32 flush (bound by HBM;
+// B200: 190 us with 3 groups, 196 with 4), four for the low-precision
+// refreshes, which are bound by issue (Philox draws, rounding, FP4
+// quantisation; bf16 refresh 478 -> 430 us with 4 groups).
+__host__ __device__ constexpr int fold_groups(int uf) { return uf == kF32 ? 3 : 4; }
+__host__ __device__ constexpr int fold_cwarps(int uf) { return (void)uf, 4; }
+__host__ __device__ constexpr int fold_threads(int uf) { return (fold_groups(uf) * fold_cwarps(uf) + 1) * 32; }
 
 template <typename TIn, int UF, int OUT4>
-__global__ void __launch_bounds__(fold_threads(), 1) k_fold_pipe(const FoldArgs a, const FoldPipeLayout lay) {
-    constexpr int CG = fold_groups(), CW = fold_cwarps(), CT = CW * 32;
+__global__ void __launch_bounds__(fold_threads(UF), 1) k_fold_pipe(const FoldArgs a, const FoldPipeLayout lay) {
+    constexpr int CG = fold_groups(UF), CW = fold_cwarps(UF), CT = CW * 32;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full_bar[kPipeStagesMax];
     __shared__ __align__(8) uint64_t empty_bar[kPipeStagesMax];
@@ -2061,13 +2065,14 @@ static cudaError_t fold_dispatch(const FoldArgs& a, int uf, size_t smem, int nbl
 template <typename TIn>
 static cudaError_t fold_pipe_dispatch(const FoldArgs& a, const FoldPipeLayout& L, int uf, int grid, size_t smem,
                                       cudaStream_t st) {
+    const int threads = fold_threads(uf);
     auto go = [&](auto kernel) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  static_cast<int>(cudaSharedmemCarveoutMaxShared));
         if (e != cudaSuccess) return e;
-        return launch_pdl(kernel, grid, fold_threads(), smem, st, a, L);
+        return launch_pdl(kernel, grid, threads, smem, st, a, L);
     };
     if (a.out_fp4) {
         switch (uf) {
@@ -2103,7 +2108,7 @@ static FoldPipeLayout fold_pipe_layout(const FoldArgs& a, int uf, int in_bf16, s
     L.meta = L.brows + align16(static_cast<uint32_t>(s.cap * s.N) * es);
     L.stage_bytes = (L.meta + 64u + 127u) & ~127u;
     L.scratch = (4u * static_cast<uint32_t>(s.cap) * (s.N + s.P) + 127u) & ~127u;
-    const size_t rows = static_cast<size_t>(fold_groups()) * L.scratch;
+    const size_t rows = static_cast<size_t>(fold_groups(uf)) * L.scratch;
     const size_t n = budget > rows ? (budget - rows) / L.stage_bytes : 0;
     L.stages = static_cast<int>(n < static_cast<size_t>(kPipeStagesMax) ? n : kPipeStagesMax);
     L.divH = make_fastdiv(static_cast<uint32_t>(s.H));
@@ -2121,7 +2126,7 @@ cudaError_t launch_fold(const FoldArgs& a, int in_bf16, int uf, cudaStream_t st)
                 const int ntiles = a.s.batch * a.s.H;
                 const int grid = ntiles < di.sms ? ntiles : di.sms;
                 const size_t smem = static_cast<size_t>(L.stages) * L.stage_bytes +
-                                    static_cast<size_t>(fold_groups()) * L.scratch;
+                                    static_cast<size_t>(fold_groups(uf)) * L.scratch;
                 return in_bf16 ? fold_pipe_dispatch<__nv_bfloat16>(a, L, uf, grid, smem, st)
                                : fold_pipe_dispatch<float>(a, L, uf, grid, smem, st);
             }
