@@ -195,7 +195,7 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
 //   buffered dt. The new tokens are appended at slots pos..pos+ntok-1.
 //   While the tile streams in, the CTA stages x_s of every slot in shared
 //   memory, forms the decay weights (warp 0) and the B_s . C_j products
-//   (all warps), in two rounds of independent loads (this call's inputs
+//   (all warps), in two batches of independent loads (this call's inputs
 //   with pos, then the buffered slots). After the tile lands, each row's
 //   output is one reduction over the row's lanes of the h.C dot product and
 //   the replay terms (lane l takes slots s = l mod lanes).
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, replay_min_blocks(NT, FUSED)) k_repl
         s_pos = a.pos[b];  // the only read of pos: every thread uses this copy
     }
 
-    // ---- round 0: C rows, this call's x and dt (with the position, above)
+    // ---- first loads: C rows, this call's x and dt (with the position, above)
     float4 c4[NT];
 #pragma unroll
     for (int j = 0; j < NT; ++j)
@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, replay_min_blocks(NT, FUSED)) k_repl
 
     if (ok) {
         const float Ah = a.A[h];
-        // ---- round 1 (independent loads): the buffered slots s < pos and this
+        // ---- second loads (independent): the buffered slots s < pos and this
         // call's tokens -> shared memory; this call's tokens -> the buffer
         if constexpr (WIDE) {
             Raw8<TIn> xr;
