@@ -28,7 +28,11 @@
  *  - Inputs are read-only; layouts are dense and row-major as documented.
  *    Device pointers must be 16-byte aligned.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream). Work is
- *    enqueued asynchronously; one state must be used from one stream.
+ *    enqueued asynchronously; one state must be used from one stream. The
+ *    persistent kernels (decode, verify, flush, refresh at d_state 128) are
+ *    launched with programmatic stream serialization: they wait for the
+ *    previous kernel's writes on entry, and the next kernel on the stream may
+ *    begin launching before they finish. Calls can be captured in CUDA graphs.
  *  - Arguments the host can check are checked before anything is launched;
  *    a bad one returns a status and launches nothing.
  *  - Kernels that find bad device state (a buffer position out of range, an
