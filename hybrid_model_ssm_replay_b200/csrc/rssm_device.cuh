@@ -1,6 +1,6 @@
 // rssm_device.cuh -- device-side building blocks of librssm (sm_100a).
 //
-//  * shared-memory bulk copies (cp.async.bulk, completion on an mbarrier)
+//  * shared-memory bulk copies (cp.async.bulk, completion on an mbarrier),
 //    and waits bounded by %globaltimer, so no kernel can spin forever;
 //  * Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers:
 //    As Easy as 1, 2, 3", SC'11);
@@ -18,13 +18,13 @@
 
 namespace rssm {
 
-constexpr int kThreads = 256;               // threads per CTA of every tile kernel
+constexpr int kThreads = 256;               // threads per CTA of the one-CTA-per-tile kernels
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxCap = 32;                 // buffer slots per request (interval + drafts)
 constexpr int kMaxTok = 8;                  // tokens per verify call (K + 1)
 constexpr int kMidTok = 5;                  // verify kernels specialised for K <= 4
 constexpr int kPipeStagesMax = 16;          // shared-memory stages of the pipelined kernels
-constexpr unsigned long long kWaitNs = 2000000000ull;  // bound of one bulk-copy wait
+constexpr unsigned long long kWaitNs = 2000000000ull;  // bound of every wait (mbarrier, stage tag)
 
 // ------------------------------------------------------------------ errors
 

@@ -1,20 +1,25 @@
 // rssm_kernels.cu -- sm_100a kernels of librssm.
 //
-// Every tile kernel runs one CTA of 256 threads per (request b, head h).
-// The CTA's state tile (P x N, one head of one request, contiguous in HBM)
-// is brought into shared memory by one bulk copy (cp.async.bulk, completion
-// on an mbarrier) issued before anything else, so the HBM stream starts at
-// once and overlaps the small per-token work (buffer reads, decay weights,
-// B.C dot products). Rows are then read from shared memory by warps: the
-// lanes of a row each hold 4 consecutive d_state elements and reduce with
-// shuffles. There are no float atomics; every result has a fixed summation
-// order, so runs are bit-reproducible.
+// The hot path at d_state 128 (head_dim a multiple of 8) runs two
+// persistent, warp-specialised kernels, one CTA per SM:
+//   k_replay_pipe  decode, verify, fused decode + flush: a producer warp
+//                  fills a ring of shared-memory stages with bulk copies of
+//                  each (request, head) record and its B rows; consumer warp
+//                  groups compute the outputs from shared memory;
+//   k_fold_pipe    interval flush and precision-split refresh: the same
+//                  producer/consumer ring over the requests that are due.
+// Other shapes run one CTA of 256 threads per (request, head) tile
+// (k_replay, k_fold), the tile brought in by one bulk copy issued first.
+// k_prefill folds a prompt into the checkpoint; k_conv is the conventional
+// per-token scheme kept for comparison. Rows are reduced across the lanes
+// that hold their columns with shuffles; there are no float atomics, every
+// result has a fixed summation order, and runs are bit-reproducible.
 //
 // Method: ReplaySSM article (devotd.net
 // "nvidia-replayssm-hybrid-model-ssm-decoding-state-buffer"):
-//   s1 "Store recent inputs instead of the full state"     -> k_replay, k_fold
-//   s3 "Roll back incorrect predictions using buffer positions" -> k_replay (verify), k_accept
-//   s4 "Prevent low-precision errors from accumulating again"   -> k_fold (refresh), FP4 reads
+//   s1 "Store recent inputs instead of the full state"          -> k_replay_pipe, k_fold_pipe (k_replay, k_fold)
+//   s3 "Roll back incorrect predictions using buffer positions" -> verify in k_replay_pipe, k_accept
+//   s4 "Prevent low-precision errors from accumulating again"   -> refresh in k_fold_pipe, FP4 reads
 //   conventional scheme of s1/s3 (in-run comparison)            -> k_conv
 #include "rssm_device.cuh"
 #include "rssm_internal.h"
