@@ -45,3 +45,24 @@ def test_single_rank_identity():
     import bench
     assert bench.reduce_max(3.0) == 3.0
     assert bench.job_throughput(100, 1, 1000.0) == pytest.approx(100.0)
+
+
+def test_reference_arm_under_torchrun_prints_one_line():
+    """bench.py --impl reference launched as the driver launches it for N > 1
+    (torchrun, two ranks): rank 0 alone runs the oracle and prints the one
+    JSON line; the other rank exits 0 without work."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--impl", "reference",
+           "--gpus", "2", "--steps", "2", "--warmup", "1"]
+    r = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    for k in ("metric", "unit", "higher_is_better", "config", "cpu_baseline", "e2e"):
+        assert k in d
