@@ -46,8 +46,8 @@ def copy_bits(t):
     return t.numpy()
 
 
-def split_state(shape, inp, kind, seed):
-    desc = desc_for(shape, update_dtype=UPD[kind][0], out_copy=rssm.RSSM_OUTCOPY_FP4, seed=seed)
+def split_state(shape, inp, kind, seed, in_dtype=torch.bfloat16):
+    desc = desc_for(shape, in_dtype, update_dtype=UPD[kind][0], out_copy=rssm.RSSM_OUTCOPY_FP4, seed=seed)
     st = rssm.RssmState(desc)
     st.ckpt.copy_(initial_update_copy(inp["ckpt"], kind))
     rssm.rssm_lowprec_refresh(st, inp["A"], force=True)      # builds the FP4 output copy
@@ -100,8 +100,9 @@ def spacing(v, kind):
     return np.exp2(e - 3)
 
 
+@pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32], ids=["bf16in", "f32in"])
 @pytest.mark.parametrize("kind", ["bf16", "e4m3"])
-def test_fp4_decode_and_refresh_match_oracle(kind):
+def test_fp4_decode_and_refresh_match_oracle(kind, in_dtype):
     """One interval from a prepared split state: every output read from the
     FP4 copy matches the oracle (fp32 vs fp64 on exact dequantised values).
     The refreshed update copy and FP4 copy match the oracle bit for bit
@@ -112,9 +113,9 @@ def test_fp4_decode_and_refresh_match_oracle(kind):
     (1e-5 rms of the state)."""
     shape = LayerShape(4, 8, 64, 128, 2)
     L = shape.interval
-    inp = make_inputs(shape, L, 31, torch.bfloat16, device="cuda")
+    inp = make_inputs(shape, L, 31, in_dtype, device="cuda")
     seed = 0xBEEF
-    desc, st = split_state(shape, inp, kind, seed)
+    desc, st = split_state(shape, inp, kind, seed, in_dtype)
     # the oracle starts from the input recipe and its own FP4 quantiser
     upd0 = copy_bits(initial_update_copy(inp["ckpt"], kind))
     codes0, scales0 = orc.fp4_quant(orc.widen(UPD[kind][1], upd0, None, upd0.shape).astype(np.float32))

@@ -97,11 +97,11 @@ def test_large_shape_batch_sweep(batch):
 
 # ----------------------------------------------------------- speculative
 
-def check_spec_case(shape, steps, seed, reqs, conv=True):
+def check_spec_case(shape, steps, seed, reqs, conv=True, in_dtype=torch.bfloat16):
     K = shape.max_draft
-    inp = make_inputs(shape, steps, seed, torch.bfloat16, device="cuda", ntok=K + 1)
+    inp = make_inputs(shape, steps, seed, in_dtype, device="cuda", ntok=K + 1)
     n_acc = accept_lengths(steps, shape.batch, K, seed, device="cuda")
-    desc = desc_for(shape)
+    desc = desc_for(shape, in_dtype)
     y, st = gpu_spec(desc, inp, n_acc, steps)
     n_np = n_acc.cpu().numpy()
     res = oracle_map([("spec", request_inputs(inp, b), (n_np[:, b], shape.interval, K)) for b in reqs])
@@ -139,6 +139,13 @@ def test_spec_pipelined_drafts_and_capacity(shape):
     (interval 27 + 5 drafts = 32 slots: four 8-slot B.C blocks), every
     request against the oracle, the conventional verify beside it."""
     check_spec_case(shape, 40, 13, list(range(shape.batch)))
+
+
+@pytest.mark.parametrize("K", [4, 6])
+def test_spec_pipelined_fp32_inputs(K):
+    """The pipelined verify with fp32 x/B/C (its float-input instantiations)."""
+    shape = LayerShape(4, 4, 32, 128, 2, interval=16, max_draft=K)
+    check_spec_case(shape, 30, 17, list(range(shape.batch)), in_dtype=torch.float32)
 
 
 def test_spec_rollback_leaves_no_trace():
