@@ -223,6 +223,39 @@ def test_shared_fp4_control_decode_matches_oracle(shape):
         assert np.mean(st.ckpt[b].cpu().numpy() == req.codes) > 0.998
 
 
+@pytest.mark.parametrize("kind", ["bf16", "e4m3"])
+def test_shared_copy_decode_and_refresh_match_oracle(kind):
+    """One bf16 or e4m3 copy both read by decode and updated by the refresh
+    (the secondary shared-precision control of s4): the outputs match the
+    oracle reading the same values, and the stochastically rounded copy
+    matches it bit for bit except at fp32 rounding straddles."""
+    shape = LayerShape(4, 8, 64, 128, 2)
+    L = shape.interval
+    inp = make_inputs(shape, L, 36, torch.bfloat16, device="cuda")
+    seed = 0xC0FFEE
+    desc = desc_for(shape, update_dtype=UPD[kind][0], seed=seed)
+    st = rssm.RssmState(desc)
+    st.ckpt.copy_(initial_update_copy(inp["ckpt"], kind))
+    upd0 = copy_bits(initial_update_copy(inp["ckpt"], kind))
+    y = torch.empty((L, 4, 8, 64), device="cuda")
+    for t in range(L):
+        rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"], y[t])
+    rssm.rssm_lowprec_refresh(st, inp["A"])
+    assert rssm.rssm_get_error(st) == 0
+    mism = total = 0
+    for b in range(shape.batch):
+        r = request_inputs(inp, b)
+        req = orc.LowPrecRequest(UPD[kind][1], False, upd0[b], None, None, shape.ngroups, L, r["A"], r["D"], seed, b)
+        ys = np.stack([req.decode(r["x"][t], r["B"][t], r["C"][t], r["dt"][t]) for t in range(L)])
+        assert_close(to_np(y[:, b]), ys, f"shared {kind} decode, request {b}")
+        req.refresh()
+        got = copy_bits(st.ckpt[b]).ravel()
+        mism += int(np.count_nonzero(got != req.upd.ravel()))
+        total += got.size
+    assert mism <= 1e-3 * total, mism
+    assert st.flush_count.cpu().tolist() == [1] * 4 and st.pos.cpu().tolist() == [0] * 4
+
+
 def run_lowprec(desc, st, inp, steps):
     y = torch.empty((steps,) + tuple(inp["x"].shape[1:]), device="cuda")
     for t in range(steps):
