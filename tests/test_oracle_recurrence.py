@@ -189,7 +189,7 @@ def test_tiny_workload_replay_equals_recurrence():
     assert torch.is_tensor(inp["x"])
 
 
-@pytest.mark.parametrize("K", [1, 4])
+@pytest.mark.parametrize("K", [1, 4, 6, 7])
 def test_verify_then_accept_equals_decoding_accepted(K):
     """For every n in 0..K: verify of K+1 tokens then accept(n) gives, for
     tokens 0..n, the outputs of plain decode, and leaves the same state."""
@@ -232,11 +232,13 @@ def test_verify_rejects_overflow():
     req.verify(pr["x"][0], pr["B"][0], pr["C"][0], pr["dt"][0])
 
 
-def test_spec_run_equals_recurrence_on_accepted_stream():
+@pytest.mark.parametrize("L,K", [(16, 4), (16, 1), (16, 6), (27, 5)])
+def test_spec_run_equals_recurrence_on_accepted_stream(L, K):
     """A whole speculative run (verify K+1, accept n, flush at L) gives, for
-    the accepted tokens, the outputs of the recurrence over those tokens."""
-    rng = np.random.default_rng(7)
-    H, P, N, G, L, K, S = 4, 3, 5, 2, 16, 4, 30
+    the accepted tokens, the outputs of the recurrence over those tokens --
+    including the largest buffer (27 + 5 = 32 slots)."""
+    rng = np.random.default_rng(7 + K + L)
+    H, P, N, G, S = 4, 3, 5, 2, 30
     pr = rand_problem(rng, S, H, P, N, G, ntok=K + 1)
     n_acc = rng.integers(0, K + 1, S)
     ys, ck, poss = orc.run_spec(pr["ckpt"], pr["x"], pr["B"], pr["C"], pr["dt"], pr["A"], pr["D"],
