@@ -57,8 +57,9 @@ def parse_args():
     p.add_argument("--fused", action="store_true", help="fold the buffer inside the 16th decode (no flush call)")
     p.add_argument("--no-extra", action="store_true",
                    help="skip the comparison, large-layer, e2e and CPU-baseline legs")
-    p.add_argument("--profile", action="store_true",
-                   help="untimed: run every hot kernel a few times on the bench workloads (for ncu)")
+    p.add_argument("--profile", nargs="?", const="all", default=None,
+                   help="untimed: run hot kernels a few times on the bench workloads (for ncu); "
+                        "a comma-separated list of sections, or all")
     return p.parse_args()
 
 
@@ -236,84 +237,13 @@ def run_ours(args):
     wl = WORKLOADS["small_b256"]
     shape = wl["shape"]
     L = shape.interval
-    WIN = 2 * L  # distinct tokens of inputs, cycled
-    inp = make_inputs(shape, WIN, wl["seed"] + rank, wl["in_dtype"], device=dev)
-    flags = rssm.RSSM_FLAG_FUSED_FLUSH if args.fused else 0
-    desc = rssm.make_desc(shape.batch, shape.nheads, shape.head_dim, shape.d_state, shape.ngroups,
-                          interval=L, flags=flags)
-    st = rssm.RssmState(desc, dev)
-    st.ckpt.copy_(inp["ckpt"])
-    y = torch.empty((L, shape.batch, shape.nheads, shape.head_dim), device=dev)
-    stream = torch.cuda.current_stream()
-    n_dec = K * L
-    ev_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_dec)]
-    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-
-    def step(k, timed):
-        base = (k % (WIN // L)) * L
-        for i in range(L):
-            t = base + i
-            if timed:
-                ev_d[k * L + i][0].record(stream)
-            rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"],
-                                  y[i])
-            if timed:
-                ev_d[k * L + i][1].record(stream)
-        if not args.fused:
-            if timed:
-                ev_f[k][0].record(stream)
-            rssm.rssm_flush(st, inp["A"])
-            if timed:
-                ev_f[k][1].record(stream)
-
-    sampler = ClockSampler(smi_gpu_id(torch, local))
-    sampler.start()
-    for k in range(W):
-        step(k, False)
-    torch.cuda.synchronize()
-    # per-launch kernel times: one eager pass of K steps, each launch bracketed by events
-    for k in range(K):
-        step(k, True)
-    torch.cuda.synchronize()
-    # the timed steps replay CUDA graphs of one step per input window (the
-    # same launches, without the host's launch gaps)
-    graphs = []
-    for w in range(WIN // L):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step(w, False)
-        graphs.append(g)
-    st.pos.zero_()
-    st.ckpt.copy_(inp["ckpt"])
-    for k in range(W):
-        graphs[k % len(graphs)].replay()
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_wall0 = time.time()
-    start.record(stream)
-    for k in range(K):
-        graphs[k % len(graphs)].replay()
-    end.record(stream)
-    torch.cuda.synchronize()
-    t_wall1 = time.time()
-    barrier()
-    torch.cuda.synchronize()
-    ms_local = start.elapsed_time(end)
-    ms = max_over_ranks(ms_local)
-    if rssm.rssm_get_error(st) != 0:
-        raise RuntimeError("device error during the timed run")
-    del graphs
-    time.sleep(0.06)
-    sampler.stop()
-    clocks = sampler.summary(t_wall0, t_wall1)
-
-    value = job_throughput(shape.batch * L * K, world, ms)
-    dec_ms = [a.elapsed_time(b) for a, b in ev_d]
-    dec_avg_ms = sum(dec_ms) / len(dec_ms)
-    dec_bytes = sum(decode_bytes_per_request(shape, i) for i in range(L)) / L * shape.batch
     peak, peak_src = measured_peaks()
+    main = replay_loop(rssm, torch, shape, wl, K, W, dev, rank, barrier, max_over_ranks, world, args.fused,
+                       repeats=0 if args.no_extra else 5)
+    ms = main["ms"]
+    value = job_throughput(shape.batch * L * K, world, ms)
+    dec_avg_ms = main["decode_us"] / 1e3
+    dec_bytes = sum(decode_bytes_per_request(shape, i) for i in range(L)) / L * shape.batch
     achieved = dec_bytes / (dec_avg_ms / 1e3) / 1e9
     traffic = ncu_traffic("replay_decode_small_b256")
     out = {
@@ -322,37 +252,64 @@ def run_ours(args):
         "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD,
                    "batch_per_gpu": shape.batch, "tokens_per_step": shape.batch * L * world,
-                   "step": "16 x rssm_decode_step + " + ("fused fold" if args.fused else "1 x rssm_flush") +
-                           ", replayed as a CUDA graph of the same launches",
+                   "step": ("16 x rssm_decode_step with the fused fold on the 16th" if args.fused else
+                            "16 x rssm_decode_step + 1 x rssm_flush") +
+                           ", replayed as CUDA graphs of the same launches (the 16 decodes, then the flush), "
+                           "with CUDA events between the graphs",
                    "l2": "no flush: the 512 MiB fp32 state read each token exceeds the 126 MB L2",
                    "parallelism": f"replicas x{world} (independent requests)"},
         "roofline": {"kernel": "k_replay_pipe (rssm_decode_step)", "bound": "hbm", "achieved": achieved,
                      "peak": peak, "peak_source": peak_src, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "algorithmic_bytes_per_launch": dec_bytes,
-                     "avg_launch_us": dec_avg_ms * 1e3,
+                     "traffic": traffic,
+                     "traffic_source": None if traffic is None else
+                     "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, from the summary under "
+                     "profiles/ taken on this kernel source (matched by source hash), not measured in this run",
+                     "algorithmic_bytes_per_launch": dec_bytes,
+                     "avg_launch_us": main["decode_us"],
+                     "launch_time_source": "CUDA events on the launching stream around each replay of the "
+                                           "16-decode graph inside the timed region, / 16",
                      "achieved_dram": None if traffic is None else traffic / (dec_avg_ms / 1e3) / 1e9,
                      "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
                      "nominal_peak": NOMINAL_HBM_GBS},
         "gpu_launches": K * (L + (0 if args.fused else 1)),
-        "clocks": clocks,
+        "clocks": main["clocks"],
     }
+    if main.get("repeats"):
+        out["repeats"] = main["repeats"]
+    if not args.fused:
+        fl_us = main["flush_us"]
+        fl_bytes = flush_bytes_per_request(shape, L) * shape.batch
+        out["flush_kernel"] = {"kernel": "k_fold_pipe (rssm_flush)", "avg_launch_us": fl_us,
+                               "achieved_gbs": fl_bytes / (fl_us / 1e6) / 1e9,
+                               "frac": fl_bytes / (fl_us / 1e6) / 1e9 / peak,
+                               "launch_time_source": "CUDA events around each replay of the flush graph inside the "
+                                                     "timed region"}
+        out["roofline"]["reconcile_us"] = {"16_decode_plus_flush": 16 * main["decode_us"] + fl_us,
+                                           "step": ms / K * 1e3}
+    inp, st = main["inp"], main["state"]
     rp = read_peak(torch, dev)
     out["roofline"]["read_peak_gbs"] = rp
     out["roofline"]["frac_of_read_peak"] = achieved / rp
     out["roofline"]["read_peak_source"] = "in-run: torch.sum over 4 GiB of fp32 (a library read-only kernel), best of 5"
-    if not args.fused:
-        fl_ms = [a.elapsed_time(b) for a, b in ev_f]
-        fl_avg = sum(fl_ms) / len(fl_ms)
-        fl_bytes = flush_bytes_per_request(shape, L) * shape.batch
-        out["flush_kernel"] = {"avg_launch_us": fl_avg * 1e3, "achieved_gbs": fl_bytes / (fl_avg / 1e3) / 1e9,
-                               "frac": fl_bytes / (fl_avg / 1e3) / 1e9 / peak}
     if not args.no_extra:
         out["conventional"] = conv_leg(rssm, torch, shape, inp, K, W, dev, barrier, max_over_ranks, world, peak)
         out["speedup_vs_conventional"] = value / out["conventional"]["value"]
+        out["bytes_saved_ratio"] = bytes_saved_ratio(shape, fused=args.fused)
         out["e2e"] = e2e_leg(rssm, torch, st, shape, inp, max(2, min(K, 20)), W, dev, barrier, max_over_ranks,
                              world, args.fused)
-        del st, inp, y
+        del st, inp, main
         torch.cuda.empty_cache()
+        if not args.fused:
+            fz = replay_loop(rssm, torch, shape, wl, K, W, dev, rank, barrier, max_over_ranks, world, True)
+            fz_value = job_throughput(shape.batch * L * K, world, fz["ms"])
+            out["fused_b256"] = {"step": "16 x rssm_decode_step with RSSM_FLAG_FUSED_FLUSH (the 16th decode folds "
+                                         "the buffer; no flush call)", "value": fz_value, "unit": UNIT,
+                                 "ms_per_step": fz["ms"] / K, "decode_avg_launch_us": fz["decode_us"],
+                                 "speedup_vs_conventional": fz_value / out["conventional"]["value"],
+                                 "bytes_saved_ratio": bytes_saved_ratio(shape, fused=True),
+                                 "vs_separate_flush": fz_value / value}
+            del fz
+            torch.cuda.empty_cache()
         out["large_b512"] = large_leg(rssm, torch, WORKLOADS["large_b512"], max(2, min(K, 50)), W, dev, barrier,
                                       max_over_ranks, world, peak, args.fused)
         torch.cuda.empty_cache()
@@ -363,12 +320,212 @@ def run_ours(args):
                                       max_over_ranks, world, peak)
         torch.cuda.empty_cache()
         out["prefill_b256"] = prefill_leg(rssm, torch, WORKLOADS["small_b256"], dev, barrier, max_over_ranks, world)
+        torch.cuda.empty_cache()
+        out["batch_sweep_large"] = sweep_leg(rssm, torch, WORKLOADS["large_b512"], max(2, min(K, 20)), W, dev,
+                                             barrier, max_over_ranks, world, peak)
     if rank == 0 and world == 1 and not args.no_extra:
         out["cpu_baseline"] = cpu_baseline()
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out))
+
+
+def replay_loop(rssm, torch, shape, wl, K, W, dev, rank, barrier, max_over_ranks, world, fused, repeats=0):
+    """The headline loop: K steps of one interval each (16 decodes + the
+    flush, or 16 decodes with the fused fold), replayed as CUDA graphs -- one
+    graph of the 16 decodes per input window and one graph of the flush --
+    with CUDA events between the graph launches on the launching stream.
+    The events give the per-kernel averages inside the timed region; the
+    first and last give the time of the K steps. repeats > 0 re-runs the
+    timed region that many more times (the median-of-runs protocol)."""
+    from hybrid_model_ssm_replay_b200.inputs import make_inputs
+    L = shape.interval
+    WIN = 2 * L  # distinct tokens of inputs, cycled
+    inp = make_inputs(shape, WIN, wl["seed"] + rank, wl["in_dtype"], device=dev)
+    flags = rssm.RSSM_FLAG_FUSED_FLUSH if fused else 0
+    desc = rssm.make_desc(shape.batch, shape.nheads, shape.head_dim, shape.d_state, shape.ngroups,
+                          interval=L, flags=flags)
+    st = rssm.RssmState(desc, dev)
+    st.ckpt.copy_(inp["ckpt"])
+    y = torch.empty((L, shape.batch, shape.nheads, shape.head_dim), device=dev)
+    stream = torch.cuda.current_stream()
+
+    def decodes(w):
+        for i in range(L):
+            t = w * L + i
+            rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"], y[i])
+
+    def flush():
+        rssm.rssm_flush(st, inp["A"])
+
+    # eager warm-up (loads the kernels, sets their attributes), then capture
+    for k in range(W):
+        decodes(k % (WIN // L))
+        if not fused:
+            flush()
+    torch.cuda.synchronize()
+    g_dec = []
+    for w in range(WIN // L):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            decodes(w)
+        g_dec.append(g)
+    g_fl = None
+    if not fused:
+        g_fl = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_fl):
+            flush()
+    st.pos.zero_()
+    st.ckpt.copy_(inp["ckpt"])
+
+    def run(k):
+        g_dec[k % len(g_dec)].replay()
+        if g_fl is not None:
+            g_fl.replay()
+
+    for k in range(W):
+        run(k)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(smi_gpu_id(torch, dev.index if dev.index is not None else 0))
+    sampler.start()
+    time.sleep(0.15)
+
+    def timed_region():
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K + 1)]
+        barrier()
+        torch.cuda.synchronize()
+        for k in range(K):
+            ev[2 * k].record(stream)
+            g_dec[k % len(g_dec)].replay()
+            ev[2 * k + 1].record(stream)
+            if g_fl is not None:
+                g_fl.replay()
+        ev[2 * K].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[2 * K])
+        dec = sum(ev[2 * k].elapsed_time(ev[2 * k + 1]) for k in range(K)) / (K * L)
+        fl = sum(ev[2 * k + 1].elapsed_time(ev[2 * k + 2]) for k in range(K)) / K
+        return ms, dec, fl
+
+    t0 = time.time()
+    ms_local, dec_ms, fl_ms = timed_region()
+    t1 = time.time()
+    ms = max_over_ranks(ms_local)
+    if rssm.rssm_get_error(st) != 0:
+        raise RuntimeError("device error during the timed run")
+    res = {"ms": ms, "decode_us": dec_ms * 1e3, "flush_us": fl_ms * 1e3 if not fused else None,
+           "inp": inp, "state": st}
+    if repeats:
+        runs = []
+        for _ in range(repeats):
+            m, d, f = timed_region()
+            runs.append((max_over_ranks(m), d, f))
+        vals = sorted(world * shape.batch * L * K / (m / 1e3) for m, _, _ in runs)
+        res["repeats"] = {"runs": repeats, "steps_each": K, "unit": UNIT,
+                          "median": statistics.median(vals), "min": vals[0], "max": vals[-1],
+                          "decode_us_median": statistics.median(d * 1e3 for _, d, _ in runs),
+                          "flush_us_median": None if fused else statistics.median(f * 1e3 for _, _, f in runs),
+                          "note": "the same timed region run again after the contract run"}
+    time.sleep(0.06)
+    sampler.stop()
+    res["clocks"] = sampler.summary(t0, t1)
+    del g_dec, g_fl
+    return res
+
+
+def bytes_saved_ratio(shape, fused=False):
+    """Conventional bytes per token / replay bytes per token (an interval of
+    16 decodes plus the flush, or the fused fold), algorithmic."""
+    L = shape.interval
+    b = shape_bytes(shape)
+    rep = sum(decode_bytes_per_request(shape, i) for i in range(L))
+    if fused:
+        rep += b["state"] - b["entry"]  # the filling token writes the folded state instead of its entry
+    else:
+        rep += flush_bytes_per_request(shape, L)
+    return conv_bytes_per_request(shape) * L / rep
+
+
+def sweep_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak, batches=(1, 32, 128, 512)):
+    """The large layer (128 heads, 64 x 128, 8 groups) at batch 1, 32, 128
+    and 512: replay (16 decodes + flush per step) against the conventional
+    step, each step a CUDA graph. "hot" replays the steps back to back (at
+    batch 1 and 32 the state, 4 and 128 MiB, stays in the 126 MB L2 or
+    nearly); "l2_flushed" writes a 256 MiB buffer before each step, outside
+    the events that time the step."""
+    from hybrid_model_ssm_replay_b200.inputs import LayerShape, make_inputs
+    base = wl["shape"]
+    L = base.interval
+    res = {"workload": "large layer shapes (128 heads, head_dim 64, d_state 128, 8 groups, interval 16)",
+           "steps": K, "points": []}
+    scrub = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for bsz in batches:
+        shape = LayerShape(bsz, base.nheads, base.head_dim, base.d_state, base.ngroups, L)
+        inp = make_inputs(shape, L, wl["seed"], wl["in_dtype"], device=dev)
+        desc = rssm.make_desc(bsz, shape.nheads, shape.head_dim, shape.d_state, shape.ngroups, interval=L)
+        st = rssm.RssmState(desc, dev)
+        st.ckpt.copy_(inp["ckpt"])
+        h = inp["ckpt"].clone()
+        y = torch.empty((bsz, shape.nheads, shape.head_dim), device=dev)
+
+        def rstep():
+            for i in range(L):
+                rssm.rssm_decode_step(st, inp["x"][i], inp["B"][i], inp["C"][i], inp["dt"][i], inp["A"], inp["D"], y)
+            rssm.rssm_flush(st, inp["A"])
+
+        def cstep():
+            for i in range(L):
+                rssm.rssm_conv_step(desc, h, inp["x"][i], inp["B"][i], inp["C"][i], inp["dt"][i], inp["A"],
+                                    inp["D"], y)
+
+        point = {"batch": bsz, "state_mib": 4 * shape.nheads * shape.head_dim * shape.d_state * bsz / 2 ** 20}
+        for name, fn in (("replay", rstep), ("conventional", cstep)):
+            for _ in range(W):
+                fn()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            for _ in range(W):
+                g.replay()
+            torch.cuda.synchronize()
+            barrier()
+            a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(K):
+                g.replay()
+            e.record()
+            torch.cuda.synchronize()
+            hot = max_over_ranks(a.elapsed_time(e)) / K
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+            for i in range(K):
+                scrub.fill_(i & 0xFF)
+                evs[i][0].record()
+                g.replay()
+                evs[i][1].record()
+            torch.cuda.synchronize()
+            barrier()
+            cold = max_over_ranks(statistics.median(x.elapsed_time(z) for x, z in evs))
+            point[name] = {"hot_tokens_per_s": world * bsz * L / (hot / 1e3), "hot_ms_per_step": hot,
+                           "l2_flushed_tokens_per_s": world * bsz * L / (cold / 1e3), "l2_flushed_ms_per_step": cold}
+            del g
+        rb = (sum(decode_bytes_per_request(shape, i) for i in range(L)) + flush_bytes_per_request(shape, L)) * bsz
+        point["replay"]["l2_flushed_frac"] = rb / (point["replay"]["l2_flushed_ms_per_step"] / 1e3) / 1e9 / peak
+        cb = conv_bytes_per_request(shape) * L * bsz
+        point["conventional"]["l2_flushed_frac"] = cb / (point["conventional"]["l2_flushed_ms_per_step"] / 1e3) / 1e9 / peak
+        point["speedup_hot"] = point["conventional"]["hot_ms_per_step"] / point["replay"]["hot_ms_per_step"]
+        point["speedup_l2_flushed"] = (point["conventional"]["l2_flushed_ms_per_step"] /
+                                       point["replay"]["l2_flushed_ms_per_step"])
+        res["points"].append(point)
+        if rssm.rssm_get_error(st) != 0:
+            raise RuntimeError("device error in the batch sweep")
+        del st, h, inp, y
+        torch.cuda.empty_cache()
+    del scrub
+    return res
 
 
 def read_peak(torch, dev, nbytes=4 << 30, reps=5):
@@ -869,11 +1026,23 @@ def run_reference(args):
     }))
 
 
-def run_profile():
-    """Each hot kernel a few times, untimed, on the small_b256 layer: 2
-    intervals of replay decode + flush, the same with the fused fold, 32
-    conventional steps, 4 speculative steps (K = 4, replay and conventional)
-    and one interval of the bf16 + FP4 precision split."""
+PROFILE_SECTIONS = ("decode", "fused", "conv", "spec", "conv_verify", "split_bf16", "split_e4m3", "shared_fp4",
+                    "prefill")
+
+
+def run_profile(sections):
+    """Hot kernels on the bench workloads, untimed, for ncu. Sections (run in
+    this order, each on the small_b256 layer unless noted):
+      decode       2 intervals of 16 rssm_decode_step + rssm_flush
+      fused        2 intervals with RSSM_FLAG_FUSED_FLUSH
+      conv         32 rssm_conv_step
+      spec         4 steps of rssm_verify (K = 4) + accept + flush (the last forced)
+      conv_verify  4 steps of rssm_conv_verify (K = 4) + rssm_conv_accept
+      split_bf16   bf16 + FP4 split: refresh(force), 16 decodes, refresh
+      split_e4m3   the same with an e4m3 update copy
+      shared_fp4   the shared FP4 control: refresh(force) of an fp32 + FP4
+                   state to build the copy, 16 decodes, refresh
+      prefill      rssm_prefill of a 64-token prompt"""
     import torch
 
     from hybrid_model_ssm_replay_b200 import rssm
@@ -884,61 +1053,97 @@ def run_profile():
     L = sh.interval
     inp = make_inputs(sh, L, wl["seed"], wl["in_dtype"], device="cuda")
     y = torch.empty((sh.batch, sh.nheads, sh.head_dim), device="cuda")
-    for flags in (0, rssm.RSSM_FLAG_FUSED_FLUSH):
-        d = rssm.make_desc(sh.batch, sh.nheads, sh.head_dim, sh.d_state, sh.ngroups, interval=L, flags=flags)
-        st = rssm.RssmState(d)
-        st.ckpt.copy_(inp["ckpt"])
-        for _ in range(2):
-            for t in range(L):
-                rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"], y)
-            if not flags:
-                rssm.rssm_flush(st, inp["A"])
-        del st
-    d = rssm.make_desc(sh.batch, sh.nheads, sh.head_dim, sh.d_state, sh.ngroups)
-    h = inp["ckpt"].clone()
-    for t in range(2 * L):
-        rssm.rssm_conv_step(d, h, inp["x"][t % L], inp["B"][t % L], inp["C"][t % L], inp["dt"][t % L], inp["A"],
-                            inp["D"], y)
-    del h
-    K = 4
-    ssh = LayerShape(sh.batch, sh.nheads, sh.head_dim, sh.d_state, sh.ngroups, L, K)
-    si = make_inputs(ssh, 4, 3, wl["in_dtype"], device="cuda", ntok=K + 1)
-    n = accept_lengths(4, sh.batch, K, 3, device="cuda")
-    ds = rssm.make_desc(sh.batch, sh.nheads, sh.head_dim, sh.d_state, sh.ngroups, interval=L, max_draft=K)
-    st = rssm.RssmState(ds)
-    st.ckpt.copy_(si["ckpt"])
-    ys = torch.empty((sh.batch, K + 1, sh.nheads, sh.head_dim), device="cuda")
-    for s in range(4):
-        rssm.rssm_verify(st, K, si["x"][s], si["B"][s], si["C"][s], si["dt"][s], si["A"], si["D"], ys)
-        rssm.rssm_accept(st, n[s])
-        rssm.rssm_flush(st, si["A"], force=(s == 3))
-    del st
-    copies = torch.zeros((K + 1,) + tuple(si["ckpt"].shape), device="cuda")
-    copies[0].copy_(si["ckpt"])
-    cur = torch.zeros(sh.batch, dtype=torch.int32, device="cuda")
-    for s in range(4):
-        rssm.rssm_conv_verify(ds, copies, cur, K, si["x"][s], si["B"][s], si["C"][s], si["dt"][s], si["A"],
-                              si["D"], ys)
-        rssm.rssm_conv_accept(ds, n[s], cur, K)
-    del copies
-    dl = rssm.make_desc(sh.batch, sh.nheads, sh.head_dim, sh.d_state, sh.ngroups, interval=L,
-                        update_dtype=rssm.RSSM_BF16, out_copy=rssm.RSSM_OUTCOPY_FP4, seed=4)
-    st = rssm.RssmState(dl)
-    st.ckpt.copy_(inp["ckpt"].to(torch.bfloat16))
-    rssm.rssm_lowprec_refresh(st, inp["A"], force=True)
-    for t in range(L):
-        rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"], y)
-    rssm.rssm_lowprec_refresh(st, inp["A"])
-    torch.cuda.synchronize()
-    if rssm.rssm_get_error(st) != 0:
-        raise RuntimeError("device error")
-    print("profile run done")
+    mk = lambda **kw: rssm.make_desc(sh.batch, sh.nheads, sh.head_dim, sh.d_state, sh.ngroups, interval=L, **kw)
+
+    def decodes(st):
+        for t in range(L):
+            rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"], y)
+
+    def check(st):
+        torch.cuda.synchronize()
+        if rssm.rssm_get_error(st) != 0:
+            raise RuntimeError("device error")
+
+    for sec in sections:
+        if sec in ("decode", "fused"):
+            st = rssm.RssmState(mk(flags=rssm.RSSM_FLAG_FUSED_FLUSH if sec == "fused" else 0))
+            st.ckpt.copy_(inp["ckpt"])
+            for _ in range(2):
+                decodes(st)
+                if sec == "decode":
+                    rssm.rssm_flush(st, inp["A"])
+            check(st)
+        elif sec == "conv":
+            d = mk()
+            h = inp["ckpt"].clone()
+            for t in range(2 * L):
+                rssm.rssm_conv_step(d, h, inp["x"][t % L], inp["B"][t % L], inp["C"][t % L], inp["dt"][t % L],
+                                    inp["A"], inp["D"], y)
+            torch.cuda.synchronize()
+            del h
+        elif sec in ("spec", "conv_verify"):
+            K = 4
+            ssh = LayerShape(sh.batch, sh.nheads, sh.head_dim, sh.d_state, sh.ngroups, L, K)
+            si = make_inputs(ssh, 4, 3, wl["in_dtype"], device="cuda", ntok=K + 1)
+            n = accept_lengths(4, sh.batch, K, 3, device="cuda")
+            ds = mk(max_draft=K)
+            ys = torch.empty((sh.batch, K + 1, sh.nheads, sh.head_dim), device="cuda")
+            if sec == "spec":
+                st = rssm.RssmState(ds)
+                st.ckpt.copy_(si["ckpt"])
+                for s_ in range(4):
+                    rssm.rssm_verify(st, K, si["x"][s_], si["B"][s_], si["C"][s_], si["dt"][s_], si["A"], si["D"], ys)
+                    rssm.rssm_accept(st, n[s_])
+                    rssm.rssm_flush(st, si["A"], force=(s_ == 3))
+                check(st)
+            else:
+                copies = torch.zeros((K + 1,) + tuple(si["ckpt"].shape), device="cuda")
+                copies[0].copy_(si["ckpt"])
+                cur = torch.zeros(sh.batch, dtype=torch.int32, device="cuda")
+                for s_ in range(4):
+                    rssm.rssm_conv_verify(ds, copies, cur, K, si["x"][s_], si["B"][s_], si["C"][s_], si["dt"][s_],
+                                          si["A"], si["D"], ys)
+                    rssm.rssm_conv_accept(ds, n[s_], cur, K)
+                torch.cuda.synchronize()
+                del copies
+        elif sec in ("split_bf16", "split_e4m3"):
+            upd = rssm.RSSM_BF16 if sec == "split_bf16" else rssm.RSSM_E4M3
+            st = rssm.RssmState(mk(update_dtype=upd, out_copy=rssm.RSSM_OUTCOPY_FP4, seed=4))
+            st.ckpt.copy_(inp["ckpt"].to(torch.bfloat16 if upd == rssm.RSSM_BF16 else torch.float8_e4m3fn)
+                          .view(st.ckpt.dtype))
+            rssm.rssm_lowprec_refresh(st, inp["A"], force=True)
+            decodes(st)
+            rssm.rssm_lowprec_refresh(st, inp["A"])
+            check(st)
+        elif sec == "shared_fp4":
+            s0 = rssm.RssmState(mk(out_copy=rssm.RSSM_OUTCOPY_FP4))
+            s0.ckpt.copy_(inp["ckpt"])
+            rssm.rssm_lowprec_refresh(s0, inp["A"], force=True)
+            st = rssm.RssmState(mk(update_dtype=rssm.RSSM_FP4, seed=4))
+            st.ckpt.copy_(s0.out_codes)
+            st.ckpt_scales.copy_(s0.out_scales)
+            del s0
+            decodes(st)
+            rssm.rssm_lowprec_refresh(st, inp["A"])
+            check(st)
+        elif sec == "prefill":
+            T0 = 64
+            pi = make_inputs(sh, T0, wl["seed"] + 11, wl["in_dtype"], device="cuda")
+            st = rssm.RssmState(mk())
+            st.ckpt.copy_(pi["ckpt"])
+            rssm.rssm_prefill(st, pi["x"], pi["B"], pi["dt"], pi["A"])
+            check(st)
+        else:
+            raise ValueError(f"unknown profile section {sec!r}; choose from {PROFILE_SECTIONS}")
+        st = None
+        torch.cuda.empty_cache()
+    print("profile run done:", ",".join(sections))
 
 
 def main():
     args = parse_args()
     if args.profile:
-        run_profile()
+        run_profile(PROFILE_SECTIONS if args.profile == "all" else args.profile.split(","))
         return
     if args.impl == "reference":
         run_reference(args)

@@ -25,6 +25,8 @@
 #include "rssm_internal.h"
 #include "rssm.h"
 
+#include <atomic>
+
 namespace rssm {
 
 __host__ __device__ inline uint32_t tile_bytes(int fmt, int P, int N) {
@@ -1833,17 +1835,21 @@ __global__ void k_round_test(int op, int64_t n, const float* v, uint64_t seed, u
 static __device__ __align__(256) uint32_t g_noalloc_arrive[RSSM_NOALLOC_MAX_BATCH];
 
 // Device address of g_noalloc_arrive on the current device, looked up once
-// per device (cudaGetSymbolAddress) and cached. nullptr when the lookup fails.
+// per device (cudaGetSymbolAddress) and cached. nullptr when the lookup
+// fails. Host threads may race on the first lookup: each stores the same
+// address, and the atomics make that well defined.
 uint32_t* noalloc_arrive_scratch() {
-    static uint32_t* cache[64] = {};
+    static std::atomic<uint32_t*> cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (cache[dev] == nullptr) {
+    uint32_t* p = cache[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_arrive) != cudaSuccess) return nullptr;
-        cache[dev] = static_cast<uint32_t*>(ptr);
+        p = static_cast<uint32_t*>(ptr);
+        cache[dev].store(p, std::memory_order_release);
     }
-    return cache[dev];
+    return p;
 }
 
 // ------------------------------------------------------------------ host
@@ -1972,18 +1978,28 @@ struct DeviceInfo {
     size_t smem_optin = 0;
 };
 
+// SM count and opt-in shared memory of the current device, queried once per
+// device. The query is idempotent; concurrent first calls store the same
+// values (the SM count last, with release order, so a reader that sees it
+// also sees the shared-memory size).
 static DeviceInfo device_info() {
-    static DeviceInfo cache[64];
+    static std::atomic<int> sms_cache[64];
+    static std::atomic<size_t> smem_cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DeviceInfo{};
-    if (cache[dev].sms == 0) {
+    DeviceInfo di;
+    di.sms = sms_cache[dev].load(std::memory_order_acquire);
+    if (di.sms == 0) {
         int sms = 0, optin = 0;
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-        cache[dev].smem_optin = static_cast<size_t>(optin);
-        cache[dev].sms = sms;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return DeviceInfo{};
+        smem_cache[dev].store(static_cast<size_t>(optin), std::memory_order_relaxed);
+        sms_cache[dev].store(sms, std::memory_order_release);
+        di.sms = sms;
     }
-    return cache[dev];
+    di.smem_optin = smem_cache[dev].load(std::memory_order_relaxed);
+    return di;
 }
 
 template <typename TIn, int NT>

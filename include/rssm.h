@@ -217,11 +217,17 @@ RSSM_API rssm_status_t rssm_flush(const rssm_desc_t *desc, const rssm_state_t *s
  * with cudaMemsetAsync on `stream` and launches the decode kernel.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    before any stream capture. The address is cached per device for the
+ *    life of the process: after a device reset, reload the library.
  *  - All calls share the one array: calls whose work overlaps on the GPU
  *    (other streams, concurrent graphs) race on it. Serialise them.
  *  - batch > RSSM_NOALLOC_MAX_BATCH returns RSSM_ERR_CAPACITY and launches
- *    nothing. */
+ *    nothing.
+ *  - Only the decode step has this variant. rssm_flush, rssm_lowprec_refresh
+ *    and rssm_verify still need state->arrive, so a caller that cannot
+ *    allocate at all runs allocation-free from start to end only with an
+ *    fp32 state (update_dtype F32, no output copy) and RSSM_FLAG_FUSED_FLUSH,
+ *    where the decode step itself folds the buffer. */
 RSSM_API rssm_status_t rssm_decode_step_noalloc(const rssm_desc_t *desc, const rssm_state_t *state,
                                                 const void *x, const void *B, const void *C,
                                                 const float *dt, const float *A, const float *D,

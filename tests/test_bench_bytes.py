@@ -29,3 +29,16 @@ def test_small_layer_bytes():
                bench.flush_bytes_per_request(sh, 16)) / 16
     assert per_tok == 2_487_936
     assert abs(4_223_232 / per_tok - 1.697) < 1e-3
+
+
+def test_bytes_saved_ratio():
+    """Conventional bytes per token over replay bytes per token: 1.697 with
+    the separate flush; with the fused fold the filling token writes the
+    folded state (2,097,152 B) instead of its buffer entry (10,496 B) and no
+    flush runs: (35,444,736 + 2,097,152 - 10,496) / 16 = 2,345,712 B per
+    token, ratio 1.800."""
+    sh = WORKLOADS["small_b256"]["shape"]
+    assert abs(bench.bytes_saved_ratio(sh) - 4_223_232 / 2_487_936) < 1e-12
+    assert sum(bench.decode_bytes_per_request(sh, t) for t in range(16)) == 35_444_736
+    assert abs(bench.bytes_saved_ratio(sh, fused=True) - 4_223_232 * 16 / (35_444_736 + 2_097_152 - 10_496)) < 1e-12
+    assert abs(bench.bytes_saved_ratio(sh, fused=True) - 1.800) < 1e-3

@@ -67,6 +67,57 @@ def fp4_control_state(shape, inp, seed):
     return desc, st
 
 
+def widened(kind, st):
+    """The values of a state's low-precision update copy, widened exactly to
+    fp32 on the device (bf16 / e4m3 casts are exact)."""
+    if kind == "bf16":
+        return st.ckpt.float()
+    if kind == "e4m3":
+        return st.ckpt.view(torch.float8_e4m3fn).float()
+    raise ValueError(kind)
+
+
+def f32_twin(shape, values, seed, in_dtype=torch.bfloat16, out_copy=True):
+    """An fp32 update copy holding exactly `values` (fp32), with an FP4
+    output copy when out_copy. Refreshing it runs the same fold as the
+    low-precision state it shadows -- same inputs, same operation order --
+    and stores the fp32 result unrounded: that result is what the
+    low-precision refresh rounds."""
+    desc = desc_for(shape, in_dtype, update_dtype=rssm.RSSM_F32,
+                    out_copy=rssm.RSSM_OUTCOPY_FP4 if out_copy else rssm.RSSM_OUTCOPY_NONE, seed=seed)
+    st = rssm.RssmState(desc)
+    st.ckpt.copy_(values)
+    return desc, st
+
+
+def assert_refresh_bits(kind, seed, st, twin, fc_before, requests, what):
+    """Kernel-level bit-exactness of a refresh (s4): for every refreshed
+    request the update copy equals the oracle's stochastic rounding, and the
+    FP4 copies equal the oracle's FP4 quantisation, of the fp32 values the
+    GPU fold produced (read from the fp32 twin). Zero mismatches."""
+    for b in requests:
+        v32 = twin.ckpt[b].cpu().numpy()                          # [H][P][N] float32
+        if kind in ("bf16", "e4m3"):
+            got = copy_bits(st.ckpt[b])
+            for h in range(v32.shape[0]):
+                exp = orc.sr_head(UPD[kind][1], seed, b, h, int(fc_before[b]), v32[h])
+                bad = int(np.count_nonzero(got[h].ravel() != exp.ravel()))
+                assert bad == 0, f"{what}: request {b} head {h}: {bad} update-copy elements differ"
+        codes, scales = orc.fp4_quant(v32)
+        for name, t in (("FP4 output copy", st.out_codes if kind != "fp4" else st.ckpt),
+                        ("FP4 twin copy", twin.out_codes)):
+            if t is None:
+                continue
+            bad = int(np.count_nonzero(t[b].cpu().numpy() != codes))
+            assert bad == 0, f"{what}: request {b}: {bad} codes of the {name} differ"
+        for name, t in (("FP4 output scales", st.out_scales if kind != "fp4" else st.ckpt_scales),
+                        ("FP4 twin scales", twin.out_scales)):
+            if t is None:
+                continue
+            bad = int(np.count_nonzero(t[b].cpu().numpy() != scales))
+            assert bad == 0, f"{what}: request {b}: {bad} scales of the {name} differ"
+
+
 # d_state 64 runs the one-CTA-per-tile fold, d_state 128 the persistent pipelined one
 SHAPES = [LayerShape(3, 4, 32, 64, 2), LayerShape(3, 4, 32, 128, 2)]
 
@@ -86,65 +137,55 @@ def test_refresh_at_empty_buffer_builds_fp4_copy_bit_exact(kind, shape):
     assert rssm.rssm_get_error(st) == 0
 
 
-def copy_values(bits, kind):
-    return orc.widen(UPD[kind][1], np.ascontiguousarray(bits).ravel())
+# the pipelined fold (d_state 128) and the one-CTA-per-tile fold (d_state 64)
+SPLIT_SHAPES = [LayerShape(4, 8, 64, 128, 2), LayerShape(3, 4, 32, 64, 2)]
 
 
-def spacing(v, kind):
-    """Distance to the next representable magnitude above |v| (bf16 or e4m3)."""
-    a = np.abs(np.asarray(v, np.float64))
-    if kind == "bf16":
-        e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
-        return np.exp2(e - 7)
-    e = np.floor(np.log2(np.maximum(a, 2.0 ** -6)))
-    return np.exp2(e - 3)
-
-
+@pytest.mark.parametrize("shape", SPLIT_SHAPES, ids=["dstate128", "dstate64"])
 @pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32], ids=["bf16in", "f32in"])
 @pytest.mark.parametrize("kind", ["bf16", "e4m3"])
-def test_fp4_decode_and_refresh_match_oracle(kind, in_dtype):
+def test_fp4_decode_and_refresh_match_oracle(kind, in_dtype, shape):
     """One interval from a prepared split state: every output read from the
     FP4 copy matches the oracle (fp32 vs fp64 on exact dequantised values).
-    The refreshed update copy and FP4 copy match the oracle bit for bit
-    except where the fp32 fold (GPU) and the fp64 fold rounded to fp32
-    (oracle) straddle a rounding threshold: at least 99.9% of the elements
-    agree exactly, and every element of the update copy lies within one
-    spacing of the oracle's unrounded value plus the fp32 fold error
-    (1e-5 rms of the state)."""
-    shape = LayerShape(4, 8, 64, 128, 2)
+    The refresh is pinned at kernel level: an fp32 twin state starting from
+    the same (widened) update-copy values runs the same fold, and the
+    refreshed update copy and FP4 copy equal, bit for bit, the oracle's
+    stochastic rounding and FP4 quantisation of that fp32 result, with zero
+    mismatches. The fp32 fold itself matches the oracle's fp64 fold within
+    the fp32 tolerance."""
     L = shape.interval
+    Bz, H, P = shape.batch, shape.nheads, shape.head_dim
     inp = make_inputs(shape, L, 31, in_dtype, device="cuda")
     seed = 0xBEEF
     desc, st = split_state(shape, inp, kind, seed, in_dtype)
+    _, tw = f32_twin(shape, widened(kind, st), seed, in_dtype)
+    rssm.rssm_lowprec_refresh(tw, inp["A"], force=True)
+    assert np.array_equal(tw.out_codes.cpu().numpy(), st.out_codes.cpu().numpy())
     # the oracle starts from the input recipe and its own FP4 quantiser
     upd0 = copy_bits(initial_update_copy(inp["ckpt"], kind))
     codes0, scales0 = orc.fp4_quant(orc.widen(UPD[kind][1], upd0, None, upd0.shape).astype(np.float32))
-    y = torch.empty((L, 4, 8, 64), device="cuda")
+    y = torch.empty((L, Bz, H, P), device="cuda")
+    y2 = torch.empty_like(y)
     for t in range(L):
-        rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"], y[t])
+        args = (inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"])
+        rssm.rssm_decode_step(st, *args, y[t])
+        rssm.rssm_decode_step(tw, *args, y2[t])
+    fc_before = st.flush_count.cpu().tolist()
     rssm.rssm_lowprec_refresh(st, inp["A"])
-    assert rssm.rssm_get_error(st) == 0
-    mism_upd = mism_codes = total = 0
-    for b in range(shape.batch):
+    rssm.rssm_lowprec_refresh(tw, inp["A"])
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
+    assert torch.equal(y, y2)                       # both read the same FP4 copy
+    assert_refresh_bits(kind, seed, st, tw, fc_before, range(Bz), f"{kind} + FP4 refresh")
+    for b in range(Bz):
         r = request_inputs(inp, b)
         req = orc.LowPrecRequest(UPD[kind][1], True, upd0[b], codes0[b], scales0[b], shape.ngroups, L, r["A"],
                                  r["D"], seed, b)
         req.flush_count.value = 1
         ys = np.stack([req.decode(r["x"][t], r["B"][t], r["C"][t], r["dt"][t]) for t in range(L)])
         assert_close(to_np(y[:, b]), ys, f"FP4-copy decode, request {b}")
-        v32 = req.refresh(want_v32=True).astype(np.float64).ravel()
-        got_upd = copy_bits(st.ckpt[b]).ravel()
-        mism_upd += int(np.count_nonzero(got_upd != req.upd.ravel()))
-        err = np.abs(copy_values(got_upd, kind) - v32)
-        bound = spacing(v32, kind) + 1e-5 * np.sqrt(np.mean(v32 ** 2))
-        assert np.all(err <= bound), float(np.max(err - bound))
-        gc = st.out_codes[b].cpu().numpy().ravel()
-        mism_codes += int(np.count_nonzero(gc != req.codes.ravel()))
-        total += gc.size
-    n_el = shape.batch * shape.nheads * shape.head_dim * shape.d_state
-    assert mism_upd <= 1e-3 * n_el, mism_upd
-    assert mism_codes <= 2e-3 * total, mism_codes
-    assert st.flush_count.cpu().tolist() == [2] * 4
+        v64 = req.refresh(want_v32=True).astype(np.float64)
+        assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of the refresh, request {b}")
+    assert st.flush_count.cpu().tolist() == [2] * Bz
 
 
 # accepted drafts per step and request (steps x batch) for K = 4 and K = 6:
@@ -162,10 +203,12 @@ def test_speculative_verify_on_split_state_matches_oracle(kind, K):
     the pending token and K drafts (K = 4 and 6: the pipelined kernel's 5-
     and 8-token bounds) reads the FP4 output copy, accept(n) advances pos,
     and the refresh after accept folds the requests whose buffer reached the
-    interval. No request reaches the interval before the last accept, so
-    every verify reads the initial FP4 copy; the outputs match the oracle
-    within the fp32 tolerance, and each refreshed request's update and FP4
-    copies match it bit for bit except at fp32 rounding straddles."""
+    interval (up to 20 buffered entries). No request reaches the interval
+    before the last accept, so every verify reads the initial FP4 copy; the
+    outputs match the oracle within the fp32 tolerance. An fp32 twin runs
+    the same calls: the refreshed requests' update and FP4 copies equal the
+    oracle's rounding of the twin's fp32 fold bit for bit (zero mismatches),
+    and the untouched request keeps its copies."""
     shape = LayerShape(4, 8, 64, 128, 2, interval=16, max_draft=K)
     n_host = SPLIT_SPEC[K]
     steps, L = n_host.shape[0], 16
@@ -173,15 +216,24 @@ def test_speculative_verify_on_split_state_matches_oracle(kind, K):
     n_acc = torch.from_numpy(n_host).cuda()
     seed = 0x5EED
     desc, st = split_state(shape, inp, kind, seed)
+    _, tw = f32_twin(shape, widened(kind, st), seed)
+    rssm.rssm_lowprec_refresh(tw, inp["A"], force=True)
+    upd_start = copy_bits(st.ckpt).copy()
+    codes_start = st.out_codes.cpu().numpy().copy()
     upd0 = copy_bits(initial_update_copy(inp["ckpt"], kind))
     codes0, scales0 = orc.fp4_quant(orc.widen(UPD[kind][1], upd0, None, upd0.shape).astype(np.float32))
     y = torch.empty((steps, shape.batch, K + 1, shape.nheads, shape.head_dim), device="cuda")
+    y2 = torch.empty_like(y)
+    fc_before = st.flush_count.cpu().tolist()
     for s in range(steps):
-        rssm.rssm_verify(st, K, inp["x"][s], inp["B"][s], inp["C"][s], inp["dt"][s], inp["A"], inp["D"], y[s])
-        rssm.rssm_accept(st, n_acc[s])
-        rssm.rssm_lowprec_refresh(st, inp["A"])
-    assert rssm.rssm_get_error(st) == 0
-    mism = total = folded = 0
+        args = (inp["x"][s], inp["B"][s], inp["C"][s], inp["dt"][s], inp["A"], inp["D"])
+        for state, out in ((st, y), (tw, y2)):
+            rssm.rssm_verify(state, K, *args, out[s])
+            rssm.rssm_accept(state, n_acc[s])
+            rssm.rssm_lowprec_refresh(state, inp["A"])
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
+    assert torch.equal(y, y2)
+    folded = []
     for b in range(shape.batch):
         r = request_inputs(inp, b)
         req = orc.LowPrecRequest(UPD[kind][1], True, upd0[b], codes0[b], scales0[b], shape.ngroups, L + K,
@@ -192,68 +244,88 @@ def test_speculative_verify_on_split_state_matches_oracle(kind, K):
             assert_close(to_np(y[s, b]), ys, f"verify on the FP4 copy, step {s}, request {b}")
             req.accept(int(n_host[s, b]))
             if req.pos >= L:
-                req.refresh()
-                folded += 1
+                v64 = req.refresh(want_v32=True).astype(np.float64)
+                assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of the refresh, request {b}")
+                folded.append(b)
         assert st.pos[b].item() == req.pos and st.flush_count[b].item() == req.flush_count.value
-        got = copy_bits(st.ckpt[b]).ravel()
-        mism += int(np.count_nonzero(got != req.upd.ravel()))
-        mism += int(np.count_nonzero(st.out_codes[b].cpu().numpy().ravel() != req.codes.ravel()))
-        total += got.size
-    assert folded == 3
-    assert mism <= 3e-3 * total, mism
+    assert len(folded) == 3
+    assert_refresh_bits(kind, seed, st, tw, fc_before, folded, f"speculative {kind} + FP4 refresh")
+    for b in set(range(shape.batch)) - set(folded):
+        assert np.array_equal(copy_bits(st.ckpt[b]), upd_start[b])
+        assert np.array_equal(st.out_codes[b].cpu().numpy(), codes_start[b])
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=["dstate64", "dstate128"])
 def test_shared_fp4_control_decode_matches_oracle(shape):
+    """The shared FP4 control (s4's ablation): decode reads the one FP4 copy
+    and the refresh re-quantises it. Outputs match the oracle; the
+    re-quantised codes and scales equal the oracle's FP4 quantisation of the
+    fp32 fold that an fp32 twin (same starting values) computes, bit for
+    bit, and that fold matches the oracle's fp64 fold."""
     L = shape.interval
+    Bz, H, P, N = shape.batch, shape.nheads, shape.head_dim, shape.d_state
     inp = make_inputs(shape, L, 32, torch.bfloat16, device="cuda")
     desc, st = fp4_control_state(shape, inp, 5)
     codes0, scales0 = orc.fp4_quant(inp["ckpt"].cpu().numpy())
-    y = torch.empty((L, 3, 4, 32), device="cuda")
+    assert np.array_equal(st.ckpt.cpu().numpy(), codes0) and np.array_equal(st.ckpt_scales.cpu().numpy(), scales0)
+    vals = orc.widen(orc.FP4, codes0, scales0, (Bz, H, P, N)).astype(np.float32)
+    _, tw = f32_twin(shape, torch.from_numpy(vals).cuda(), 5, out_copy=False)
+    y = torch.empty((L, Bz, H, P), device="cuda")
+    y2 = torch.empty_like(y)
     for t in range(L):
-        rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"], y[t])
+        args = (inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"])
+        rssm.rssm_decode_step(st, *args, y[t])
+        rssm.rssm_decode_step(tw, *args, y2[t])
     rssm.rssm_lowprec_refresh(st, inp["A"])
-    assert rssm.rssm_get_error(st) == 0
-    for b in range(3):
+    rssm.rssm_lowprec_refresh(tw, inp["A"])
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
+    assert_refresh_bits("fp4", 5, st, tw, None, range(Bz), "shared FP4 refresh")
+    for b in range(Bz):
         r = request_inputs(inp, b)
-        req = orc.LowPrecRequest(orc.FP4, False, None, codes0[b], scales0[b], 2, L, r["A"], r["D"], 5, b)
+        req = orc.LowPrecRequest(orc.FP4, False, None, codes0[b], scales0[b], shape.ngroups, L, r["A"], r["D"], 5, b)
         ys = np.stack([req.decode(r["x"][t], r["B"][t], r["C"][t], r["dt"][t]) for t in range(L)])
         assert_close(to_np(y[:, b]), ys, f"shared FP4 decode, request {b}")
-        req.refresh()
-        assert np.mean(st.ckpt[b].cpu().numpy() == req.codes) > 0.998
+        assert_close(to_np(y2[:, b]), ys, f"fp32 twin decode, request {b}")
+        v64 = req.refresh(want_v32=True).astype(np.float64)
+        assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of the shared FP4 refresh, request {b}")
 
 
+@pytest.mark.parametrize("shape", SPLIT_SHAPES, ids=["dstate128", "dstate64"])
 @pytest.mark.parametrize("kind", ["bf16", "e4m3"])
-def test_shared_copy_decode_and_refresh_match_oracle(kind):
+def test_shared_copy_decode_and_refresh_match_oracle(kind, shape):
     """One bf16 or e4m3 copy both read by decode and updated by the refresh
     (the secondary shared-precision control of s4): the outputs match the
     oracle reading the same values, and the stochastically rounded copy
-    matches it bit for bit except at fp32 rounding straddles."""
-    shape = LayerShape(4, 8, 64, 128, 2)
+    equals the oracle's rounding of the fp32 fold (from an fp32 twin with the
+    same starting values) bit for bit."""
     L = shape.interval
+    Bz, H, P = shape.batch, shape.nheads, shape.head_dim
     inp = make_inputs(shape, L, 36, torch.bfloat16, device="cuda")
     seed = 0xC0FFEE
     desc = desc_for(shape, update_dtype=UPD[kind][0], seed=seed)
     st = rssm.RssmState(desc)
     st.ckpt.copy_(initial_update_copy(inp["ckpt"], kind))
+    _, tw = f32_twin(shape, widened(kind, st), seed, out_copy=False)
     upd0 = copy_bits(initial_update_copy(inp["ckpt"], kind))
-    y = torch.empty((L, 4, 8, 64), device="cuda")
+    y = torch.empty((L, Bz, H, P), device="cuda")
+    y2 = torch.empty_like(y)
     for t in range(L):
-        rssm.rssm_decode_step(st, inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"], y[t])
+        args = (inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"])
+        rssm.rssm_decode_step(st, *args, y[t])
+        rssm.rssm_decode_step(tw, *args, y2[t])
+    fc_before = st.flush_count.cpu().tolist()
     rssm.rssm_lowprec_refresh(st, inp["A"])
-    assert rssm.rssm_get_error(st) == 0
-    mism = total = 0
-    for b in range(shape.batch):
+    rssm.rssm_lowprec_refresh(tw, inp["A"])
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
+    assert_refresh_bits(kind, seed, st, tw, fc_before, range(Bz), f"shared {kind} refresh")
+    for b in range(Bz):
         r = request_inputs(inp, b)
         req = orc.LowPrecRequest(UPD[kind][1], False, upd0[b], None, None, shape.ngroups, L, r["A"], r["D"], seed, b)
         ys = np.stack([req.decode(r["x"][t], r["B"][t], r["C"][t], r["dt"][t]) for t in range(L)])
         assert_close(to_np(y[:, b]), ys, f"shared {kind} decode, request {b}")
-        req.refresh()
-        got = copy_bits(st.ckpt[b]).ravel()
-        mism += int(np.count_nonzero(got != req.upd.ravel()))
-        total += got.size
-    assert mism <= 1e-3 * total, mism
-    assert st.flush_count.cpu().tolist() == [1] * 4 and st.pos.cpu().tolist() == [0] * 4
+        v64 = req.refresh(want_v32=True).astype(np.float64)
+        assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of the shared {kind} refresh, request {b}")
+    assert st.flush_count.cpu().tolist() == [1] * Bz and st.pos.cpu().tolist() == [0] * Bz
 
 
 def run_lowprec(desc, st, inp, steps):
