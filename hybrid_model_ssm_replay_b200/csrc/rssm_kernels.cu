@@ -23,9 +23,11 @@
 //   conventional scheme of s1/s3 (in-run comparison)            -> k_conv
 #include "rssm_device.cuh"
 #include "rssm_internal.h"
+#include "rssm_mma.cuh"
 #include "rssm.h"
 
 #include <atomic>
+#include <type_traits>
 
 namespace rssm {
 
@@ -569,6 +571,196 @@ __host__ __device__ constexpr size_t pipe_static_smem(int nt, int rf) {
     return static_cast<size_t>(pipe_groups(nt, rf)) * nt * (2 * kMaxCap + 1) * 4 + 2 * kPipeStagesMax * 8 + 1024;
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core dot products of k_replay_pipe (bf16 inputs, d_state 128; the
+// operand layouts and precision are described in rssm_mma.cuh). Lane
+// 4 g + t owns the 32 columns 32t..32t+31 of a row, in four 8-column chunks.
+// ---------------------------------------------------------------------------
+constexpr int kD128 = 128;
+
+// The four 8-column chunks (bf16) of a 128-column row that lane t owns;
+// chunk c read from position (c + t) & 3 when rot (spreads the banks of rows
+// 256 B apart), else c. Zeros for a null row.
+__device__ __forceinline__ void load_bf16_chunks(uint4 (&dst)[4], const __nv_bfloat16* row, int t, bool rot) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int pc = rot ? ((c + t) & 3) : c;
+        dst[c] = row ? *reinterpret_cast<const uint4*>(row + 32 * t + 8 * pc) : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// g[j][s] = B_s . C_j for the slots s0..s0+15 below T and the tokens j < ntok,
+// by one warp: product rows = slots, k = d_state, columns = tokens. Slot s
+// is the stage's row br + s N (s < pos) or this call's row nb + (s - pos) N.
+// s_g: [tokens][kMaxCap].
+__device__ __forceinline__ void bc_products_mma(const __nv_bfloat16* br, const __nv_bfloat16* nb,
+                                                const __nv_bfloat16* nc, int pos, int T, int ntok, int s0,
+                                                float* s_g) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    auto row_of = [&](int sl) -> const __nv_bfloat16* {
+        return sl < pos ? br + sl * kD128 : (sl < T ? nb + (sl - pos) * kD128 : nullptr);
+    };
+    uint4 cb[4], r0[4], r1[4];
+    load_bf16_chunks(cb, g < ntok ? nc + g * kD128 : nullptr, t, true);
+    load_bf16_chunks(r0, row_of(s0 + g), t, true);
+    load_bf16_chunks(r1, row_of(s0 + g + 8), t, true);
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        mma_bf16(d, r0[c].x, r1[c].x, r0[c].y, r1[c].y, cb[c].x, cb[c].y);
+        mma_bf16(d, r0[c].z, r1[c].z, r0[c].w, r1[c].w, cb[c].z, cb[c].w);
+    }
+    const int sa = s0 + g, sb = s0 + g + 8, j0 = 2 * t, j1 = 2 * t + 1;
+    if (sa < T) {
+        if (j0 < ntok) s_g[j0 * kMaxCap + sa] = d[0];
+        if (j1 < ntok) s_g[j1 * kMaxCap + sa] = d[1];
+    }
+    if (sb < T) {
+        if (j0 < ntok) s_g[j0 * kMaxCap + sb] = d[2];
+        if (j1 < ntok) s_g[j1 * kMaxCap + sb] = d[3];
+    }
+}
+
+// Whether a copy format reads its rows in rotated chunk order (rows 256 B or
+// 512 B apart) or in order (128 B / 64 B rows spread the banks already).
+__host__ __device__ constexpr bool hc_rotated(int rf) { return rf == kF32 || rf == kBF16; }
+
+// B operand of h . C_j for lane (g, t): token j = g, from the lane's chunks of
+// C_g (bf16, cb); bfrag[4 c + u] stands for columns 2u, 2u + 1 of chunk c.
+// F32 and BF16: the bf16 words as they are (the tf32 steps take each half as
+// an fp32 value); E4M3 / FP4: f16 pairs. For the k16 steps, bfrag[2 m],
+// bfrag[2 m + 1] are b0, b1 of step m.
+template <int RF>
+__device__ __forceinline__ void hc_bfrag(const uint4 (&cb)[4], uint32_t (&bfrag)[16]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const uint32_t w[4] = {cb[c].x, cb[c].y, cb[c].z, cb[c].w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) bfrag[4 * c + u] = (RF == kF32 || RF == kBF16) ? w[u] : bf16x2_to_f16x2(w[u]);
+    }
+}
+
+// d += h . C for the rows R0 + g (d0, d1) and R0 + g + 8 (d2, d3) of a stage
+// tile (format RF, d_state 128), columns j = 2t, 2t+1 of the product: the
+// tokens (bfrag from hc_bfrag) or, for the FP4 decode, the scale blocks
+// (bfrag zero except in column g = block). SCALE_A: multiply FP4 codes by
+// their block scale before the product (verify); else the product is of the
+// bare codes (the decode applies the scales per block afterwards). Rows at or
+// past P read as zero.
+template <int RF, bool SCALE_A>
+__device__ __forceinline__ void hc_mma(const unsigned char* tile, const unsigned char* sc, int R0, int P,
+                                       const uint32_t (&bfrag)[16], float (&d)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int ra = R0 + g, rb = R0 + g + 8;
+    const bool va = ra < P, vb = rb < P;
+    if constexpr (RF == kF32) {
+        const float* pa = reinterpret_cast<const float*>(tile) + ra * kD128 + 32 * t;
+        const float* pb = reinterpret_cast<const float*>(tile) + rb * kD128 + 32 * t;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int pc = 8 * ((c + t) & 3);
+            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 a0 = va ? *reinterpret_cast<const float4*>(pa + pc) : z;
+            const float4 a1 = va ? *reinterpret_cast<const float4*>(pa + pc + 4) : z;
+            const float4 b0 = vb ? *reinterpret_cast<const float4*>(pb + pc) : z;
+            const float4 b1 = vb ? *reinterpret_cast<const float4*>(pb + pc + 4) : z;
+            const float ra8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float rb8[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                uint32_t h0, l0, h1, l1, h2, l2, h3, l3;
+                tf32_split(ra8[2 * u], h0, l0);      // row g, k lo
+                tf32_split(rb8[2 * u], h1, l1);      // row g + 8, k lo
+                tf32_split(ra8[2 * u + 1], h2, l2);  // row g, k hi
+                tf32_split(rb8[2 * u + 1], h3, l3);  // row g + 8, k hi
+                // step 4c + u: k lo = column 2u of the chunk, k hi = column 2u + 1
+                const uint32_t q0 = bf16lo_bits(bfrag[4 * c + u]), q1 = bf16hi_bits(bfrag[4 * c + u]);
+                mma_tf32(d, h0, h1, h2, h3, q0, q1);
+                mma_tf32(d, l0, l1, l2, l3, q0, q1);
+            }
+        }
+    } else if constexpr (RF == kBF16) {
+        uint4 u0[4], u1[4];
+        const __nv_bfloat16* rows = reinterpret_cast<const __nv_bfloat16*>(tile);
+        load_bf16_chunks(u0, va ? rows + ra * kD128 : nullptr, t, true);
+        load_bf16_chunks(u1, vb ? rows + rb * kD128 : nullptr, t, true);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            mma_bf16(d, u0[c].x, u1[c].x, u0[c].y, u1[c].y, bfrag[4 * c], bfrag[4 * c + 1]);
+            mma_bf16(d, u0[c].z, u1[c].z, u0[c].w, u1[c].w, bfrag[4 * c + 2], bfrag[4 * c + 3]);
+        }
+    } else if constexpr (RF == kE4M3) {
+        // 32 codes of a row per lane: two 16-byte words, chunk c = word half c & 1 of e[c >> 1]
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 ea0 = va ? *reinterpret_cast<const uint4*>(tile + ra * kD128 + 32 * t) : z;
+        const uint4 ea1 = va ? *reinterpret_cast<const uint4*>(tile + ra * kD128 + 32 * t + 16) : z;
+        const uint4 eb0 = vb ? *reinterpret_cast<const uint4*>(tile + rb * kD128 + 32 * t) : z;
+        const uint4 eb1 = vb ? *reinterpret_cast<const uint4*>(tile + rb * kD128 + 32 * t + 16) : z;
+        const uint32_t wa[8] = {ea0.x, ea0.y, ea0.z, ea0.w, ea1.x, ea1.y, ea1.z, ea1.w};
+        const uint32_t wb[8] = {eb0.x, eb0.y, eb0.z, eb0.w, eb1.x, eb1.y, eb1.z, eb1.w};
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {  // step m: codes 4m..4m+3 of the lane's 32
+            uint32_t a0, a2, a1, a3;
+            e4m3x4_h2(wa[m], a0, a2);
+            e4m3x4_h2(wb[m], a1, a3);
+            mma_f16(d, a0, a1, a2, a3, bfrag[2 * m], bfrag[2 * m + 1]);
+        }
+    } else {
+        // FP4: 32 codes of a row per lane in one 16-byte word; scales of the
+        // lane's two blocks (2t, 2t + 1) in one 16-bit word
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 qa = va ? *reinterpret_cast<const uint4*>(tile + ra * (kD128 / 2) + 16 * t) : z;
+        const uint4 qb = vb ? *reinterpret_cast<const uint4*>(tile + rb * (kD128 / 2) + 16 * t) : z;
+        const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
+        uint32_t sa = 0u, sb = 0u;
+        if constexpr (SCALE_A) {
+            sa = va ? e4m3x2_h2(*reinterpret_cast<const uint16_t*>(sc + ra * (kD128 / 16) + 2 * t)) : 0u;
+            sb = vb ? e4m3x2_h2(*reinterpret_cast<const uint16_t*>(sc + rb * (kD128 / 16) + 2 * t)) : 0u;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {  // chunk c: codes 8c..8c+7 (block 2t + c / 2)
+            uint32_t ha[4], hb[4];
+            e2m1x8_h2(wa[c], ha);
+            e2m1x8_h2(wb[c], hb);
+            if constexpr (SCALE_A) {
+                const uint32_t s2a = (c < 2) ? h2_dup_lo(sa) : h2_dup_hi(sa);
+                const uint32_t s2b = (c < 2) ? h2_dup_lo(sb) : h2_dup_hi(sb);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    ha[k] = hmul2_u32(ha[k], s2a);
+                    hb[k] = hmul2_u32(hb[k], s2b);
+                }
+            }
+            mma_f16(d, ha[0], hb[0], ha[1], hb[1], bfrag[4 * c], bfrag[4 * c + 1]);
+            mma_f16(d, ha[2], hb[2], ha[3], hb[3], bfrag[4 * c + 2], bfrag[4 * c + 3]);
+        }
+    }
+}
+
+// Replay terms of the verify: d += sum_s coef[j][s] x_s[row] for the rows
+// R0 + g, R0 + g + 8 and the tokens j = 2t, 2t+1, over the slots below T
+// (tf32 k8 steps of 8 slots; x exact, coef split hi + lo in cfrag).
+// x_s: the stage's xr + s P (s < pos) or this call's nx + (s - pos) P.
+__device__ __forceinline__ void replay_mma(const __nv_bfloat16* xr, const __nv_bfloat16* nx, int pos, int T, int P,
+                                           int R0, const uint32_t (&cfrag)[16], float (&d)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int ra = R0 + g, rb = R0 + g + 8;
+    auto xbits = [&](int sl, int r) -> uint32_t {
+        if (sl >= T || r >= P) return 0u;
+        const __nv_bfloat16* row = sl < pos ? xr + sl * P : nx + (sl - pos) * P;
+        return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(row + r)) << 16;
+    };
+#pragma unroll
+    for (int q = 0; q < kMaxCap / 8; ++q) {
+        if (8 * q < T) {
+            const int s_lo = 8 * q + t, s_hi = 8 * q + t + 4;
+            const uint32_t a0 = xbits(s_lo, ra), a1 = xbits(s_lo, rb), a2 = xbits(s_hi, ra), a3 = xbits(s_hi, rb);
+            mma_tf32(d, a0, a1, a2, a3, cfrag[4 * q], cfrag[4 * q + 1]);
+            mma_tf32(d, a0, a1, a2, a3, cfrag[4 * q + 2], cfrag[4 * q + 3]);
+        }
+    }
+}
+
 // Stage meta (int words): the position and the index k of the tile the
 // stage holds (-1 before its first use).
 constexpr int kMetaPos = 0, kMetaTile = 1;
@@ -577,6 +769,9 @@ template <typename TIn, int RF, int NT, int FUSED>
 __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const ReplayArgs a, const PipeLayout lay) {
     constexpr int CG = pipe_groups(NT, RF), CW = pipe_cwarps(NT, RF), CT = CW * 32;
     static_assert(!FUSED || (RF == kF32 && NT == 1), "the fused fold is for fp32 decode");
+    // bf16 inputs: verify (every copy format) and the FP4 decode form their
+    // dot products on the tensor cores
+    constexpr bool kMma = std::is_same<TIn, __nv_bfloat16>::value && (NT > 1 || RF == kFP4);
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full_bar[kPipeStagesMax];
     __shared__ __align__(8) uint64_t empty_bar[kPipeStagesMax];
@@ -812,7 +1007,14 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
             // a tile that folds (fused flush) needs neither the B.C products nor
             // the replay rows: its output comes from the folded state
             const bool fold_now = FUSED && T == a.s.L;
-            for (int s0 = cw * 8; !fold_now && s0 < T; s0 += CW * 8) {
+            if constexpr (kMma) {
+                // B_s . C_j on the tensor cores, 16 slots per warp
+                for (int s0 = 16 * cw; s0 < T; s0 += 16 * CW)
+                    bc_products_mma(reinterpret_cast<const __nv_bfloat16*>(br),
+                                    reinterpret_cast<const __nv_bfloat16*>(nb),
+                                    reinterpret_cast<const __nv_bfloat16*>(nc), pos, T, ntok, s0, &s_g[gi][0][0]);
+            }
+            for (int s0 = cw * 8; !kMma && !fold_now && s0 < T; s0 += CW * 8) {
                 // B_s . C_j for slots s0..s0+7, reduced together; the 8 B rows
                 // are read once for all tokens
                 float4 bv[8];
@@ -912,7 +1114,98 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                     part[7] = fmaf(coef, xb.w, part[7]);
                 }
             };
-            if constexpr (RF == kFP4 && NT == 1) {
+            if constexpr (kMma && NT == 1) {
+                // FP4 decode on the tensor cores: the product's 8 columns are the
+                // 8 scale blocks of a row (B holds C in the column of the block
+                // its k falls in), so lane (g, t) receives the bare code . C sums
+                // of blocks 2t, 2t + 1 of rows g and g + 8 and scales them; its
+                // replay terms (slots t, t + 4, ...) join before the row's four
+                // lanes add up.
+                const int g = lane >> 2, t = lane & 3;
+                uint4 cb[4];
+                load_bf16_chunks(cb, reinterpret_cast<const __nv_bfloat16*>(nc), t, false);
+                uint32_t bf[16];
+                hc_bfrag<kFP4>(cb, bf);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const bool mine = g == 2 * t + (c >> 1);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) bf[4 * c + u] = mine ? bf[4 * c + u] : 0u;
+                }
+                const float dec = s_decay[gi][0];
+                float cf[kMaxCap / 4];
+#pragma unroll
+                for (int m = 0; m < kMaxCap / 4; ++m) {
+                    const int sl = t + 4 * m;
+                    cf[m] = (sl <= pos) ? s_w[gi][0][sl] * s_g[gi][0][sl] : 0.f;
+                }
+                for (int R0 = 16 * cw; R0 < P; R0 += 16 * CW) {
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    hc_mma<kFP4, false>(tile, sc, R0, P, bf, d);
+                    const int ra = R0 + g, rb = ra + 8;
+                    const bool va = ra < P, vb = rb < P;
+                    const float2 sa = va ? h2_f2(e4m3x2_h2(*reinterpret_cast<const uint16_t*>(sc + ra * (N >> 4) + 2 * t)))
+                                         : make_float2(0.f, 0.f);
+                    const float2 sb = vb ? h2_f2(e4m3x2_h2(*reinterpret_cast<const uint16_t*>(sc + rb * (N >> 4) + 2 * t)))
+                                         : make_float2(0.f, 0.f);
+                    float pa = dec * fmaf(sa.x, d[0], sa.y * d[1]);
+                    float pb = dec * fmaf(sb.x, d[2], sb.y * d[3]);
+#pragma unroll
+                    for (int m = 0; m < kMaxCap / 4; ++m) {
+                        const int sl = t + 4 * m;
+                        if (sl <= pos) {
+                            const TIn* xrow = sl < pos ? xr + sl * P : nx;
+                            if (va) pa = fmaf(cf[m], to_f32(xrow[ra]), pa);
+                            if (vb) pb = fmaf(cf[m], to_f32(xrow[rb]), pb);
+                        }
+                    }
+                    pa += __shfl_xor_sync(0xffffffffu, pa, 1);
+                    pb += __shfl_xor_sync(0xffffffffu, pb, 1);
+                    pa += __shfl_xor_sync(0xffffffffu, pa, 2);
+                    pb += __shfl_xor_sync(0xffffffffu, pb, 2);
+                    if (t == 0) {
+                        if (va) yout[ra] = fmaf(Dh, to_f32(nx[ra]), pa);
+                        if (vb) yout[rb] = fmaf(Dh, to_f32(nx[rb]), pb);
+                    }
+                }
+            } else if constexpr (kMma) {
+                // verify on the tensor cores: lane (g, t) receives h . C_j and the
+                // replay sums of rows g, g + 8 for the tokens j = 2t, 2t + 1
+                const int g = lane >> 2, t = lane & 3;
+                uint4 cb[4];
+                load_bf16_chunks(cb, g < ntok ? reinterpret_cast<const __nv_bfloat16*>(nc) + g * kD128 : nullptr, t,
+                                 hc_rotated(RF));
+                uint32_t bf[16];
+                hc_bfrag<RF>(cb, bf);
+                // coef of token g for the slots 8q + t (b0) and 8q + t + 4 (b1), hi + lo
+                uint32_t cfr[16];
+#pragma unroll
+                for (int q = 0; q < kMaxCap / 8; ++q) {
+                    const int s0 = 8 * q + t, s1 = s0 + 4;
+                    const float c0 = (g < ntok && s0 <= pos + g) ? s_w[gi][g][s0] * s_g[gi][g][s0] : 0.f;
+                    const float c1 = (g < ntok && s1 <= pos + g) ? s_w[gi][g][s1] * s_g[gi][g][s1] : 0.f;
+                    tf32_split(c0, cfr[4 * q], cfr[4 * q + 2]);
+                    tf32_split(c1, cfr[4 * q + 1], cfr[4 * q + 3]);
+                }
+                const int j0 = 2 * t, j1 = 2 * t + 1;
+                const float dec0 = j0 < ntok ? s_decay[gi][j0] : 0.f, dec1 = j1 < ntok ? s_decay[gi][j1] : 0.f;
+                const __nv_bfloat16* xr16 = reinterpret_cast<const __nv_bfloat16*>(xr);
+                const __nv_bfloat16* nx16 = reinterpret_cast<const __nv_bfloat16*>(nx);
+                for (int R0 = 16 * cw; R0 < P; R0 += 16 * CW) {
+                    float dh[4] = {0.f, 0.f, 0.f, 0.f}, dx[4] = {0.f, 0.f, 0.f, 0.f};
+                    hc_mma<RF, true>(tile, sc, R0, P, bf, dh);
+                    replay_mma(xr16, nx16, pos, T, P, R0, cfr, dx);
+                    const int ra = R0 + g, rb = ra + 8;
+                    if (ra < P) {
+                        if (j0 < ntok) yout[j0 * HP + ra] = fmaf(Dh, to_f32(nx[j0 * P + ra]), fmaf(dec0, dh[0], dx[0]));
+                        if (j1 < ntok) yout[j1 * HP + ra] = fmaf(Dh, to_f32(nx[j1 * P + ra]), fmaf(dec1, dh[1], dx[1]));
+                    }
+                    if (rb < P) {
+                        if (j0 < ntok) yout[j0 * HP + rb] = fmaf(Dh, to_f32(nx[j0 * P + rb]), fmaf(dec0, dh[2], dx[2]));
+                        if (j1 < ntok) yout[j1 * HP + rb] = fmaf(Dh, to_f32(nx[j1 * P + rb]), fmaf(dec1, dh[3], dx[3]));
+                    }
+                }
+            } else if constexpr (RF == kFP4 && NT == 1) {
                 // FP4 decode: lane l takes row r0 + l/4 and columns 32 (l % 4) ..
                 // +31 of an 8-row block: one 16-byte load of codes and one of
                 // two scales per row, codes.C per 16 columns times the block

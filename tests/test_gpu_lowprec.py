@@ -137,11 +137,13 @@ def test_refresh_at_empty_buffer_builds_fp4_copy_bit_exact(kind, shape):
     assert rssm.rssm_get_error(st) == 0
 
 
-# the pipelined fold (d_state 128) and the one-CTA-per-tile fold (d_state 64)
-SPLIT_SHAPES = [LayerShape(4, 8, 64, 128, 2), LayerShape(3, 4, 32, 64, 2)]
+# the pipelined kernels (d_state 128; head_dim 40 leaves a half-empty last
+# 16-row group) and the one-CTA-per-tile kernels (d_state 64)
+SPLIT_SHAPES = [LayerShape(4, 8, 64, 128, 2), LayerShape(3, 4, 40, 128, 2), LayerShape(3, 4, 32, 64, 2)]
+SPLIT_IDS = ["dstate128", "headdim40", "dstate64"]
 
 
-@pytest.mark.parametrize("shape", SPLIT_SHAPES, ids=["dstate128", "dstate64"])
+@pytest.mark.parametrize("shape", SPLIT_SHAPES, ids=SPLIT_IDS)
 @pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32], ids=["bf16in", "f32in"])
 @pytest.mark.parametrize("kind", ["bf16", "e4m3"])
 def test_fp4_decode_and_refresh_match_oracle(kind, in_dtype, shape):
@@ -290,7 +292,7 @@ def test_shared_fp4_control_decode_matches_oracle(shape):
         assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of the shared FP4 refresh, request {b}")
 
 
-@pytest.mark.parametrize("shape", SPLIT_SHAPES, ids=["dstate128", "dstate64"])
+@pytest.mark.parametrize("shape", SPLIT_SHAPES, ids=SPLIT_IDS)
 @pytest.mark.parametrize("kind", ["bf16", "e4m3"])
 def test_shared_copy_decode_and_refresh_match_oracle(kind, shape):
     """One bf16 or e4m3 copy both read by decode and updated by the refresh
@@ -326,6 +328,52 @@ def test_shared_copy_decode_and_refresh_match_oracle(kind, shape):
         v64 = req.refresh(want_v32=True).astype(np.float64)
         assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of the shared {kind} refresh, request {b}")
     assert st.flush_count.cpu().tolist() == [1] * Bz and st.pos.cpu().tolist() == [0] * Bz
+
+
+@pytest.mark.parametrize("K", [4, 6])
+@pytest.mark.parametrize("kind", ["bf16", "e4m3"])
+def test_speculative_verify_on_shared_copy_matches_oracle(kind, K):
+    """Verify (s3) reading a bf16 or e4m3 copy that is also the update copy
+    (the secondary shared-precision control of s4): the K+1 outputs of every
+    step match the oracle reading the same copy values, and the refresh
+    after accept equals the oracle's rounding of the fp32 twin's fold."""
+    shape = LayerShape(4, 8, 64, 128, 2, interval=16, max_draft=K)
+    n_host = SPLIT_SPEC[K]
+    steps, L = n_host.shape[0], 16
+    inp = make_inputs(shape, steps, 35, torch.bfloat16, device="cuda", ntok=K + 1)
+    n_acc = torch.from_numpy(n_host).cuda()
+    seed = 0xACE
+    desc = desc_for(shape, update_dtype=UPD[kind][0], seed=seed)
+    st = rssm.RssmState(desc)
+    st.ckpt.copy_(initial_update_copy(inp["ckpt"], kind))
+    _, tw = f32_twin(shape, widened(kind, st), seed, out_copy=False)
+    upd0 = copy_bits(initial_update_copy(inp["ckpt"], kind))
+    y = torch.empty((steps, shape.batch, K + 1, shape.nheads, shape.head_dim), device="cuda")
+    y2 = torch.empty_like(y)
+    fc_before = st.flush_count.cpu().tolist()
+    for s in range(steps):
+        args = (inp["x"][s], inp["B"][s], inp["C"][s], inp["dt"][s], inp["A"], inp["D"])
+        for state, out in ((st, y), (tw, y2)):
+            rssm.rssm_verify(state, K, *args, out[s])
+            rssm.rssm_accept(state, n_acc[s])
+            rssm.rssm_lowprec_refresh(state, inp["A"])
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
+    folded = []
+    for b in range(shape.batch):
+        r = request_inputs(inp, b)
+        req = orc.LowPrecRequest(UPD[kind][1], False, upd0[b], None, None, shape.ngroups, L + K, r["A"], r["D"],
+                                 seed, b)
+        for s in range(steps):
+            ys = req.verify(r["x"][s], r["B"][s], r["C"][s], r["dt"][s])
+            assert_close(to_np(y[s, b]), ys, f"verify on the shared {kind} copy, step {s}, request {b}")
+            assert_close(to_np(y2[s, b]), ys, f"verify on the fp32 twin, step {s}, request {b}")
+            req.accept(int(n_host[s, b]))
+            if req.pos >= L:
+                req.refresh()
+                folded.append(b)
+        assert st.pos[b].item() == req.pos
+    assert len(folded) == 3
+    assert_refresh_bits(kind, seed, st, tw, fc_before, folded, f"speculative shared {kind} refresh")
 
 
 def run_lowprec(desc, st, inp, steps):

@@ -131,13 +131,16 @@ def test_spec_b512_k4_sampled():
 
 @pytest.mark.parametrize("shape", [LayerShape(5, 4, 32, 128, 2, interval=16, max_draft=1),
                                    LayerShape(5, 4, 32, 128, 2, interval=16, max_draft=6),
-                                   LayerShape(3, 4, 32, 128, 2, interval=27, max_draft=5)],
-                         ids=["k1", "k6", "cap32"])
+                                   LayerShape(3, 4, 32, 128, 2, interval=27, max_draft=5),
+                                   LayerShape(4, 6, 40, 128, 3, interval=16, max_draft=4)],
+                         ids=["k1", "k6", "cap32", "headdim40"])
 def test_spec_pipelined_drafts_and_capacity(shape):
     """The pipelined verify at other draft counts (2 and 7 tokens per call,
-    under the kernel's 5- and 8-token bounds) and with the largest buffer
-    (interval 27 + 5 drafts = 32 slots: four 8-slot B.C blocks), every
-    request against the oracle, the conventional verify beside it."""
+    under the kernel's 5- and 8-token bounds), with the largest buffer
+    (interval 27 + 5 drafts = 32 slots: two 16-slot B.C products, four
+    8-slot replay steps), and with head_dim 40 (a last 16-row group that is
+    half empty), every request against the oracle, the conventional verify
+    beside it."""
     check_spec_case(shape, 40, 13, list(range(shape.batch)))
 
 
