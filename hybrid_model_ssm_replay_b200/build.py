@@ -15,8 +15,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "librssm.so")
-SOURCES = ["rssm_kernels.cu", "rssm_api.cu"]
-HEADERS = ["rssm_device.cuh", "rssm_internal.h"]
+SOURCES = ["rssm_kernels.cu", "rssm_api.cu", "rssm_stage.cu"]
+HEADERS = ["rssm_device.cuh", "rssm_internal.h", "rssm_mma.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -35,7 +35,7 @@ def nvcc() -> str:
 
 def _inputs():
     files = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
-    files += [os.path.join(INCLUDE, "rssm.h"), os.path.abspath(__file__)]
+    files += [os.path.join(INCLUDE, "rssm.h"), os.path.join(INCLUDE, "rssm_stage.h"), os.path.abspath(__file__)]
     return files
 
 

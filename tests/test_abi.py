@@ -19,14 +19,19 @@ def L():
 
 
 def declared_functions():
-    text = open(os.path.join(ROOT, "include", "rssm.h")).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(rssm_[a-z_0-9]+)\s*\(", text)))
+    """Every function declared in include/*.h."""
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(rssm_[a-z_0-9]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_exports_every_declared_symbol(L):
     names = declared_functions()
-    assert len(names) >= 14
+    assert len(names) >= 18 and "rssm_stage_conv" in names and "rssm_stage_gate_norm" in names
     for n in names:
         assert hasattr(L, n), n
     assert L.rssm_abi_version() == 2
@@ -139,3 +144,18 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         rssm._ptr(torch.zeros(4), torch.float32, "x")
+
+
+def test_stage_calls_reject_bad_arguments_on_the_host(L):
+    """The stage's element-wise calls check their arguments before any CUDA
+    call: null pointers, an fp32 input description, a bad eps."""
+    from hybrid_model_ssm_replay_b200 import stage  # noqa: F401  (sets the signatures)
+    stage._lib()
+    d = cfg()
+    p = ct.c_void_p(0x1000)
+    assert L.rssm_stage_conv(ct.byref(d), None, p, p, p, p, p, p, p, p, None) == 1
+    assert L.rssm_stage_gate_norm(ct.byref(d), p, p, p, ct.c_float(0.0), p, None) == 1
+    f = cfg(in_dtype=rssm.RSSM_F32)
+    assert L.rssm_stage_conv(ct.byref(f), p, p, p, p, p, p, p, p, p, None) == 3
+    assert L.rssm_stage_gate_norm(ct.byref(f), p, p, p, ct.c_float(1e-5), p, None) == 3
+    assert L.rssm_stage_conv(None, p, p, p, p, p, p, p, p, p, None) == 1
