@@ -944,8 +944,11 @@ def split_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
 
 def prefill_leg(rssm, torch, wl, dev, barrier, max_over_ranks, world, T0=512, reps=5):
     """Prefill of a 512-token prompt into the fp32 checkpoint of the small
-    layer (rssm_prefill): prompt tokens/s and the fold's FMA rate against the
-    fp32 CUDA-core peak (148 SMs x 128 lanes x 2 flop x SM clock)."""
+    layer (rssm_prefill): prompt tokens/s. At these shapes (bf16, d_state 128,
+    head_dim 64) the fold is one tensor-core contraction per (request, head),
+    X_w^T B with K = T0, and the kernel is bound by HBM: algorithmic bytes per
+    request = the prompt's x (H P T0 2) + B (G N T0 2) + dt (4 H T0) + one
+    read and one write of the fp32 state (2 x 4 H P N)."""
     from hybrid_model_ssm_replay_b200.inputs import make_inputs
     shape = wl["shape"]
     inp = make_inputs(shape, T0, wl["seed"] + 11, wl["in_dtype"], device=dev)
@@ -966,12 +969,18 @@ def prefill_leg(rssm, torch, wl, dev, barrier, max_over_ranks, world, T0=512, re
     ms = max_over_ranks(a.elapsed_time(e)) / reps
     if rssm.rssm_get_error(st) != 0:
         raise RuntimeError("device error in the prefill leg")
-    flops = 2.0 * shape.nheads * shape.head_dim * shape.d_state * T0 * shape.batch
-    peak_tf = 148 * 128 * 2 * 1.965e9 / 1e12
+    H, P, N, G = shape.nheads, shape.head_dim, shape.d_state, shape.ngroups
+    req_bytes = H * P * T0 * 2 + G * N * T0 * 2 + 4 * H * T0 + 2 * 4 * H * P * N
+    gbs = req_bytes * shape.batch / (ms / 1e3) / 1e9
+    peak, peak_src = measured_peaks()
+    flops = 2.0 * H * P * N * T0 * shape.batch
     return {"workload": f"small_b256 shapes, prompt of {T0} tokens per request", "prompt_tokens_per_s":
-            world * shape.batch * T0 / (ms / 1e3), "ms_per_prefill": ms, "fold_tflops": flops / (ms / 1e3) / 1e12,
-            "bound": "alu", "peak_tflops": peak_tf, "frac": flops / (ms / 1e3) / 1e12 / peak_tf,
-            "peak_source": "148 SMs x 128 fp32 lanes x 2 flop x 1.965 GHz (nominal max SM clock)"}
+            world * shape.batch * T0 / (ms / 1e3), "ms_per_prefill": ms,
+            "kernel": "k_prefill_mma (mma.sync bf16, x_w split hi + lo)",
+            "bound": "hbm", "algorithmic_bytes_per_request": req_bytes, "achieved_gbs": gbs, "peak": peak,
+            "peak_source": peak_src, "frac": gbs / peak,
+            "contraction_tflops": flops / (ms / 1e3) / 1e12,
+            "note": "fold flops = 2 H P N T0 per request; the hi + lo split issues twice that on the tensor cores"}
 
 
 # ---------------------------------------------------- the CPU oracle arm
@@ -1099,7 +1108,7 @@ def run_profile(sections):
       split_e4m3   the same with an e4m3 update copy
       shared_fp4   the shared FP4 control: refresh(force) of an fp32 + FP4
                    state to build the copy, 16 decodes, refresh
-      prefill      rssm_prefill of a 64-token prompt"""
+      prefill      rssm_prefill of a 512-token prompt"""
     import torch
 
     from hybrid_model_ssm_replay_b200 import rssm
@@ -1184,7 +1193,7 @@ def run_profile(sections):
             rssm.rssm_lowprec_refresh(st, inp["A"])
             check(st)
         elif sec == "prefill":
-            T0 = 64
+            T0 = 512
             pi = make_inputs(sh, T0, wl["seed"] + 11, wl["in_dtype"], device="cuda")
             st = rssm.RssmState(mk())
             st.ckpt.copy_(pi["ckpt"])

@@ -21,9 +21,10 @@ namespace rssm {
 constexpr int kThreads = 256;               // threads per CTA of the one-CTA-per-tile kernels
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxCap = 32;                 // buffer slots per request (interval + drafts)
+constexpr int kMaxHeadDim = 256;           // largest head_dim (rssm_check_desc)
 constexpr int kMaxTok = 8;                  // tokens per verify call (K + 1)
 constexpr int kMidTok = 5;                  // verify kernels specialised for K <= 4
-constexpr int kPipeStagesMax = 16;          // shared-memory stages of the pipelined kernels
+constexpr int kPipeStagesMax = 24;          // shared-memory stages of the pipelined kernels
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bound of every wait (mbarrier, stage tag)
 
 // ------------------------------------------------------------------ errors
@@ -114,6 +115,48 @@ __device__ __forceinline__ float dot4(float4 a, float4 b) {
     return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
 }
 
+// d = a * b + c on two fp32 lanes at once: the packed fp32 FMA of sm_100
+// (each lane an IEEE fma, rounded to nearest, exactly as fmaf).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+// The rank-T update of an 8-row x 4-column register block with packed FMAs:
+// acc2[p][c] holds rows 2p, 2p+1 of column c; per slot, w2[p] = the slot's
+// weighted x of rows 2p, 2p+1 and b the slot's 4 B values. Each element sees
+// acc = fma(w, b, acc) in slot order, as with scalar FMAs.
+__device__ __forceinline__ void rank1_8x4(float2 (&acc2)[4][4], const float2 (&w2)[4], float4 b) {
+    const float2 bd[4] = {make_float2(b.x, b.x), make_float2(b.y, b.y), make_float2(b.z, b.z), make_float2(b.w, b.w)};
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc2[p][c] = fma2(w2[p], bd[c], acc2[p][c]);
+}
+
+__device__ __forceinline__ float4 acc2_row(const float2 (&acc2)[4][4], int k) {
+    const int p = k >> 1;
+    return (k & 1) ? make_float4(acc2[p][0].y, acc2[p][1].y, acc2[p][2].y, acc2[p][3].y)
+                   : make_float4(acc2[p][0].x, acc2[p][1].x, acc2[p][2].x, acc2[p][3].x);
+}
+
+__device__ __forceinline__ void acc2_set_row(float2 (&acc2)[4][4], int k, float4 v) {
+    const int p = k >> 1;
+    if (k & 1) {
+        acc2[p][0].y = v.x; acc2[p][1].y = v.y; acc2[p][2].y = v.z; acc2[p][3].y = v.w;
+    } else {
+        acc2[p][0].x = v.x; acc2[p][1].x = v.y; acc2[p][2].x = v.z; acc2[p][3].x = v.w;
+    }
+}
+
 // Sum over aligned groups of `width` lanes (width a power of two <= 32).
 __device__ __forceinline__ float group_sum(float v, int width) {
 #pragma unroll
@@ -125,18 +168,39 @@ __device__ __forceinline__ float group_sum(float v, int width) {
 // ------------------------------------------------------------------ Philox
 
 // Philox4x32-10: ten rounds; round i uses key + i * (0x9E3779B9, 0xBB67AE85).
-__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
+// The round keys depend only on the seed, so a kernel forms them once
+// (PhiloxKeys) and every draw spends per round two 32 x 32 -> 64-bit
+// multiplies (high and low halves at once) and two three-input XORs.
+struct PhiloxKeys {
+    uint32_t x[10], y[10];
+};
+
+__device__ __forceinline__ PhiloxKeys philox_keys(uint64_t seed) {
+    PhiloxKeys K;
+    uint32_t kx = static_cast<uint32_t>(seed), ky = static_cast<uint32_t>(seed >> 32);
 #pragma unroll
     for (int i = 0; i < 10; ++i) {
-        if (i) {
-            k.x += 0x9E3779B9u;
-            k.y += 0xBB67AE85u;
-        }
-        const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
-        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
-        c = make_uint4(hi1 ^ c.y ^ k.x, lo1, hi0 ^ c.w ^ k.y, lo0);
+        K.x[i] = kx;
+        K.y[i] = ky;
+        kx += 0x9E3779B9u;
+        ky += 0xBB67AE85u;
+    }
+    return K;
+}
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys& K) {
+#pragma unroll
+    for (int i = 0; i < 10; ++i) {
+        const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;
+        const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+        c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ c.y ^ K.x[i], static_cast<uint32_t>(p1),
+                       static_cast<uint32_t>(p0 >> 32) ^ c.w ^ K.y[i], static_cast<uint32_t>(p0));
     }
     return c;
+}
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
+    return philox4x32_10(c, philox_keys(static_cast<uint64_t>(k.x) | (static_cast<uint64_t>(k.y) << 32)));
 }
 
 // ------------------------------------------------------ stochastic rounding
@@ -166,7 +230,7 @@ __device__ __forceinline__ uint32_t sr_e4m3(float v, uint32_t r) {
         F = (a & 0xFFFFFu) << 12;
     } else {
         // below 2^-6: t = |v| 2^9 < 8 is exact, code = floor(t), and the
-        // fraction scaled by 2^32 is exact too
+        // fraction scaled by 2^32 is exact too (at most 24 significant bits)
         const float t = __uint_as_float(a) * 512.0f;
         const float m = truncf(t);
         code = static_cast<uint32_t>(m);

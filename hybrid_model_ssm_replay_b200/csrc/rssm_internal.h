@@ -66,7 +66,7 @@ inline FastDiv make_fastdiv(uint32_t d) {
 // Shared-memory stage of the pipelined replay kernel: a mirror of the
 // record prefix (same offsets as RecLayout, x rows up to cap), the buffered
 // B rows [cap][N] at `brows` and the position and tile index at `meta`;
-// `stages` stages. After them, per consumer group, three buffers of
+// `stages` stages. After them, per consumer group, two buffers of
 // `newrows` bytes for this call's x, B and C rows ([ntok][P], [ntok][N],
 // [ntok][N] at 0, nb_off, nc_off) and its dt [8], A_h, D_h (at nd_off).
 struct PipeLayout {
@@ -75,6 +75,7 @@ struct PipeLayout {
     int stages;
     size_t budget;  // dynamic shared memory the layout may use
     FastDiv divH, divHpg;  // tile -> (request, head), head -> group
+    FastDiv divTok;        // prefetch item -> token (16-byte chunks per token)
 };
 
 // Fold of the buffer into the update copy (flush / refresh; s1, s4).

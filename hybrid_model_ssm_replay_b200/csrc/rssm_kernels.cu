@@ -103,7 +103,7 @@ __device__ __forceinline__ void fold_tile(const float* s32, const float* s_xw, i
     const int rows_per_pass = kWarps * rpw * kRB;
     for (int base = 0; base < P; base += rows_per_pass) {
         const int rb = base + (warp * rpw + rsub) * kRB;
-        float4 acc[kRB];
+        float2 acc2[4][4];  // rows paired for the packed FMAs
 #pragma unroll
         for (int k = 0; k < kRB; ++k) {
             const int r = rb + k;
@@ -115,7 +115,7 @@ __device__ __forceinline__ void fold_tile(const float* s32, const float* s_xw, i
                 v.z *= alpha;
                 v.w *= alpha;
             }
-            acc[k] = v;
+            acc2_set_row(acc2, k, v);
         }
         if (rb < P) {
 #pragma unroll 2
@@ -123,18 +123,13 @@ __device__ __forceinline__ void fold_tile(const float* s32, const float* s_xw, i
                 const float4 bv = brow(s, col4);
                 const float4* xw4 = reinterpret_cast<const float4*>(s_xw + s * xs + rb);
                 const float4 xa = xw4[0], xb = xw4[1];
-                const float w[kRB] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-                for (int k = 0; k < kRB; ++k) {
-                    acc[k].x = fmaf(w[k], bv.x, acc[k].x);
-                    acc[k].y = fmaf(w[k], bv.y, acc[k].y);
-                    acc[k].z = fmaf(w[k], bv.z, acc[k].z);
-                    acc[k].w = fmaf(w[k], bv.w, acc[k].w);
-                }
+                const float2 w2[4] = {make_float2(xa.x, xa.y), make_float2(xa.z, xa.w), make_float2(xb.x, xb.y),
+                                      make_float2(xb.z, xb.w)};
+                rank1_8x4(acc2, w2, bv);
             }
         }
 #pragma unroll
-        for (int k = 0; k < kRB; ++k) emit(rb + k, col4, acc[k], rb + k < P);
+        for (int k = 0; k < kRB; ++k) emit(rb + k, col4, acc2_row(acc2, k), rb + k < P);
     }
 }
 
@@ -568,7 +563,8 @@ __host__ __device__ constexpr int pipe_threads(int nt, int rf) {
 // B.C products and decays, the stage barriers, the abort flag (plus slack for
 // what the compiler adds); the dynamic stages get the rest.
 __host__ __device__ constexpr size_t pipe_static_smem(int nt, int rf) {
-    return static_cast<size_t>(pipe_groups(nt, rf)) * nt * (2 * kMaxCap + 1) * 4 + 2 * kPipeStagesMax * 8 + 1024;
+    return static_cast<size_t>(pipe_groups(nt, rf)) * nt * (2 * kMaxCap + 1) * 4 + 2 * kPipeStagesMax * 8 + 1024 +
+           (nt == 1 && rf == kFP4 ? static_cast<size_t>(pipe_groups(nt, rf)) * kMaxHeadDim * 4 : 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -604,12 +600,14 @@ __device__ __forceinline__ void bc_products_mma(const __nv_bfloat16* br, const _
     load_bf16_chunks(cb, g < ntok ? nc + g * kD128 : nullptr, t, true);
     load_bf16_chunks(r0, row_of(s0 + g), t, true);
     load_bf16_chunks(r1, row_of(s0 + g + 8), t, true);
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    float d[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};  // two independent chains
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         mma_bf16(d, r0[c].x, r1[c].x, r0[c].y, r1[c].y, cb[c].x, cb[c].y);
-        mma_bf16(d, r0[c].z, r1[c].z, r0[c].w, r1[c].w, cb[c].z, cb[c].w);
+        mma_bf16(e, r0[c].z, r1[c].z, r0[c].w, r1[c].w, cb[c].z, cb[c].w);
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] += e[i];
     const int sa = s0 + g, sb = s0 + g + 8, j0 = 2 * t, j1 = 2 * t + 1;
     if (sa < T) {
         if (j0 < ntok) s_g[j0 * kMaxCap + sa] = d[0];
@@ -649,8 +647,10 @@ __device__ __forceinline__ void hc_bfrag(const uint4 (&cb)[4], uint32_t (&bfrag)
 // past P read as zero.
 template <int RF, bool SCALE_A>
 __device__ __forceinline__ void hc_mma(const unsigned char* tile, const unsigned char* sc, int R0, int P,
-                                       const uint32_t (&bfrag)[16], float (&d)[4]) {
+                                       const uint32_t (&bfrag)[16], float (&d_out)[4]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    // two independent accumulation chains (even / odd steps), added at the end
+    float d[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
     const int ra = R0 + g, rb = R0 + g + 8;
     const bool va = ra < P, vb = rb < P;
     if constexpr (RF == kF32) {
@@ -676,7 +676,7 @@ __device__ __forceinline__ void hc_mma(const unsigned char* tile, const unsigned
                 // step 4c + u: k lo = column 2u of the chunk, k hi = column 2u + 1
                 const uint32_t q0 = bf16lo_bits(bfrag[4 * c + u]), q1 = bf16hi_bits(bfrag[4 * c + u]);
                 mma_tf32(d, h0, h1, h2, h3, q0, q1);
-                mma_tf32(d, l0, l1, l2, l3, q0, q1);
+                mma_tf32(e, l0, l1, l2, l3, q0, q1);
             }
         }
     } else if constexpr (RF == kBF16) {
@@ -687,7 +687,7 @@ __device__ __forceinline__ void hc_mma(const unsigned char* tile, const unsigned
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             mma_bf16(d, u0[c].x, u1[c].x, u0[c].y, u1[c].y, bfrag[4 * c], bfrag[4 * c + 1]);
-            mma_bf16(d, u0[c].z, u1[c].z, u0[c].w, u1[c].w, bfrag[4 * c + 2], bfrag[4 * c + 3]);
+            mma_bf16(e, u0[c].z, u1[c].z, u0[c].w, u1[c].w, bfrag[4 * c + 2], bfrag[4 * c + 3]);
         }
     } else if constexpr (RF == kE4M3) {
         // 32 codes of a row per lane: two 16-byte words, chunk c = word half c & 1 of e[c >> 1]
@@ -703,7 +703,10 @@ __device__ __forceinline__ void hc_mma(const unsigned char* tile, const unsigned
             uint32_t a0, a2, a1, a3;
             e4m3x4_h2(wa[m], a0, a2);
             e4m3x4_h2(wb[m], a1, a3);
-            mma_f16(d, a0, a1, a2, a3, bfrag[2 * m], bfrag[2 * m + 1]);
+            if (m & 1)
+                mma_f16(e, a0, a1, a2, a3, bfrag[2 * m], bfrag[2 * m + 1]);
+            else
+                mma_f16(d, a0, a1, a2, a3, bfrag[2 * m], bfrag[2 * m + 1]);
         }
     } else {
         // FP4: 32 codes of a row per lane in one 16-byte word; scales of the
@@ -732,33 +735,59 @@ __device__ __forceinline__ void hc_mma(const unsigned char* tile, const unsigned
                 }
             }
             mma_f16(d, ha[0], hb[0], ha[1], hb[1], bfrag[4 * c], bfrag[4 * c + 1]);
-            mma_f16(d, ha[2], hb[2], ha[3], hb[3], bfrag[4 * c + 2], bfrag[4 * c + 3]);
+            mma_f16(e, ha[2], hb[2], ha[3], hb[3], bfrag[4 * c + 2], bfrag[4 * c + 3]);
         }
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d_out[i] += d[i] + e[i];
+}
+
+// d += the bare code . C block sums of the FP4 decode for rows g (qa) and
+// g + 8 (qb): the lane's 32 codes of each row in one 16-byte word; bfrag
+// holds C only in the column of the block a step's k falls in.
+__device__ __forceinline__ void fp4_codes_mma(const uint4& qa, const uint4& qb, const uint32_t (&bfrag)[16],
+                                              float (&d_out)[4]) {
+    float d[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t ha[4], hb[4];
+        e2m1x8_h2(wa[c], ha);
+        e2m1x8_h2(wb[c], hb);
+        mma_f16(d, ha[0], hb[0], ha[1], hb[1], bfrag[4 * c], bfrag[4 * c + 1]);
+        mma_f16(e, ha[2], hb[2], ha[3], hb[3], bfrag[4 * c + 2], bfrag[4 * c + 3]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d_out[i] += d[i] + e[i];
 }
 
 // Replay terms of the verify: d += sum_s coef[j][s] x_s[row] for the rows
 // R0 + g, R0 + g + 8 and the tokens j = 2t, 2t+1, over the slots below T
-// (tf32 k8 steps of 8 slots; x exact, coef split hi + lo in cfrag).
-// x_s: the stage's xr + s P (s < pos) or this call's nx + (s - pos) P.
-__device__ __forceinline__ void replay_mma(const __nv_bfloat16* xr, const __nv_bfloat16* nx, int pos, int T, int P,
-                                           int R0, const uint32_t (&cfrag)[16], float (&d)[4]) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int ra = R0 + g, rb = R0 + g + 8;
-    auto xbits = [&](int sl, int r) -> uint32_t {
-        if (sl >= T || r >= P) return 0u;
-        const __nv_bfloat16* row = sl < pos ? xr + sl * P : nx + (sl - pos) * P;
-        return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(row + r)) << 16;
-    };
+// (tf32 k8 steps of 8 slots; x exact, coef split hi + lo in cfrag). xrow[2q]
+// / xrow[2q + 1]: this lane's slot rows 8q + t / 8q + t + 4 (0 past T).
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void replay_mma(const uint32_t (&xrow)[kMaxCap / 4], int T, int P, int R0,
+                                           const uint32_t (&cfrag)[16], float (&d_out)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2;
+    const int ra = min(R0 + g, P - 1), rb = min(R0 + g + 8, P - 1);  // rows past P: read and discarded
+    float d[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
+    // xrow[i]: shared-memory address of the slot's x row (bf16), 0 past T
+    auto xb = [&](int i, int r) -> uint32_t { return xrow[i] ? lds_u16(xrow[i] + 2u * r) << 16 : 0u; };
 #pragma unroll
     for (int q = 0; q < kMaxCap / 8; ++q) {
         if (8 * q < T) {
-            const int s_lo = 8 * q + t, s_hi = 8 * q + t + 4;
-            const uint32_t a0 = xbits(s_lo, ra), a1 = xbits(s_lo, rb), a2 = xbits(s_hi, ra), a3 = xbits(s_hi, rb);
+            const uint32_t a0 = xb(2 * q, ra), a1 = xb(2 * q, rb), a2 = xb(2 * q + 1, ra), a3 = xb(2 * q + 1, rb);
             mma_tf32(d, a0, a1, a2, a3, cfrag[4 * q], cfrag[4 * q + 1]);
-            mma_tf32(d, a0, a1, a2, a3, cfrag[4 * q + 2], cfrag[4 * q + 3]);
+            mma_tf32(e, a0, a1, a2, a3, cfrag[4 * q + 2], cfrag[4 * q + 3]);
         }
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d_out[i] += d[i] + e[i];
 }
 
 // Stage meta (int words): the position and the index k of the tile the
@@ -778,6 +807,7 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
     __shared__ float s_w[CG][NT][kMaxCap];  // dt_s exp(A (S_t - S_s)) for token j; 0 for s > t
     __shared__ float s_g[CG][NT][kMaxCap];  // B_s . C_j
     __shared__ float s_decay[CG][NT];       // exp(A S_t)
+    __shared__ float s_rep[kMma && NT == 1 ? CG : 1][kMma && NT == 1 ? kMaxHeadDim : 1];  // FP4 decode: replay terms
     __shared__ volatile int s_abort;
 
     const int H = a.s.H, P = a.s.P, N = a.s.N, G = a.s.G, cap = a.s.cap;
@@ -895,10 +925,10 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
     // buffer, all of them 8 rows at a time of the output.
     const int gi = warp / CW, cw = warp - gi * CW;
     const int ctid = tid - gi * CT;
-    unsigned char* nbase = smem + static_cast<size_t>(S) * lay.stage_bytes + static_cast<size_t>(gi) * 3 * lay.newrows;
+    unsigned char* nbase = smem + static_cast<size_t>(S) * lay.stage_bytes + static_cast<size_t>(gi) * 2 * lay.newrows;
     // fused fold: w_s x_s in fp32, [cap][P], per group after the row buffers
     float* s_xw = reinterpret_cast<float*>(smem + static_cast<size_t>(S) * lay.stage_bytes +
-                                           static_cast<size_t>(CG) * 3 * lay.newrows +
+                                           static_cast<size_t>(CG) * 2 * lay.newrows +
                                            static_cast<size_t>(gi) * lay.xw_bytes);
     // this call's rows of tile kk -> buf: [ntok][P] x, [ntok][N] B, [ntok][N] C in
     // 16-byte chunks, then the scalars dt [ntok], A_h, D_h at nd_off
@@ -907,44 +937,41 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
         const uint32_t t = blockIdx.x + static_cast<uint32_t>(kk) * gridDim.x;
         if (t < static_cast<uint32_t>(ntiles)) {
             const int b = fdiv(t, lay.divH), h = t - b * H, g = fdiv(h, lay.divHpg);
-            const int nq = ntok * per_tok;
-            for (int q = ctid; q < nq + ntok + 2; q += CT) {
-                if (q >= nq) {  // scalars, 4 bytes each
-                    const int i = q - nq;
-                    const float* src = i < ntok ? a.dt + (static_cast<size_t>(b) * ntok + i) * H + h
-                                                : (i == ntok ? a.A + h : a.D + h);
-                    const uint32_t dst = smem_u32(buf + lay.nd_off + 4 * (i < ntok ? i : kMaxTok + (i - ntok)));
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-                    continue;
-                }
-                const int j = q / per_tok;
-                int r = q - j * per_tok;
-                const size_t bj = static_cast<size_t>(b) * ntok + j;
+            const size_t b0 = static_cast<size_t>(b) * ntok;
+            const unsigned char* xs = reinterpret_cast<const unsigned char*>(
+                static_cast<const TIn*>(a.x) + b0 * HP + static_cast<size_t>(h) * P);
+            const unsigned char* bs = reinterpret_cast<const unsigned char*>(
+                static_cast<const TIn*>(a.B) + b0 * GN + static_cast<size_t>(g) * N);
+            const unsigned char* cs = reinterpret_cast<const unsigned char*>(
+                static_cast<const TIn*>(a.C) + b0 * GN + static_cast<size_t>(g) * N);
+            // item q = (token j, chunk r): x row (xc chunks of 16 B), B row (bc), C row (bc)
+            for (int q = ctid; q < ntok * per_tok; q += CT) {
+                const int j = static_cast<int>(fdiv(static_cast<uint32_t>(q), lay.divTok)), r = q - j * per_tok;
                 const unsigned char* src;
                 uint32_t dst;
                 if (r < xc) {
-                    src = reinterpret_cast<const unsigned char*>(static_cast<const TIn*>(a.x) + bj * HP +
-                                                                 static_cast<size_t>(h) * P);
-                    dst = smem_u32(buf + j * P * es);
+                    src = xs + static_cast<size_t>(j) * HP * es + 16 * r;
+                    dst = smem_u32(buf + j * P * es) + 16u * r;
                 } else if (r < xc + bc) {
-                    r -= xc;
-                    src = reinterpret_cast<const unsigned char*>(static_cast<const TIn*>(a.B) + bj * GN +
-                                                                 static_cast<size_t>(g) * N);
-                    dst = smem_u32(buf + lay.nb_off + j * N * es);
+                    src = bs + static_cast<size_t>(j) * GN * es + 16 * (r - xc);
+                    dst = smem_u32(buf + lay.nb_off + j * N * es) + 16u * (r - xc);
                 } else {
-                    r -= xc + bc;
-                    src = reinterpret_cast<const unsigned char*>(static_cast<const TIn*>(a.C) + bj * GN +
-                                                                 static_cast<size_t>(g) * N);
-                    dst = smem_u32(buf + lay.nc_off + j * N * es);
+                    src = cs + static_cast<size_t>(j) * GN * es + 16 * (r - xc - bc);
+                    dst = smem_u32(buf + lay.nc_off + j * N * es) + 16u * (r - xc - bc);
                 }
-                cp_async16(dst + 16u * r, src + 16 * r);
+                cp_async16(dst, src);
+            }
+            if (ctid < ntok + 2) {  // scalars, 4 bytes each: dt of each token, A_h, D_h
+                const int i = ctid;
+                const float* src = i < ntok ? a.dt + (b0 + i) * H + h : (i == ntok ? a.A + h : a.D + h);
+                const uint32_t dst = smem_u32(buf + lay.nd_off + 4 * (i < ntok ? i : kMaxTok + (i - ntok)));
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
             }
         }
         cp_async_commit();  // one group per tile, empty past the last tile
     };
-    // rows of this group's first two tiles; later tiles two ahead
+    // rows of this group's first tile; each tile then fetches the next one's
     prefetch(gi, nbase);
-    prefetch(gi + CG, nbase + lay.newrows);
     const uint32_t step = static_cast<uint32_t>(CG) * gridDim.x;
     const int dh = static_cast<int>(step % static_cast<uint32_t>(H)), db = static_cast<int>(step / H);
     const uint32_t t0 = blockIdx.x + static_cast<uint32_t>(gi) * gridDim.x;
@@ -982,11 +1009,15 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                 mbar_wait_bounded(smem_u32(&full_bar[st]), use & 1, kWaitNs);  // copies in flight
             }
         }
-        asm volatile("cp.async.wait_group 1;" ::: "memory");  // this tile's rows (the next may be in flight)
+        cp_async_wait_all();  // this tile's rows
         // the stage and this tile's rows have landed; this group's previous
         // readers of s_w / s_g and of the row buffers are done
         if (group_sync_or(gi, CT, stop)) break;
-        const unsigned char* nr = nbase + (it % 3) * lay.newrows;
+        // the next tile's rows, into the buffer the previous tile used (its
+        // readers all passed the barrier above); they land while this tile works
+        prefetch(k + CG, nbase + ((it + 1) & 1) * lay.newrows);
+        bool released = false;  // the stage went back to the producer before the tile's end
+        const unsigned char* nr = nbase + (it & 1) * lay.newrows;
         const float* sc4 = reinterpret_cast<const float*>(nr + lay.nd_off);  // dt [8], A, D
         const int pos = reinterpret_cast<const int*>(sp + lay.meta)[kMetaPos];
         const int T = pos + ntok;
@@ -1133,39 +1164,73 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                     for (int u = 0; u < 4; ++u) bf[4 * c + u] = mine ? bf[4 * c + u] : 0u;
                 }
                 const float dec = s_decay[gi][0];
-                float cf[kMaxCap / 4];
-#pragma unroll
-                for (int m = 0; m < kMaxCap / 4; ++m) {
-                    const int sl = t + 4 * m;
-                    cf[m] = (sl <= pos) ? s_w[gi][0][sl] * s_g[gi][0][sl] : 0.f;
-                }
-                for (int R0 = 16 * cw; R0 < P; R0 += 16 * CW) {
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    hc_mma<kFP4, false>(tile, sc, R0, P, bf, d);
-                    const int ra = R0 + g, rb = ra + 8;
-                    const bool va = ra < P, vb = rb < P;
-                    const float2 sa = va ? h2_f2(e4m3x2_h2(*reinterpret_cast<const uint16_t*>(sc + ra * (N >> 4) + 2 * t)))
-                                         : make_float2(0.f, 0.f);
-                    const float2 sb = vb ? h2_f2(e4m3x2_h2(*reinterpret_cast<const uint16_t*>(sc + rb * (N >> 4) + 2 * t)))
-                                         : make_float2(0.f, 0.f);
-                    float pa = dec * fmaf(sa.x, d[0], sa.y * d[1]);
-                    float pb = dec * fmaf(sb.x, d[2], sb.y * d[3]);
-#pragma unroll
-                    for (int m = 0; m < kMaxCap / 4; ++m) {
-                        const int sl = t + 4 * m;
-                        if (sl <= pos) {
-                            const TIn* xrow = sl < pos ? xr + sl * P : nx;
-                            if (va) pa = fmaf(cf[m], to_f32(xrow[ra]), pa);
-                            if (vb) pb = fmaf(cf[m], to_f32(xrow[rb]), pb);
-                        }
+                // replay terms sum_{s <= pos} coef_s x_s[p] of every row: lane l
+                // takes rows 2l, 2l + 1 (+ 64 ...), one 32-bit load of x per slot
+                float* rep = s_rep[gi];
+                for (int p0 = 2 * (lane + 32 * cw); p0 < P; p0 += 64 * CW) {
+                    float r0 = 0.f, r1 = 0.f;
+                    for (int sl = 0; sl <= pos; ++sl) {
+                        const float cfs = s_w[gi][0][sl] * s_g[gi][0][sl];
+                        const uint32_t w2 = *reinterpret_cast<const uint32_t*>((sl < pos ? xr + sl * P : nx) + p0);
+                        r0 = fmaf(cfs, __uint_as_float(bf16lo_bits(w2)), r0);
+                        r1 = fmaf(cfs, __uint_as_float(bf16hi_bits(w2)), r1);
                     }
+                    rep[p0] = r0;
+                    rep[p0 + 1] = r1;
+                }
+                if constexpr (CW == 1)
+                    __syncwarp();
+                else
+                    group_sync(gi, CT);
+                // rows R0 + g, R0 + g + 8: scale the two block sums, add the row's
+                // four lanes, then the replay term and D x
+                auto finish = [&](int R0, const float (&d)[4], uint32_t s2a, uint32_t s2b) {
+                    const int ra = R0 + g, rb = ra + 8;
+                    const float2 sa = h2_f2(s2a), sb = h2_f2(s2b);
+                    float pa = fmaf(sa.x, d[0], sa.y * d[1]);
+                    float pb = fmaf(sb.x, d[2], sb.y * d[3]);
                     pa += __shfl_xor_sync(0xffffffffu, pa, 1);
                     pb += __shfl_xor_sync(0xffffffffu, pb, 1);
                     pa += __shfl_xor_sync(0xffffffffu, pa, 2);
                     pb += __shfl_xor_sync(0xffffffffu, pb, 2);
                     if (t == 0) {
-                        if (va) yout[ra] = fmaf(Dh, to_f32(nx[ra]), pa);
-                        if (vb) yout[rb] = fmaf(Dh, to_f32(nx[rb]), pb);
+                        if (ra < P) yout[ra] = fmaf(Dh, to_f32(nx[ra]), fmaf(dec, pa, rep[ra]));
+                        if (rb < P) yout[rb] = fmaf(Dh, to_f32(nx[rb]), fmaf(dec, pb, rep[rb]));
+                    }
+                };
+                auto scales2 = [&](int r) -> uint32_t {  // e4m3 scales of blocks 2t, 2t + 1 of row r as f16
+                    return r < P ? e4m3x2_h2(*reinterpret_cast<const uint16_t*>(sc + r * (N >> 4) + 2 * t)) : 0u;
+                };
+                if (CW == 1 && P <= 64) {
+                    // the lane's codes and scales of every row group into registers,
+                    // then the stage goes back to the producer before the products
+                    uint4 qa[4], qb[4];
+                    uint32_t s2a[4], s2b[4];
+#pragma unroll
+                    for (int rg = 0; rg < 4; ++rg) {
+                        const int ra = 16 * rg + g, rb = ra + 8;
+                        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                        qa[rg] = ra < P ? *reinterpret_cast<const uint4*>(tile + ra * (kD128 / 2) + 16 * t) : z;
+                        qb[rg] = rb < P ? *reinterpret_cast<const uint4*>(tile + rb * (kD128 / 2) + 16 * t) : z;
+                        s2a[rg] = scales2(ra);
+                        s2b[rg] = scales2(rb);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+                    released = true;
+#pragma unroll
+                    for (int rg = 0; rg < 4; ++rg) {
+                        if (16 * rg < P) {
+                            float d[4] = {0.f, 0.f, 0.f, 0.f};
+                            fp4_codes_mma(qa[rg], qb[rg], bf, d);
+                            finish(16 * rg, d, s2a[rg], s2b[rg]);
+                        }
+                    }
+                } else {
+                    for (int R0 = 16 * cw; R0 < P; R0 += 16 * CW) {
+                        float d[4] = {0.f, 0.f, 0.f, 0.f};
+                        hc_mma<kFP4, false>(tile, sc, R0, P, bf, d);
+                        finish(R0, d, scales2(R0 + g), scales2(R0 + g + 8));
                     }
                 }
             } else if constexpr (kMma) {
@@ -1189,12 +1254,17 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                 }
                 const int j0 = 2 * t, j1 = 2 * t + 1;
                 const float dec0 = j0 < ntok ? s_decay[gi][j0] : 0.f, dec1 = j1 < ntok ? s_decay[gi][j1] : 0.f;
-                const __nv_bfloat16* xr16 = reinterpret_cast<const __nv_bfloat16*>(xr);
-                const __nv_bfloat16* nx16 = reinterpret_cast<const __nv_bfloat16*>(nx);
+                // this lane's slot rows for the replay steps: 8q + t and 8q + t + 4
+                uint32_t xrow[kMaxCap / 4];
+#pragma unroll
+                for (int i = 0; i < kMaxCap / 4; ++i) {
+                    const int sl = 8 * (i >> 1) + t + 4 * (i & 1);
+                    xrow[i] = sl < pos ? smem_u32(xr + sl * P) : (sl < T ? smem_u32(nx + (sl - pos) * P) : 0u);
+                }
                 for (int R0 = 16 * cw; R0 < P; R0 += 16 * CW) {
                     float dh[4] = {0.f, 0.f, 0.f, 0.f}, dx[4] = {0.f, 0.f, 0.f, 0.f};
                     hc_mma<RF, true>(tile, sc, R0, P, bf, dh);
-                    replay_mma(xr16, nx16, pos, T, P, R0, cfr, dx);
+                    replay_mma(xrow, T, P, R0, cfr, dx);
                     const int ra = R0 + g, rb = ra + 8;
                     if (ra < P) {
                         if (j0 < ntok) yout[j0 * HP + ra] = fmaf(Dh, to_f32(nx[j0 * P + ra]), fmaf(dec0, dh[0], dx[0]));
@@ -1327,31 +1397,27 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                 float* ck = reinterpret_cast<float*>(rec);
                 for (int r0 = cw * kRB; r0 < P; r0 += CW * kRB) {
                     // acc = alpha h, then the slots in order (as the flush kernels)
-                    float4 acc[kRB];
+                    float2 acc2[4][4];
 #pragma unroll
                     for (int kk = 0; kk < kRB; ++kk) {
                         const float4 hv = reinterpret_cast<const float4*>(sp)[(r0 + kk) * (N >> 2) + lane];
-                        acc[kk] = make_float4(alpha * hv.x, alpha * hv.y, alpha * hv.z, alpha * hv.w);
+                        acc2_set_row(acc2, kk, make_float4(alpha * hv.x, alpha * hv.y, alpha * hv.z, alpha * hv.w));
                     }
 #pragma unroll 2
                     for (int sl = 0; sl < T; ++sl) {
                         const float4 bv = load4((sl < pos ? br + sl * N : nb) + 4 * lane);
                         const float4* xw4 = reinterpret_cast<const float4*>(s_xw + sl * P + r0);
                         const float4 xa = xw4[0], xb = xw4[1];
-                        const float w[kRB] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-                        for (int kk = 0; kk < kRB; ++kk) {
-                            acc[kk].x = fmaf(w[kk], bv.x, acc[kk].x);
-                            acc[kk].y = fmaf(w[kk], bv.y, acc[kk].y);
-                            acc[kk].z = fmaf(w[kk], bv.z, acc[kk].z);
-                            acc[kk].w = fmaf(w[kk], bv.w, acc[kk].w);
-                        }
+                        const float2 w2[4] = {make_float2(xa.x, xa.y), make_float2(xa.z, xa.w),
+                                              make_float2(xb.x, xb.y), make_float2(xb.z, xb.w)};
+                        rank1_8x4(acc2, w2, bv);
                     }
                     float part[kRB];
 #pragma unroll
                     for (int kk = 0; kk < kRB; ++kk) {
-                        stream_store4(ck + (r0 + kk) * N + 4 * lane, acc[kk]);
-                        part[kk] = dot4(acc[kk], c4[0]);
+                        const float4 v = acc2_row(acc2, kk);
+                        stream_store4(ck + (r0 + kk) * N + 4 * lane, v);
+                        part[kk] = dot4(v, c4[0]);
                     }
                     const float z = warp_reduce8(part);
                     const int r = r0 + ((lane >> 2) & 7);
@@ -1362,10 +1428,7 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
-        // rows of the tile after next, into the buffer this group's previous
-        // tile used (every reader of it passed the barrier above)
-        prefetch(k + 2 * CG, nbase + ((it + 2) % 3) * lay.newrows);
+        if (lane == 0 && !released) mbar_arrive(smem_u32(&empty_bar[st]));
         h += dh;
         b += db;
         if (h >= H) {
@@ -1496,6 +1559,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_fold(const FoldArgs a) {
         __syncthreads();
     }
 
+    const PhiloxKeys pkeys = philox_keys(a.seed);
     auto brow = [&](int s, int c) {
         const float w = s_cw[s];
         const float4 v = reinterpret_cast<const float4*>(s_B + s * N)[c];
@@ -1508,9 +1572,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_fold(const FoldArgs a) {
         } else if constexpr (UF == kBF16 || UF == kE4M3) {
             if (valid) {
                 // Philox counter (e/4, head, request, flush_count)
-                const uint4 rw = philox4x32_10(make_uint4(e >> 2, h, b, fc),
-                                               make_uint2(static_cast<uint32_t>(a.seed),
-                                                          static_cast<uint32_t>(a.seed >> 32)));
+                const uint4 rw = philox4x32_10(make_uint4(e >> 2, h, b, fc), pkeys);
                 if constexpr (UF == kBF16) {
                     const uint2 w = make_uint2(sr_bf16(v.x, rw.x) | (sr_bf16(v.y, rw.y) << 16),
                                                sr_bf16(v.z, rw.z) | (sr_bf16(v.w, rw.w) << 16));
@@ -1726,6 +1788,7 @@ __global__ void __launch_bounds__(fold_threads(UF), 1) k_fold_pipe(const FoldArg
     // --------------------------------------------------------------- consumers
     const int gi = warp / CW, cw = warp - gi * CW;
     const int ctid = tid - gi * CT;
+    const PhiloxKeys pkeys = philox_keys(a.seed);
     float* s_Bf = reinterpret_cast<float*>(smem + static_cast<size_t>(S) * lay.stage_bytes +
                                            static_cast<size_t>(gi) * lay.scratch);  // [T][N]
     float* s_xw = s_Bf + cap * N;                                                    // [T][P]
@@ -1811,38 +1874,32 @@ __global__ void __launch_bounds__(fold_threads(UF), 1) k_fold_pipe(const FoldArg
         unsigned char* upd = a.upd + static_cast<size_t>(t) * a.upd_stride;
         unsigned char* rec = a.record + static_cast<size_t>(t) * a.rec.bytes;
         for (int r0 = cw * kRB; r0 < P; r0 += CW * kRB) {
-            // acc = alpha h, then the slots in order (the one-CTA fold's order)
-            float4 acc[kRB];
+            // acc = alpha h, then the slots in order (the one-CTA fold's order),
+            // rows paired for the packed FMAs
+            float2 acc2[4][4];
 #pragma unroll
             for (int kk = 0; kk < kRB; ++kk) {
                 const float4 hv = tile_load4<UF>(tile, tsc, r0 + kk, lane, N);
-                acc[kk] = make_float4(alpha * hv.x, alpha * hv.y, alpha * hv.z, alpha * hv.w);
+                acc2_set_row(acc2, kk, make_float4(alpha * hv.x, alpha * hv.y, alpha * hv.z, alpha * hv.w));
             }
 #pragma unroll 2
             for (int sl = 0; sl < T; ++sl) {
                 const float4 bv = reinterpret_cast<const float4*>(s_Bf + sl * N)[lane];
                 const float4* xw4 = reinterpret_cast<const float4*>(s_xw + sl * P + r0);
                 const float4 xa = xw4[0], xb = xw4[1];
-                const float w[kRB] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-                for (int kk = 0; kk < kRB; ++kk) {
-                    acc[kk].x = fmaf(w[kk], bv.x, acc[kk].x);
-                    acc[kk].y = fmaf(w[kk], bv.y, acc[kk].y);
-                    acc[kk].z = fmaf(w[kk], bv.z, acc[kk].z);
-                    acc[kk].w = fmaf(w[kk], bv.w, acc[kk].w);
-                }
+                const float2 w2[4] = {make_float2(xa.x, xa.y), make_float2(xa.z, xa.w), make_float2(xb.x, xb.y),
+                                      make_float2(xb.z, xb.w)};
+                rank1_8x4(acc2, w2, bv);
             }
 #pragma unroll
             for (int kk = 0; kk < kRB; ++kk) {
                 const int r = r0 + kk;
-                const float4 v = acc[kk];
+                const float4 v = acc2_row(acc2, kk);
                 const uint32_t e = static_cast<uint32_t>(r * N + 4 * lane);  // element of v.x within the head
                 if constexpr (UF == kF32) {
                     stream_store4(reinterpret_cast<float*>(upd) + e, v);
                 } else if constexpr (UF == kBF16 || UF == kE4M3) {
-                    const uint4 rw = philox4x32_10(make_uint4(e >> 2, h, b, fc),
-                                                   make_uint2(static_cast<uint32_t>(a.seed),
-                                                              static_cast<uint32_t>(a.seed >> 32)));
+                    const uint4 rw = philox4x32_10(make_uint4(e >> 2, h, b, fc), pkeys);
                     if constexpr (UF == kBF16) {
                         const uint2 wv = make_uint2(sr_bf16(v.x, rw.x) | (sr_bf16(v.y, rw.y) << 16),
                                                     sr_bf16(v.z, rw.z) | (sr_bf16(v.w, rw.w) << 16));
@@ -1979,6 +2036,205 @@ __global__ void __launch_bounds__(kThreads, 2) k_prefill(const PrefillArgs a) {
         };
         fold_tile(s32, s_x, xs, P, N, lpr, T, s_alpha, brow, emit);
         __syncthreads();  // every reader of this chunk's staging is done
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Prefill on the tensor cores (bf16 inputs, d_state 128, head_dim a multiple
+// of 16 up to 64). The fold of a whole prompt is one contraction per
+// (request, head):
+//   h_T = exp(A S) h_0 + sum_{t < T0} w_t x_t B_t^T,   w_t = dt_t exp(A R_t),
+//   R_t = sum_{t < r < T0} dt_r (the decay from token t to the end), S = R_{-1},
+// i.e. h_T - exp(A S) h_0 = X_w^T B with X_w[t][p] = w_t x_t[p] (K = T0).
+// One CTA of 8 warps per tile walks the prompt in chunks of 64 tokens from
+// the last to the first, so R_t is a running suffix sum (no cancellation).
+// Per chunk: the x rows, B rows and dt land by cp.async (double-buffered,
+// the next chunk while this one computes); warp 0 forms w_t; all threads
+// split w_t x_t[p] into bf16 hi + lo parts (x_w carries ~16 bits; B is bf16,
+// exact); warp w accumulates rows 16 (w % 4).. of the product against the
+// 64 columns 64 (w / 4).. with mma.sync bf16 m16n8k16, operands from shared
+// memory by ldmatrix (rows XOR-swizzled by 16-byte chunk, conflict-free).
+// ---------------------------------------------------------------------------
+constexpr int kPfChunk = 64;                                 // prompt tokens per chunk
+constexpr int kPfThreads = 256;
+constexpr uint32_t kPfX = kPfChunk * 64 * 2;                 // x rows [64][64] bf16
+constexpr uint32_t kPfB = kPfChunk * kD128 * 2;              // B rows [64][128] bf16 (swizzled)
+constexpr uint32_t kPfBuf = kPfX + kPfB + kPfChunk * 4;      // + dt [64]
+constexpr uint32_t kPfA = kPfChunk * 64 * 2;                 // x_w hi or lo [64 tokens][64 rows] (swizzled)
+constexpr size_t kPfSmem = 2 * static_cast<size_t>(kPfBuf) + 2 * kPfA + kPfChunk * 4;
+
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16u : 0u)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4_zfill(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4u : 0u)
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(kPfThreads, 2) k_prefill_mma(const PrefillArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ int s_pos;
+    const int H = a.s.H, P = a.s.P, G = a.s.G, batch = a.s.batch, T0 = a.T0;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.x / H, h = blockIdx.x - b * H, g = h / (H / G);
+    unsigned char* rec = a.record + (static_cast<size_t>(b) * H + h) * a.rec.bytes;
+    unsigned char* aw_hi = smem + 2 * kPfBuf;
+    unsigned char* aw_lo = aw_hi + kPfA;
+    float* s_wt = reinterpret_cast<float*>(aw_lo + kPfA);
+
+    if (tid == 0) s_pos = a.pos[b];  // the only read of pos
+    __syncthreads();
+    if (s_pos != 0) {
+        if (tid == 0) set_error(a.err, RSSM_DEVERR_POS_RANGE);
+        return;
+    }
+    if (T0 <= 0) return;
+    const size_t HP = static_cast<size_t>(H) * P, GN = static_cast<size_t>(G) * kD128;
+    const __nv_bfloat16* xin = static_cast<const __nv_bfloat16*>(a.x) + static_cast<size_t>(b) * HP +
+                               static_cast<size_t>(h) * P;
+    const __nv_bfloat16* Bin = static_cast<const __nv_bfloat16*>(a.B) + static_cast<size_t>(b) * GN +
+                               static_cast<size_t>(g) * kD128;
+    const size_t xstep = static_cast<size_t>(batch) * HP, bstep = static_cast<size_t>(batch) * GN;
+    const int nchunk = (T0 + kPfChunk - 1) / kPfChunk;
+
+    // chunk c (tokens 64c ..) into buffer `buf`: x rows (P bf16), B rows
+    // (chunk j of token k at (j ^ (k & 7))), dt; zeros past T0
+    auto fetch = [&](int c, int buf) {
+        unsigned char* base = smem + static_cast<size_t>(buf) * kPfBuf;
+        const int t0 = c * kPfChunk;
+        const int xq = P / 8;  // 16-byte chunks per x row
+        for (int i = tid; i < kPfChunk * 16; i += kPfThreads) {  // B: 16 chunks per token
+            const int k = i >> 4, j = i & 15, t = t0 + k;
+            const bool ok = t < T0;
+            cp_async16_zfill(smem_u32(base + kPfX + k * (kD128 * 2) + 16 * (j ^ (k & 7))),
+                             Bin + static_cast<size_t>(ok ? t : t0) * bstep + 8 * j, ok);
+        }
+        for (int i = tid; i < kPfChunk * xq; i += kPfThreads) {
+            const int k = i / xq, j = i - k * xq, t = t0 + k;
+            const bool ok = t < T0;
+            cp_async16_zfill(smem_u32(base + k * 128 + 16 * j), xin + static_cast<size_t>(ok ? t : t0) * xstep + 8 * j,
+                             ok);
+        }
+        if (tid < kPfChunk) {
+            const int t = t0 + tid;
+            const bool ok = t < T0;
+            cp_async4_zfill(smem_u32(base + kPfX + kPfB + 4 * tid),
+                            a.dt + (static_cast<size_t>(ok ? t : t0) * batch + b) * H + h, ok);
+        }
+        cp_async_commit();
+    };
+
+    const float Ah = a.A[h];
+    float carry = 0.f;  // sum of dt over the chunks already folded (warp 0)
+    const int mt = warp & 3, nh = warp >> 2;
+    const int R0 = 16 * mt;
+    const bool rows_live = R0 < P;
+    float acc[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+
+    fetch(nchunk - 1, (nchunk - 1) & 1);
+    for (int c = nchunk - 1; c >= 0; --c) {
+        const int buf = c & 1;
+        unsigned char* base = smem + static_cast<size_t>(buf) * kPfBuf;
+        cp_async_wait_all();
+        __syncthreads();  // chunk c landed; the previous chunk's readers are done
+        if (c > 0) fetch(c - 1, buf ^ 1);
+        if (warp == 0) {
+            // w_t = dt_t exp(A R_t): lane l takes tokens l and l + 32 of the chunk
+            const float* dts = reinterpret_cast<const float*>(base + kPfX + kPfB);
+            const float v0 = dts[lane], v1 = dts[lane + 32];
+            float s0 = v0, s1 = v1;  // inclusive suffix sums within each half
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float u0 = __shfl_down_sync(0xffffffffu, s0, off);
+                const float u1 = __shfl_down_sync(0xffffffffu, s1, off);
+                if (lane + off < 32) {
+                    s0 += u0;
+                    s1 += u1;
+                }
+            }
+            const float tot1 = __shfl_sync(0xffffffffu, s1, 0), tot0 = __shfl_sync(0xffffffffu, s0, 0);
+            // R_t = (later chunks) + (later tokens of this chunk), exclusive of t
+            s_wt[lane + 32] = v1 * expf(Ah * (carry + (s1 - v1)));
+            s_wt[lane] = v0 * expf(Ah * ((carry + tot1) + (s0 - v0)));
+            carry = (carry + tot1) + tot0;
+        }
+        __syncthreads();  // weights ready
+        {
+            // x_w = w_t x_t[p] as bf16 hi + lo: thread -> token tid / 4, rows 16 (tid % 4) ..
+            const int k = tid >> 2, p0 = 16 * (tid & 3);
+            const float w = s_wt[k];
+            uint32_t hi[8], lo[8];
+            if (p0 < P) {
+                const uint4 u0 = *reinterpret_cast<const uint4*>(base + k * 128 + 2 * p0);
+                const uint4 u1 = *reinterpret_cast<const uint4*>(base + k * 128 + 2 * p0 + 16);
+                const uint32_t xw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float f0 = w * __uint_as_float(bf16lo_bits(xw[q]));
+                    const float f1 = w * __uint_as_float(bf16hi_bits(xw[q]));
+                    const uint32_t hh = f32x2_to_bf16x2(f0, f1);
+                    hi[q] = hh;
+                    lo[q] = f32x2_to_bf16x2(f0 - __uint_as_float(bf16lo_bits(hh)), f1 - __uint_as_float(bf16hi_bits(hh)));
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) hi[q] = lo[q] = 0u;
+            }
+            const int c0 = p0 >> 3;  // 16-byte chunk of the row
+            uint4* dh0 = reinterpret_cast<uint4*>(aw_hi + k * 128 + 16 * (c0 ^ (k & 7)));
+            uint4* dh1 = reinterpret_cast<uint4*>(aw_hi + k * 128 + 16 * ((c0 + 1) ^ (k & 7)));
+            uint4* dl0 = reinterpret_cast<uint4*>(aw_lo + k * 128 + 16 * (c0 ^ (k & 7)));
+            uint4* dl1 = reinterpret_cast<uint4*>(aw_lo + k * 128 + 16 * ((c0 + 1) ^ (k & 7)));
+            *dh0 = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *dh1 = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+            *dl0 = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            *dl1 = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+        }
+        __syncthreads();  // x_w ready
+        if (rows_live) {
+            const int j = lane >> 3, r = lane & 7;
+#pragma unroll
+            for (int ks = 0; ks < kPfChunk / 16; ++ks) {
+                // A (rows R0.., tokens 16 ks..): matrix j = (rows 8 (j & 1).., tokens 8 (j >> 1)..)
+                const int ka = 16 * ks + r + 8 * (j >> 1), pc = (R0 >> 3) + (j & 1);
+                uint32_t ah[4], al[4];
+                ldsm_x4_trans(smem_u32(aw_hi + ka * 128 + 16 * (pc ^ (ka & 7))), ah[0], ah[1], ah[2], ah[3]);
+                ldsm_x4_trans(smem_u32(aw_lo + ka * 128 + 16 * (pc ^ (ka & 7))), al[0], al[1], al[2], al[3]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    // B of n-tiles 8 nh + 2q, + 1: matrix j = (tokens 8 (j & 1).., n-tile 2q + (j >> 1))
+                    const int kb = 16 * ks + r + 8 * (j & 1), ncn = 8 * nh + 2 * q + (j >> 1);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_trans(smem_u32(base + kPfX + kb * (kD128 * 2) + 16 * (ncn ^ (kb & 7))), b0, b1, b2, b3);
+                    mma_bf16(acc[2 * q], ah[0], ah[1], ah[2], ah[3], b0, b1);
+                    mma_bf16(acc[2 * q], al[0], al[1], al[2], al[3], b0, b1);
+                    mma_bf16(acc[2 * q + 1], ah[0], ah[1], ah[2], ah[3], b2, b3);
+                    mma_bf16(acc[2 * q + 1], al[0], al[1], al[2], al[3], b2, b3);
+                }
+            }
+        }
+    }
+    // h_T = exp(A S) h_0 + acc, S = the prompt's dt sum (warp 0's carry)
+    if (warp == 0 && lane == 0) s_wt[0] = expf(Ah * carry);
+    __syncthreads();
+    const float alpha = s_wt[0];
+    if (rows_live) {
+        const int gq = lane >> 2, tq = lane & 3;
+        float* hrow = reinterpret_cast<float*>(rec);
+#pragma unroll
+        for (int jn = 0; jn < 8; ++jn) {
+            const int n = 64 * nh + 8 * jn + 2 * tq;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int r = R0 + gq + 8 * half;
+                float2* pp = reinterpret_cast<float2*>(hrow + static_cast<size_t>(r) * kD128 + n);
+                const float2 h0 = *pp;
+                *pp = make_float2(fmaf(alpha, h0.x, acc[jn][2 * half]), fmaf(alpha, h0.y, acc[jn][2 * half + 1]));
+            }
+        }
     }
 }
 
@@ -2257,12 +2513,13 @@ PipeLayout pipe_layout(const Shape& s, const RecLayout& rec, int ntok, int in_bf
     L.nd_off = L.nc_off + align16(static_cast<uint32_t>(ntok * s.N) * es);
     L.newrows = (L.nd_off + 4u * (kMaxTok + 2) + 127u) & ~127u;
     L.xw_bytes = fused ? (4u * static_cast<uint32_t>(s.cap * s.P) + 127u) & ~127u : 0u;
-    const size_t rows = static_cast<size_t>(groups) * (3u * L.newrows + L.xw_bytes);
+    const size_t rows = static_cast<size_t>(groups) * (2u * L.newrows + L.xw_bytes);
     const size_t n = smem_budget > rows ? (smem_budget - rows) / L.stage_bytes : 0;
     L.stages = static_cast<int>(n < static_cast<size_t>(kPipeStagesMax) ? n : kPipeStagesMax);
     L.budget = smem_budget;
     L.divH = make_fastdiv(static_cast<uint32_t>(s.H));
     L.divHpg = make_fastdiv(static_cast<uint32_t>(s.H / s.G));
+    L.divTok = make_fastdiv((static_cast<uint32_t>(s.P) + 2u * static_cast<uint32_t>(s.N)) * es / 16u);
     return L;
 }
 
@@ -2298,7 +2555,7 @@ static DeviceInfo device_info() {
 template <typename TIn, int NT>
 static cudaError_t pipe_dispatch(const ReplayArgs& a, const PipeLayout& L, int rf, int grid, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(L.stages) * L.stage_bytes +
-                        static_cast<size_t>(pipe_groups(NT, rf)) * (3u * L.newrows + L.xw_bytes);
+                        static_cast<size_t>(pipe_groups(NT, rf)) * (2u * L.newrows + L.xw_bytes);
     if (smem > L.budget) return cudaErrorInvalidValue;
     if constexpr (NT == 1) {
         if (a.fused) {
@@ -2452,6 +2709,14 @@ cudaError_t launch_fold(const FoldArgs& a, int in_bf16, int uf, cudaStream_t st)
 }
 
 cudaError_t launch_prefill(const PrefillArgs& a, int in_bf16, cudaStream_t st) {
+    if (in_bf16 && a.s.N == 128 && a.s.P % 16 == 0 && a.s.P <= 64) {
+        if (a.s.batch * a.s.H <= 0) return cudaSuccess;
+        cudaError_t e = cudaFuncSetAttribute(k_prefill_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kPfSmem));
+        if (e != cudaSuccess) return e;
+        k_prefill_mma<<<a.s.batch * a.s.H, kPfThreads, kPfSmem, st>>>(a);
+        return cudaGetLastError();
+    }
     const size_t smem = 4u * (static_cast<size_t>(a.s.P) * a.s.N + static_cast<size_t>(kPrefillChunk) * a.s.N +
                               static_cast<size_t>(kPrefillChunk) * round_up8(a.s.P));
     const int nblk = a.s.batch * a.s.H;

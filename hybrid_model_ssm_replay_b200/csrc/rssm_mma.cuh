@@ -117,6 +117,25 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
     return d;
 }
 
+// Four 8x8 b16 matrices from shared memory, transposed: lane 8j + r gives
+// the address of row r of matrix j; register j receives matrix j with lane
+// (g, t) holding its elements (2t, g) and (2t + 1, g) -- the A fragment of a
+// row-major operand stored k-major, or the B fragment of an operand stored
+// [k][n].
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                              uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// Two fp32 values as a bf16 pair, rounded to nearest (lo in the low half).
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
 // An f16 pair (h, h) from the low or high half of x.
 __device__ __forceinline__ uint32_t h2_dup_lo(uint32_t x) { return (x & 0xFFFFu) | (x << 16); }
 __device__ __forceinline__ uint32_t h2_dup_hi(uint32_t x) { return (x >> 16) | (x & 0xFFFF0000u); }

@@ -1,7 +1,10 @@
 """Prefill of a prompt into the checkpoint (the step before the decode path;
 the article is silent on it): the checkpoint after rssm_prefill equals the
 fp64 recurrence over the prompt, and decoding on from it equals the
-recurrence over prompt + decoded tokens."""
+recurrence over prompt + decoded tokens. bf16 inputs at d_state 128 and
+head_dim 16/32/48/64 run the tensor-core contraction over 64-token chunks
+(whole and partial chunks are covered); other shapes the chunked CUDA-core
+fold."""
 import numpy as np
 import pytest
 import torch
@@ -29,7 +32,9 @@ def split(inp, T0):
 
 @pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
 @pytest.mark.parametrize("shape,T0", [(LayerShape(4, 4, 40, 128, 2), 50), (LayerShape(3, 4, 17, 64, 1), 33),
-                                      (LayerShape(2, 2, 8, 16, 1), 16)], ids=["d128", "ragged", "one-chunk"])
+                                      (LayerShape(2, 2, 8, 16, 1), 16), (LayerShape(3, 4, 64, 128, 2), 150),
+                                      (LayerShape(2, 4, 32, 128, 2), 64), (LayerShape(2, 2, 48, 128, 1), 200)],
+                         ids=["d128", "ragged", "one-chunk", "mma-3chunks", "mma-1chunk", "mma-headdim48"])
 def test_prefill_then_decode_matches_recurrence(shape, T0, in_dtype):
     steps = T0 + 24
     inp = make_inputs(shape, steps, 41, in_dtype, device="cuda")
