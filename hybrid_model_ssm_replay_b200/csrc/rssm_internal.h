@@ -75,7 +75,6 @@ struct PipeLayout {
     int stages;
     size_t budget;  // dynamic shared memory the layout may use
     FastDiv divH, divHpg;  // tile -> (request, head), head -> group
-    FastDiv divTok;        // prefetch item -> token (16-byte chunks per token)
 };
 
 // Fold of the buffer into the update copy (flush / refresh; s1, s4).

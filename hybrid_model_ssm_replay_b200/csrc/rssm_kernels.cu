@@ -944,22 +944,26 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                 static_cast<const TIn*>(a.B) + b0 * GN + static_cast<size_t>(g) * N);
             const unsigned char* cs = reinterpret_cast<const unsigned char*>(
                 static_cast<const TIn*>(a.C) + b0 * GN + static_cast<size_t>(g) * N);
-            // item q = (token j, chunk r): x row (xc chunks of 16 B), B row (bc), C row (bc)
-            for (int q = ctid; q < ntok * per_tok; q += CT) {
-                const int j = static_cast<int>(fdiv(static_cast<uint32_t>(q), lay.divTok)), r = q - j * per_tok;
-                const unsigned char* src;
-                uint32_t dst;
-                if (r < xc) {
-                    src = xs + static_cast<size_t>(j) * HP * es + 16 * r;
-                    dst = smem_u32(buf + j * P * es) + 16u * r;
-                } else if (r < xc + bc) {
-                    src = bs + static_cast<size_t>(j) * GN * es + 16 * (r - xc);
-                    dst = smem_u32(buf + lay.nb_off + j * N * es) + 16u * (r - xc);
-                } else {
-                    src = cs + static_cast<size_t>(j) * GN * es + 16 * (r - xc - bc);
-                    dst = smem_u32(buf + lay.nc_off + j * N * es) + 16u * (r - xc - bc);
+            for (int j = 0; j < ntok; ++j) {
+                // token j: x row (xc chunks of 16 B), B row (bc), C row (bc)
+                for (int r = ctid; r < per_tok; r += CT) {
+                    const unsigned char* src;
+                    uint32_t dst;
+                    if (r < xc) {
+                        src = xs + 16 * r;
+                        dst = smem_u32(buf + j * P * es) + 16u * r;
+                    } else if (r < xc + bc) {
+                        src = bs + 16 * (r - xc);
+                        dst = smem_u32(buf + lay.nb_off + j * N * es) + 16u * (r - xc);
+                    } else {
+                        src = cs + 16 * (r - xc - bc);
+                        dst = smem_u32(buf + lay.nc_off + j * N * es) + 16u * (r - xc - bc);
+                    }
+                    cp_async16(dst, src);
                 }
-                cp_async16(dst, src);
+                xs += HP * es;
+                bs += GN * es;
+                cs += GN * es;
             }
             if (ctid < ntok + 2) {  // scalars, 4 bytes each: dt of each token, A_h, D_h
                 const int i = ctid;
@@ -2519,7 +2523,6 @@ PipeLayout pipe_layout(const Shape& s, const RecLayout& rec, int ntok, int in_bf
     L.budget = smem_budget;
     L.divH = make_fastdiv(static_cast<uint32_t>(s.H));
     L.divHpg = make_fastdiv(static_cast<uint32_t>(s.H / s.G));
-    L.divTok = make_fastdiv((static_cast<uint32_t>(s.P) + 2u * static_cast<uint32_t>(s.N)) * es / 16u);
     return L;
 }
 
