@@ -393,7 +393,7 @@ def replay_loop(rssm, torch, shape, wl, K, W, dev, rank, barrier, max_over_ranks
     sampler.start()
     time.sleep(0.15)
 
-    def timed_region():
+    def timed_region(K):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K + 1)]
         barrier()
         torch.cuda.synchronize()
@@ -413,7 +413,7 @@ def replay_loop(rssm, torch, shape, wl, K, W, dev, rank, barrier, max_over_ranks
         return ms, dec, fl
 
     t0 = time.time()
-    ms_local, dec_ms, fl_ms = timed_region()
+    ms_local, dec_ms, fl_ms = timed_region(K)
     t1 = time.time()
     ms = max_over_ranks(ms_local)
     if rssm.rssm_get_error(st) != 0:
@@ -421,16 +421,21 @@ def replay_loop(rssm, torch, shape, wl, K, W, dev, rank, barrier, max_over_ranks
     res = {"ms": ms, "decode_us": dec_ms * 1e3, "flush_us": fl_ms * 1e3 if not fused else None,
            "inp": inp, "state": st}
     if repeats:
+        # each run: two untimed intervals, then at least 512 decode tokens
+        KR = max(K, -(-512 // L))
         runs = []
         for _ in range(repeats):
-            m, d, f = timed_region()
+            run(0)
+            run(1)
+            m, d, f = timed_region(KR)
             runs.append((max_over_ranks(m), d, f))
-        vals = sorted(world * shape.batch * L * K / (m / 1e3) for m, _, _ in runs)
-        res["repeats"] = {"runs": repeats, "steps_each": K, "unit": UNIT,
+        vals = sorted(world * shape.batch * L * KR / (m / 1e3) for m, _, _ in runs)
+        res["repeats"] = {"runs": repeats, "steps_each": KR, "decode_tokens_each": KR * L,
+                          "warmup_intervals_each": 2, "unit": UNIT,
                           "median": statistics.median(vals), "min": vals[0], "max": vals[-1],
                           "decode_us_median": statistics.median(d * 1e3 for _, d, _ in runs),
                           "flush_us_median": None if fused else statistics.median(f * 1e3 for _, _, f in runs),
-                          "note": "the same timed region run again after the contract run"}
+                          "note": "the timed region run again after the contract run, each run at least 512 decode tokens after two untimed intervals"}
     time.sleep(0.06)
     sampler.stop()
     res["clocks"] = sampler.summary(t0, t1)

@@ -333,17 +333,34 @@ __device__ __forceinline__ float4 bf16x4_val(uint2 w) {
 }
 
 // FP4 copy of 16 contiguous values held as one float4 by each of 4
-// consecutive lanes: scale = e4m3_rn(amax / 6), codes = e2m1_rn(v / scale),
-// all codes 0 when the scale is 0. All 32 lanes must call it. Returns this
-// lane's 16 code bits and sets *scale_code.
+// consecutive lanes: scale = e4m3_rn(amax / 6), codes = e2m1_rn(v / scale)
+// with both quotients the correctly rounded fp32 ones, all codes 0 when the
+// scale is 0. All 32 lanes must call it. Returns this lane's 16 code bits
+// and sets *scale_code.
+//
+// The quotients are bracketed instead of divided: for x >= 0 and c_lo <=
+// 1/d <= c_hi, x c_lo <= x / d <= x c_hi, and fp32 rounding and both
+// nearest-even conversions are monotone, so when the two ends convert to the
+// same code, that is the code of the rounded quotient. 1/6 lies between two
+// adjacent floats; 1/scale comes from rcp.approx (within 2^-23 relative) and
+// is widened by 2^-19 either way. Only a lane whose ends differ (a quotient
+// within about 2^-19 of a rounding boundary) divides.
 __device__ __forceinline__ uint32_t fp4_quant_quad(float4 v, uint32_t* scale_code) {
     float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    const uint32_t sc = e4m3_rn(__fdiv_rn(amax, 6.0f));
+    constexpr float kSixthLo = 0x1.555555p-3f, kSixthHi = 0x1.555556p-3f;  // kSixthLo < 1/6 < kSixthHi
+    uint32_t sc = e4m3_rn(amax * kSixthLo);
+    if (sc != e4m3_rn(amax * kSixthHi)) sc = e4m3_rn(__fdiv_rn(amax, 6.0f));
     *scale_code = sc;
     const float s = e4m3_val(sc);
     if (s == 0.0f) return 0u;
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));  // s >= 2^-9: never subnormal
+    const float rlo = r * (1.0f - 0x1p-19f), rhi = r * (1.0f + 0x1p-19f);
+    const uint32_t lo = e2m1x2_rn(v.x * rlo, v.y * rlo) | (e2m1x2_rn(v.z * rlo, v.w * rlo) << 8);
+    const uint32_t hi = e2m1x2_rn(v.x * rhi, v.y * rhi) | (e2m1x2_rn(v.z * rhi, v.w * rhi) << 8);
+    if (lo == hi) return lo;
     const uint32_t c01 = e2m1x2_rn(__fdiv_rn(v.x, s), __fdiv_rn(v.y, s));
     const uint32_t c23 = e2m1x2_rn(__fdiv_rn(v.z, s), __fdiv_rn(v.w, s));
     return c01 | (c23 << 8);

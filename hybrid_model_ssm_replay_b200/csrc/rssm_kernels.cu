@@ -487,8 +487,9 @@ __global__ void __launch_bounds__(kThreads, replay_min_blocks(NT, FUSED)) k_repl
 // Persistent, warp-specialised replay decode / verify for d_state 128 and
 // head_dim a multiple of 8. One CTA per SM walks the tiles
 // t = blockIdx.x + k * gridDim.x ((request, head) = (t / H, t % H)).
-// A producer warp reads each tile's position one tile ahead and brings the
-// tile's state into a ring of shared-memory stages with two bulk copies (the
+// A producer warp (one lane per tile, a batch of tiles per pass) reads each
+// tile's position a batch ahead and brings the tile's state into a ring of
+// shared-memory stages with two bulk copies (the
 // record prefix -- copy, dt row and buffered x rows -- and the buffered B
 // rows; completion on the stage's "full" mbarrier). Consumer warps compute
 // the outputs from shared memory only and release the stage (its "empty"
@@ -793,6 +794,8 @@ __device__ __forceinline__ void replay_mma(const uint32_t (&xrow)[kMaxCap / 4], 
 // Stage meta (int words): the position and the index k of the tile the
 // stage holds (-1 before its first use).
 constexpr int kMetaPos = 0, kMetaTile = 1;
+constexpr int kProdBatch = 8;  // most tiles the producer warp issues per pass (one per lane)
+constexpr int kProdDiv = 3;    // ... and at most a third of the stages
 
 template <typename TIn, int RF, int NT, int FUSED>
 __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const ReplayArgs a, const PipeLayout lay) {
@@ -830,89 +833,74 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
 
     if (warp == CG * CW) {
         // ------------------------------------------------------------ producer
-        // Only what the copies need: the position (lane i holds that of the
-        // i-th tile of the current batch of 32 and loads the next batch, so
-        // no load latency sits between two issues), the record and B-row
-        // addresses, the stage. Everything else is the consumers' work.
-        int p0 = 0, p1 = 0;
-        auto fetch = [&](int kbase, int& pp) {
-            const uint32_t tt = blockIdx.x + static_cast<uint32_t>(kbase + lane) * gridDim.x;
-            if (tt < static_cast<uint32_t>(ntiles)) pp = a.pos[fdiv(tt, lay.divH)];
+        // Only what the copies need, for nb tiles per pass: lane i takes tile
+        // kb + i of the batch kb.. -- its position (loaded one batch ahead),
+        // its stage, the record and B-row addresses -- so one pass of the
+        // warp's instructions issues the copies of nb tiles. A batch waits
+        // for its nb stages together, so nb is a third of the ring (the rest
+        // stays in flight meanwhile); the lanes of a batch never share a
+        // stage. Everything else is the consumers' work.
+        const int nb = S / kProdDiv < 1 ? 1 : (S / kProdDiv > kProdBatch ? kProdBatch : S / kProdDiv);
+        const bool lane_on = lane < nb;
+        auto tile_of = [&](int k) { return blockIdx.x + static_cast<uint32_t>(k) * gridDim.x; };
+        auto load_pos = [&](int k) {
+            const uint32_t t = tile_of(k);
+            return (lane_on && t < static_cast<uint32_t>(ntiles)) ? a.pos[fdiv(t, lay.divH)] : 0;
         };
-        fetch(0, p0);
-        fetch(32, p1);
-        const uint32_t step = gridDim.x;
-        const int dh = static_cast<int>(step % static_cast<uint32_t>(H)), db = static_cast<int>(step / H);
-        int b = fdiv(blockIdx.x, lay.divH), h = static_cast<int>(blockIdx.x) - b * H;
-        const unsigned char* rsrc = a.record + static_cast<size_t>(blockIdx.x) * a.rec.bytes;
-        const size_t rstep = static_cast<size_t>(step) * a.rec.bytes;
         const size_t brow_bytes = static_cast<size_t>(cap) * N * es;
-        int st = 0, use = 0;
-        int k_issued = -1;  // last tile index issued
+        int pnext = load_pos(lane);
+        int st = lane, use = 0;  // stage of tile kb + lane and its use count
+        int kb = 0;
         bool aborted = false;
-        for (int k = 0; blockIdx.x + static_cast<uint32_t>(k) * step < static_cast<uint32_t>(ntiles); ++k) {
-            const bool cur = (k >> 5) & 1;
-            const int sel = k & 31;
-            if (sel == 0 && k > 0) {  // refill the other buffer with the batch after this one
-                if (cur)
-                    fetch(k + 32, p0);
-                else
-                    fetch(k + 32, p1);
+        for (; tile_of(kb) < static_cast<uint32_t>(ntiles); kb += nb) {
+            const int k = kb + lane;
+            const uint32_t t = tile_of(k);
+            const bool mine = lane_on && t < static_cast<uint32_t>(ntiles);
+            const int pos = pnext;
+            pnext = load_pos(k + nb);
+            bool fail = false;
+            if (mine && use > 0) fail = !mbar_wait_bounded(smem_u32(&empty_bar[st]), (use - 1) & 1, kWaitNs);
+            if (fail) {
+                set_error(a.err, RSSM_DEVERR_TIMEOUT);
+                s_abort = 1;
             }
-            // a uniform branch picks the batch, so the warp never reads the
-            // registers of the batch still being loaded
-            const int pos = cur ? __shfl_sync(0xffffffffu, p1, sel) : __shfl_sync(0xffffffffu, p0, sel);
-            const bool ok = pos >= 0 && pos + ntok <= cap;
-            unsigned char* sp = smem + static_cast<size_t>(st) * lay.stage_bytes;
-            int live = 1;
-            if (lane == 0) {
-                if (use > 0 && !mbar_wait_bounded(smem_u32(&empty_bar[st]), (use - 1) & 1, kWaitNs)) {
-                    set_error(a.err, RSSM_DEVERR_TIMEOUT);
-                    s_abort = 1;
-                }
-                live = !s_abort;
-            }
-            live = __shfl_sync(0xffffffffu, live, 0);  // one decision for the whole warp
-            if (!live) {
+            // one decision for the whole warp, before any copy of the batch
+            if (__any_sync(0xffffffffu, fail || s_abort)) {
                 aborted = true;
                 break;
             }
-            if (lane == 0) {
+            if (mine) {
+                const int b = fdiv(t, lay.divH), h = static_cast<int>(t) - b * H;
+                unsigned char* sp = smem + static_cast<size_t>(st) * lay.stage_bytes;
                 const uint32_t fb = smem_u32(&full_bar[st]);
                 int* meta = reinterpret_cast<int*>(sp + lay.meta);
                 meta[kMetaPos] = pos;
                 reinterpret_cast<volatile int*>(meta)[kMetaTile] = k;
+                const bool ok = pos >= 0 && pos + ntok <= cap;
                 // record prefix: copy, scales, dt row and x rows 0..pos-1
                 const uint32_t nrec = a.rec.x + static_cast<uint32_t>(pos * P * es);
-                const uint32_t nb = static_cast<uint32_t>(pos * N * es);
-                mbar_expect_tx(fb, ok ? nrec + nb : 0u);  // nothing to copy for a bad position
+                const uint32_t nbr = static_cast<uint32_t>(pos * N * es);
+                mbar_expect_tx(fb, ok ? nrec + nbr : 0u);  // nothing to copy for a bad position
                 if (ok) {
-                    bulk_g2s(smem_u32(sp), rsrc, nrec, fb);
-                    if (nb > 0) {
+                    bulk_g2s(smem_u32(sp), a.record + static_cast<size_t>(t) * a.rec.bytes, nrec, fb);
+                    if (nbr > 0) {
                         const size_t bg = static_cast<size_t>(b) * G + fdiv(h, lay.divHpg);
                         bulk_g2s(smem_u32(sp + lay.brows), static_cast<const unsigned char*>(a.bbuf) + bg * brow_bytes,
-                                 nb, fb);
+                                 nbr, fb);
                     }
                 }
             }
-            k_issued = k;
-            rsrc += rstep;
-            h += dh;
-            b += db;
-            if (h >= H) {
-                h -= H;
-                ++b;
-            }
-            if (++st == S) {
-                st = 0;
+            st += nb;
+            if (st >= S) {
+                st -= S;
                 ++use;
             }
             __syncwarp();
         }
         if (aborted && lane == 0) {
             // let every copy this warp issued land before the CTA can exit:
-            // the last S tiles issued are the ones that may be in flight
-            for (int kk = k_issued; kk >= 0 && kk > k_issued - S; --kk)
+            // tiles 0..kb-1 were issued, the last S of them may be in flight
+            for (int kk = kb - 1; kk >= 0 && kk > kb - 1 - S; --kk)
                 mbar_wait_bounded(smem_u32(&full_bar[kk % S]), (kk / S) & 1, kWaitNs);
         }
         return;

@@ -88,10 +88,38 @@ def fp4_tie_blocks():
     return np.concatenate(out).astype(np.float32)
 
 
+def fp4_near_tie_blocks():
+    """Blocks whose quotients v/s, or whose amax/6, lie a few ulps from a
+    rounding boundary of e2m1 or e4m3 (where a bracketed quotient cannot
+    decide the code and the exact division must)."""
+    out = []
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    for sc in (0x01, 0x08, 0x20, 0x38, 0x3A, 0x41, 0x5B, 0x70, 0x7E):
+        s = np.float32(orc.e4m3_value(sc))
+        for k in (1, 2, 3):
+            blk = [np.float32(6.0) * s]
+            for m in mids:
+                x = np.float32(m) * s
+                up, dn = x, x
+                for _ in range(k):
+                    up, dn = np.nextafter(up, np.float32(np.inf)), np.nextafter(dn, np.float32(0))
+                blk += [up, -dn]
+            out.append(np.array(blk + [np.float32(0)], np.float32))
+    # amax / 6 near the midpoint of two adjacent e4m3 values
+    for sc in (0x02, 0x09, 0x21, 0x38, 0x3B, 0x55, 0x7C):
+        m = np.float32((orc.e4m3_value(sc) + orc.e4m3_value(sc + 1)) / 2 * 6)
+        for k in (-3, -1, 0, 1, 3):
+            a = m
+            for _ in range(abs(k)):
+                a = np.nextafter(a, np.float32(np.inf) if k > 0 else np.float32(0))
+            out.append(np.array([a] + [a * np.float32(f) for f in np.linspace(-0.9, 0.9, 15)], np.float32))
+    return np.concatenate(out).astype(np.float32)
+
+
 def test_fp4_block_copy_bit_exact():
     rng = np.random.default_rng(3)
     blocks = (rng.normal(0, 1, (1 << 16, 16)) * np.exp2(rng.uniform(-20, 10, (1 << 16, 1)))).astype(np.float32)
-    v = np.concatenate([fp4_tie_blocks(), blocks.ravel()]).astype(np.float32)
+    v = np.concatenate([fp4_tie_blocks(), fp4_near_tie_blocks(), blocks.ravel()]).astype(np.float32)
     n = v.size
     got = rssm.rssm_round_test(3, torch.from_numpy(v).cuda()).cpu().numpy()
     codes, scales = orc.fp4_quant(v)
