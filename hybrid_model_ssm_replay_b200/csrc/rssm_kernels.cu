@@ -1621,7 +1621,7 @@ constexpr int kFMetaTile = 0, kFMetaPos = 1, kFMetaFc = 2, kFMetaA = 3, kFMetaTa
 // B200: 190 us with 3 groups, 196 with 4), four for the low-precision
 // refreshes, which are bound by issue (Philox draws, rounding, FP4
 // quantisation; bf16 refresh 478 -> 430 us with 4 groups).
-__host__ __device__ constexpr int fold_groups(int uf) { return uf == kF32 ? 3 : 4; }
+__host__ __device__ constexpr int fold_groups(int uf) { return uf == kF32 ? 3 : 5; }
 __host__ __device__ constexpr int fold_cwarps(int uf) { return (void)uf, 4; }
 __host__ __device__ constexpr int fold_threads(int uf) { return (fold_groups(uf) * fold_cwarps(uf) + 1) * 32; }
 
