@@ -349,7 +349,7 @@ __device__ __forceinline__ uint32_t fp4_quant_quad(float4 v, uint32_t* scale_cod
     float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    constexpr float kSixthLo = 0x1.555555p-3f, kSixthHi = 0x1.555556p-3f;  // kSixthLo < 1/6 < kSixthHi
+    constexpr float kSixthLo = 0x1.555554p-3f, kSixthHi = 0x1.555556p-3f;  // adjacent floats around 1/6
     uint32_t sc = e4m3_rn(amax * kSixthLo);
     if (sc != e4m3_rn(amax * kSixthHi)) sc = e4m3_rn(__fdiv_rn(amax, 6.0f));
     *scale_code = sc;

@@ -66,11 +66,13 @@ inline FastDiv make_fastdiv(uint32_t d) {
 // Shared-memory stage of the pipelined replay kernel: a mirror of the
 // record prefix (same offsets as RecLayout, x rows up to cap), the buffered
 // B rows [cap][N] at `brows` and the position and tile index at `meta`;
-// `stages` stages. After them, per consumer group, two buffers of
-// `newrows` bytes for this call's x, B and C rows ([ntok][P], [ntok][N],
-// [ntok][N] at 0, nb_off, nc_off) and its dt [8], A_h, D_h (at nd_off).
+// `stages` stages. This call's x, B and C rows of a tile ([ntok][P],
+// [ntok][N], [ntok][N] at 0, nb_off, nc_off of a row area) come either with
+// the stage (rows != 0: the area at `rows`; the FP4-reading decode) or, by
+// the consumers, into two buffers per consumer group of `newrows` bytes
+// after the stages, with the tile's dt [8], A_h, D_h at nd_off.
 struct PipeLayout {
-    uint32_t stage_bytes, brows, meta, newrows, nb_off, nc_off, nd_off;
+    uint32_t stage_bytes, brows, meta, rows, newrows, nb_off, nc_off, nd_off;
     uint32_t xw_bytes;  // fused fold: per-group fp32 w_s x_s scratch (0 otherwise)
     int stages;
     size_t budget;  // dynamic shared memory the layout may use

@@ -557,6 +557,12 @@ __host__ __device__ constexpr int pipe_groups(int nt, int rf) {
 __host__ __device__ constexpr int pipe_cwarps(int nt, int rf) {
     return nt > 1 ? 4 : (rf == kF32 ? 4 : (rf == kBF16 ? 2 : 1));
 }
+// The FP4-reading decode's producer also brings this call's x, B and C rows
+// with the stage (its consumers are single warps, for which fetching them is
+// a long step of each tile); the other forms fetch them in the consumers.
+__host__ __device__ constexpr bool pipe_rows_in_stage(int nt, int rf, int fused) {
+    return nt == 1 && rf == kFP4 && !fused;
+}
 __host__ __device__ constexpr int pipe_threads(int nt, int rf) {
     return (pipe_groups(nt, rf) * pipe_cwarps(nt, rf) + 1) * 32;
 }
@@ -804,6 +810,7 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
     // bf16 inputs: verify (every copy format) and the FP4 decode form their
     // dot products on the tensor cores
     constexpr bool kMma = std::is_same<TIn, __nv_bfloat16>::value && (NT > 1 || RF == kFP4);
+    constexpr bool kRowsInStage = pipe_rows_in_stage(NT, RF, FUSED);
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full_bar[kPipeStagesMax];
     __shared__ __align__(8) uint64_t empty_bar[kPipeStagesMax];
@@ -880,13 +887,20 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                 // record prefix: copy, scales, dt row and x rows 0..pos-1
                 const uint32_t nrec = a.rec.x + static_cast<uint32_t>(pos * P * es);
                 const uint32_t nbr = static_cast<uint32_t>(pos * N * es);
-                mbar_expect_tx(fb, ok ? nrec + nbr : 0u);  // nothing to copy for a bad position
+                const uint32_t nnew = kRowsInStage ? static_cast<uint32_t>(ntok * (P + 2 * N) * es) : 0u;
+                mbar_expect_tx(fb, ok ? nrec + nbr + nnew : 0u);  // nothing to copy for a bad position
                 if (ok) {
                     bulk_g2s(smem_u32(sp), a.record + static_cast<size_t>(t) * a.rec.bytes, nrec, fb);
-                    if (nbr > 0) {
-                        const size_t bg = static_cast<size_t>(b) * G + fdiv(h, lay.divHpg);
+                    const int g = fdiv(h, lay.divHpg);
+                    const size_t bg = static_cast<size_t>(b) * G + g;
+                    if (nbr > 0)
                         bulk_g2s(smem_u32(sp + lay.brows), static_cast<const unsigned char*>(a.bbuf) + bg * brow_bytes,
                                  nbr, fb);
+                    if constexpr (kRowsInStage) {  // this call's x, B and C rows (one token)
+                        const uint32_t rw = smem_u32(sp + lay.rows);
+                        bulk_g2s(rw, static_cast<const TIn*>(a.x) + static_cast<size_t>(t) * P, P * es, fb);
+                        bulk_g2s(rw + lay.nb_off, static_cast<const TIn*>(a.B) + bg * N, N * es, fb);
+                        bulk_g2s(rw + lay.nc_off, static_cast<const TIn*>(a.C) + bg * N, N * es, fb);
                     }
                 }
             }
@@ -963,7 +977,7 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
         cp_async_commit();  // one group per tile, empty past the last tile
     };
     // rows of this group's first tile; each tile then fetches the next one's
-    prefetch(gi, nbase);
+    if constexpr (!kRowsInStage) prefetch(gi, nbase);
     const uint32_t step = static_cast<uint32_t>(CG) * gridDim.x;
     const int dh = static_cast<int>(step % static_cast<uint32_t>(H)), db = static_cast<int>(step / H);
     const uint32_t t0 = blockIdx.x + static_cast<uint32_t>(gi) * gridDim.x;
@@ -982,6 +996,14 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
         const int g = fdiv(h, lay.divHpg);
         const size_t bh = static_cast<size_t>(b) * H + h, bg = static_cast<size_t>(b) * G + g;
         const unsigned char* sp = smem + static_cast<size_t>(st) * lay.stage_bytes;
+        // rows with the stage: this call's scalars of the tile, loaded before
+        // the waits so that they arrive meanwhile (dt of token `lane`, A_h, D_h)
+        float dtl = 0.f, Ahr = 0.f, Dhr = 0.f;
+        if constexpr (kRowsInStage) {
+            dtl = lane < ntok ? a.dt[(static_cast<size_t>(b) * ntok + lane) * H + h] : 0.f;
+            Ahr = a.A[h];
+            Dhr = a.D[h];
+        }
         int stop = 0;
         if (ctid == 0) {
             stop = s_abort;
@@ -1001,16 +1023,16 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                 mbar_wait_bounded(smem_u32(&full_bar[st]), use & 1, kWaitNs);  // copies in flight
             }
         }
-        cp_async_wait_all();  // this tile's rows
+        if constexpr (!kRowsInStage) cp_async_wait_all();  // this tile's rows
         // the stage and this tile's rows have landed; this group's previous
         // readers of s_w / s_g and of the row buffers are done
         if (group_sync_or(gi, CT, stop)) break;
         // the next tile's rows, into the buffer the previous tile used (its
         // readers all passed the barrier above); they land while this tile works
-        prefetch(k + CG, nbase + ((it + 1) & 1) * lay.newrows);
+        if constexpr (!kRowsInStage) prefetch(k + CG, nbase + ((it + 1) & 1) * lay.newrows);
         bool released = false;  // the stage went back to the producer before the tile's end
-        const unsigned char* nr = nbase + (it & 1) * lay.newrows;
-        const float* sc4 = reinterpret_cast<const float*>(nr + lay.nd_off);  // dt [8], A, D
+        const unsigned char* nr = kRowsInStage ? sp + lay.rows : nbase + (it & 1) * lay.newrows;
+        const float* sc4 = reinterpret_cast<const float*>(nr + lay.nd_off);  // row buffers: dt [8], A, D
         const int pos = reinterpret_cast<const int*>(sp + lay.meta)[kMetaPos];
         const int T = pos + ntok;
         const bool ok = pos >= 0 && T <= cap;
@@ -1061,11 +1083,16 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
             }
             if (cw == CW - 1) {
                 const float* dtrow = reinterpret_cast<const float*>(sp + a.rec.dt);
-                const float dnew = (lane >= pos && lane < T) ? sc4[lane - pos] : 0.f;
+                float dnv;
+                if constexpr (kRowsInStage)
+                    dnv = __shfl_sync(0xffffffffu, dtl, (lane - pos) & 31);
+                else
+                    dnv = (lane >= pos && lane < T) ? sc4[lane - pos] : 0.f;
+                const float dnew = (lane >= pos && lane < T) ? dnv : 0.f;
                 const float dts = (lane < pos) ? dtrow[lane] : dnew;
                 if (lane >= pos && lane < T) reinterpret_cast<float*>(rec + a.rec.dt)[lane] = dnew;
                 const float Sx = warp_prefix(dts);
-                const float Ah = sc4[kMaxTok];
+                const float Ah = kRowsInStage ? Ahr : sc4[kMaxTok];
 #pragma unroll
                 for (int j = 0; j < NT; ++j) {
                     if (j < ntok) {
@@ -1103,7 +1130,7 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
         if (ok && !(FUSED && T == a.s.L)) {
             const unsigned char* tile = sp;
             const unsigned char* sc = sp + a.rec.scales;
-            const float Dh = sc4[kMaxTok + 1];
+            const float Dh = kRowsInStage ? Dhr : sc4[kMaxTok + 1];
             float* yout = a.y + static_cast<size_t>(b) * ntok * HP + static_cast<size_t>(h) * P;
             const TIn* xrow = (lane < pos) ? xr + lane * P : nx + (lane - pos) * P;  // slot `lane`
             // partials of rows r0..r0+7 for token j: lane l holds columns 4l..4l+3
@@ -1176,7 +1203,8 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                     group_sync(gi, CT);
                 // rows R0 + g, R0 + g + 8: scale the two block sums, add the row's
                 // four lanes, then the replay term and D x
-                auto finish = [&](int R0, const float (&d)[4], uint32_t s2a, uint32_t s2b) {
+                // (xa, xb: this call's x of the two rows)
+                auto finish = [&](int R0, const float (&d)[4], uint32_t s2a, uint32_t s2b, float xa, float xb) {
                     const int ra = R0 + g, rb = ra + 8;
                     const float2 sa = h2_f2(s2a), sb = h2_f2(s2b);
                     float pa = fmaf(sa.x, d[0], sa.y * d[1]);
@@ -1186,18 +1214,19 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                     pa += __shfl_xor_sync(0xffffffffu, pa, 2);
                     pb += __shfl_xor_sync(0xffffffffu, pb, 2);
                     if (t == 0) {
-                        if (ra < P) yout[ra] = fmaf(Dh, to_f32(nx[ra]), fmaf(dec, pa, rep[ra]));
-                        if (rb < P) yout[rb] = fmaf(Dh, to_f32(nx[rb]), fmaf(dec, pb, rep[rb]));
+                        if (ra < P) yout[ra] = fmaf(Dh, xa, fmaf(dec, pa, rep[ra]));
+                        if (rb < P) yout[rb] = fmaf(Dh, xb, fmaf(dec, pb, rep[rb]));
                     }
                 };
                 auto scales2 = [&](int r) -> uint32_t {  // e4m3 scales of blocks 2t, 2t + 1 of row r as f16
                     return r < P ? e4m3x2_h2(*reinterpret_cast<const uint16_t*>(sc + r * (N >> 4) + 2 * t)) : 0u;
                 };
                 if (CW == 1 && P <= 64) {
-                    // the lane's codes and scales of every row group into registers,
-                    // then the stage goes back to the producer before the products
+                    // the lane's codes, scales and x (this call's, of its rows) of
+                    // every row group into registers, then the stage goes back to
+                    // the producer before the products
                     uint4 qa[4], qb[4];
-                    uint32_t s2a[4], s2b[4];
+                    uint32_t s2a[4], s2b[4], xab[4];
 #pragma unroll
                     for (int rg = 0; rg < 4; ++rg) {
                         const int ra = 16 * rg + g, rb = ra + 8;
@@ -1206,6 +1235,8 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                         qb[rg] = rb < P ? *reinterpret_cast<const uint4*>(tile + rb * (kD128 / 2) + 16 * t) : z;
                         s2a[rg] = scales2(ra);
                         s2b[rg] = scales2(rb);
+                        const uint16_t* xw = reinterpret_cast<const uint16_t*>(nx);
+                        xab[rg] = (ra < P ? xw[ra] : 0u) | ((rb < P ? static_cast<uint32_t>(xw[rb]) : 0u) << 16);
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
@@ -1215,14 +1246,17 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                         if (16 * rg < P) {
                             float d[4] = {0.f, 0.f, 0.f, 0.f};
                             fp4_codes_mma(qa[rg], qb[rg], bf, d);
-                            finish(16 * rg, d, s2a[rg], s2b[rg]);
+                            finish(16 * rg, d, s2a[rg], s2b[rg], __uint_as_float(xab[rg] << 16),
+                                   __uint_as_float(xab[rg] & 0xFFFF0000u));
                         }
                     }
                 } else {
                     for (int R0 = 16 * cw; R0 < P; R0 += 16 * CW) {
                         float d[4] = {0.f, 0.f, 0.f, 0.f};
                         hc_mma<kFP4, false>(tile, sc, R0, P, bf, d);
-                        finish(R0, d, scales2(R0 + g), scales2(R0 + g + 8));
+                        const int ra = R0 + g, rb = ra + 8;
+                        finish(R0, d, scales2(ra), scales2(rb), ra < P ? to_f32(nx[ra]) : 0.f,
+                               rb < P ? to_f32(nx[rb]) : 0.f);
                     }
                 }
             } else if constexpr (kMma) {
@@ -2493,17 +2527,25 @@ RecLayout record_layout(const Shape& s, int rf, int in_bytes) {
 
 // Stage layout of k_replay_pipe (16-byte aligned pieces, 128-byte aligned
 // stages and row buffers); the stages fill what the row buffers leave.
+// rows_in_stage: this call's rows travel with the stage (no row buffers).
 PipeLayout pipe_layout(const Shape& s, const RecLayout& rec, int ntok, int in_bf16, int groups, int fused,
-                       size_t smem_budget) {
+                       size_t smem_budget, int rows_in_stage) {
     const uint32_t es = in_bf16 ? 2u : 4u;
     PipeLayout L;
     L.brows = align16(rec.x + static_cast<uint32_t>(s.cap * s.P) * es);
     L.meta = L.brows + align16(static_cast<uint32_t>(s.cap * s.N) * es);
-    L.stage_bytes = (L.meta + 64u + 127u) & ~127u;
     L.nb_off = align16(static_cast<uint32_t>(ntok * s.P) * es);
     L.nc_off = L.nb_off + align16(static_cast<uint32_t>(ntok * s.N) * es);
     L.nd_off = L.nc_off + align16(static_cast<uint32_t>(ntok * s.N) * es);
-    L.newrows = (L.nd_off + 4u * (kMaxTok + 2) + 127u) & ~127u;
+    if (rows_in_stage) {
+        L.rows = L.meta + 64u;
+        L.stage_bytes = (L.rows + L.nc_off + static_cast<uint32_t>(ntok * s.N) * es + 127u) & ~127u;
+        L.newrows = 0u;
+    } else {
+        L.rows = 0u;
+        L.stage_bytes = (L.meta + 64u + 127u) & ~127u;
+        L.newrows = (L.nd_off + 4u * (kMaxTok + 2) + 127u) & ~127u;
+    }
     L.xw_bytes = fused ? (4u * static_cast<uint32_t>(s.cap * s.P) + 127u) & ~127u : 0u;
     const size_t rows = static_cast<size_t>(groups) * (2u * L.newrows + L.xw_bytes);
     const size_t n = smem_budget > rows ? (smem_budget - rows) / L.stage_bytes : 0;
@@ -2586,7 +2628,8 @@ cudaError_t launch_replay(const ReplayArgs& a, int in_bf16, int rf, cudaStream_t
             const size_t stat = pipe_static_smem(nt, rf);
             const size_t budget = di.smem_optin > stat ? di.smem_optin - stat : 0;
             const int groups = pipe_groups(nt, rf);
-            const PipeLayout L = pipe_layout(a.s, a.rec, a.ntok, in_bf16, groups, a.fused, budget);
+            const PipeLayout L = pipe_layout(a.s, a.rec, a.ntok, in_bf16, groups, a.fused, budget,
+                                             pipe_rows_in_stage(a.ntok, rf, a.fused));
             if (L.stages >= 2) {
                 const int ntiles = a.s.batch * a.s.H;
                 const int grid = ntiles < di.sms ? ntiles : di.sms;
