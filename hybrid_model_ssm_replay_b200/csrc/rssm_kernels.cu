@@ -935,6 +935,7 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
     // this call's rows of tile kk -> buf: [ntok][P] x, [ntok][N] B, [ntok][N] C in
     // 16-byte chunks, then the scalars dt [ntok], A_h, D_h at nd_off
     const int xc = (P * es) >> 4, bc = (N * es) >> 4, per_tok = xc + 2 * bc;
+    const float inv_xc = 1.0f / static_cast<float>(xc);
     auto prefetch = [&](int kk, unsigned char* buf) {
         const uint32_t t = blockIdx.x + static_cast<uint32_t>(kk) * gridDim.x;
         if (t < static_cast<uint32_t>(ntiles)) {
@@ -946,9 +947,32 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                 static_cast<const TIn*>(a.B) + b0 * GN + static_cast<size_t>(g) * N);
             const unsigned char* cs = reinterpret_cast<const unsigned char*>(
                 static_cast<const TIn*>(a.C) + b0 * GN + static_cast<size_t>(g) * N);
-            for (int j = 0; j < ntok; ++j) {
+            if constexpr (NT > 1) {
+                // verify: all tokens' chunks in one branch-free sweep, so a warp
+                // issues its copies in one or two instructions: chunks [0, ntok xc)
+                // are the x rows, then ntok bc of B rows, then ntok bc of C rows
+                const int nxc = ntok * xc, nbc = ntok * bc;
+                const int bsh = bc == 16 ? 4 : 5;  // bc = 128 es / 16
+                for (int c = ctid; c < nxc + 2 * nbc; c += CT) {
+                    const bool isx = c < nxc;
+                    const int cb = c - nxc;
+                    const bool isb = !isx && cb < nbc;
+                    const int cc = isb ? cb : cb - nbc;
+                    const int jx = static_cast<int>((static_cast<float>(c) + 0.5f) * inv_xc);  // c / xc, exact (c < 2^10)
+                    const int j = isx ? jx : (cc >> bsh), q = isx ? c - jx * xc : (cc & (bc - 1));
+                    const unsigned char* src = isx ? xs + static_cast<size_t>(j) * HP * es
+                                                   : (isb ? bs : cs) + static_cast<size_t>(j) * GN * es;
+                    const uint32_t dof = isx ? static_cast<uint32_t>(j * P * es)
+                                             : (isb ? lay.nb_off : lay.nc_off) + static_cast<uint32_t>(j * N * es);
+                    cp_async16(smem_u32(buf) + dof + 16u * q, src + 16 * q);
+                }
+            }
+            for (int j = 0; NT == 1 && j < ntok; ++j) {
                 // token j: x row (xc chunks of 16 B), B row (bc), C row (bc)
-                for (int r = ctid; r < per_tok; r += CT) {
+                // (decode: the group's last threads take the chunks, so that its
+                // first warps start the B.C products at once; measured faster
+                // for decode, slower for verify)
+                for (int r = CT - 1 - ctid; r < per_tok; r += CT) {
                     const unsigned char* src;
                     uint32_t dst;
                     if (r < xc) {
@@ -2075,7 +2099,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_prefill(const PrefillArgs a) {
 // One CTA of 8 warps per tile walks the prompt in chunks of 64 tokens from
 // the last to the first, so R_t is a running suffix sum (no cancellation).
 // Per chunk: the x rows, B rows and dt land by cp.async (double-buffered,
-// the next chunk while this one computes); warp 0 forms w_t; all threads
+// the next chunk while this one computes); every warp forms the chunk's w_t
+// itself (the same arithmetic in each, so no barrier waits on it); all threads
 // split w_t x_t[p] into bf16 hi + lo parts (x_w carries ~16 bits; B is bf16,
 // exact); warp w accumulates rows 16 (w % 4).. of the product against the
 // 64 columns 64 (w / 4).. with mma.sync bf16 m16n8k16, operands from shared
@@ -2087,7 +2112,7 @@ constexpr uint32_t kPfX = kPfChunk * 64 * 2;                 // x rows [64][64] 
 constexpr uint32_t kPfB = kPfChunk * kD128 * 2;              // B rows [64][128] bf16 (swizzled)
 constexpr uint32_t kPfBuf = kPfX + kPfB + kPfChunk * 4;      // + dt [64]
 constexpr uint32_t kPfA = kPfChunk * 64 * 2;                 // x_w hi or lo [64 tokens][64 rows] (swizzled)
-constexpr size_t kPfSmem = 2 * static_cast<size_t>(kPfBuf) + 2 * kPfA + kPfChunk * 4;
+constexpr size_t kPfSmem = 2 * static_cast<size_t>(kPfBuf) + 2 * kPfA;
 
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16u : 0u)
@@ -2098,7 +2123,7 @@ __device__ __forceinline__ void cp_async4_zfill(uint32_t dst, const void* src, b
                  : "memory");
 }
 
-__global__ void __launch_bounds__(kPfThreads, 2) k_prefill_mma(const PrefillArgs a) {
+__global__ void __launch_bounds__(kPfThreads, 3) k_prefill_mma(const PrefillArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int s_pos;
     const int H = a.s.H, P = a.s.P, G = a.s.G, batch = a.s.batch, T0 = a.T0;
@@ -2107,7 +2132,6 @@ __global__ void __launch_bounds__(kPfThreads, 2) k_prefill_mma(const PrefillArgs
     unsigned char* rec = a.record + (static_cast<size_t>(b) * H + h) * a.rec.bytes;
     unsigned char* aw_hi = smem + 2 * kPfBuf;
     unsigned char* aw_lo = aw_hi + kPfA;
-    float* s_wt = reinterpret_cast<float*>(aw_lo + kPfA);
 
     if (tid == 0) s_pos = a.pos[b];  // the only read of pos
     __syncthreads();
@@ -2167,8 +2191,9 @@ __global__ void __launch_bounds__(kPfThreads, 2) k_prefill_mma(const PrefillArgs
         cp_async_wait_all();
         __syncthreads();  // chunk c landed; the previous chunk's readers are done
         if (c > 0) fetch(c - 1, buf ^ 1);
-        if (warp == 0) {
-            // w_t = dt_t exp(A R_t): lane l takes tokens l and l + 32 of the chunk
+        {
+            // w_t = dt_t exp(A R_t), formed by every warp alike (no barrier):
+            // lane l takes tokens l and l + 32 of the chunk
             const float* dts = reinterpret_cast<const float*>(base + kPfX + kPfB);
             const float v0 = dts[lane], v1 = dts[lane + 32];
             float s0 = v0, s1 = v1;  // inclusive suffix sums within each half
@@ -2183,15 +2208,13 @@ __global__ void __launch_bounds__(kPfThreads, 2) k_prefill_mma(const PrefillArgs
             }
             const float tot1 = __shfl_sync(0xffffffffu, s1, 0), tot0 = __shfl_sync(0xffffffffu, s0, 0);
             // R_t = (later chunks) + (later tokens of this chunk), exclusive of t
-            s_wt[lane + 32] = v1 * expf(Ah * (carry + (s1 - v1)));
-            s_wt[lane] = v0 * expf(Ah * ((carry + tot1) + (s0 - v0)));
+            const float w1 = v1 * expf(Ah * (carry + (s1 - v1)));
+            const float w0 = v0 * expf(Ah * ((carry + tot1) + (s0 - v0)));
             carry = (carry + tot1) + tot0;
-        }
-        __syncthreads();  // weights ready
-        {
             // x_w = w_t x_t[p] as bf16 hi + lo: thread -> token tid / 4, rows 16 (tid % 4) ..
             const int k = tid >> 2, p0 = 16 * (tid & 3);
-            const float w = s_wt[k];
+            const float wa = __shfl_sync(0xffffffffu, w0, k & 31), wb = __shfl_sync(0xffffffffu, w1, k & 31);
+            const float w = k < 32 ? wa : wb;  // uniform over the warp
             uint32_t hi[8], lo[8];
             if (p0 < P) {
                 const uint4 u0 = *reinterpret_cast<const uint4*>(base + k * 128 + 2 * p0);
@@ -2243,10 +2266,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) k_prefill_mma(const PrefillArgs
             }
         }
     }
-    // h_T = exp(A S) h_0 + acc, S = the prompt's dt sum (warp 0's carry)
-    if (warp == 0 && lane == 0) s_wt[0] = expf(Ah * carry);
-    __syncthreads();
-    const float alpha = s_wt[0];
+    // h_T = exp(A S) h_0 + acc, S = the prompt's dt sum (each warp's carry)
+    const float alpha = expf(Ah * carry);
     if (rows_live) {
         const int gq = lane >> 2, tq = lane & 3;
         float* hrow = reinterpret_cast<float*>(rec);
