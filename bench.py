@@ -310,21 +310,33 @@ def run_ours(args):
                                  "vs_separate_flush": fz_value / value}
             del fz
             torch.cuda.empty_cache()
-        out["large_b512"] = large_leg(rssm, torch, WORKLOADS["large_b512"], max(2, min(K, 50)), W, dev, barrier,
-                                      max_over_ranks, world, peak, args.fused)
-        torch.cuda.empty_cache()
-        out["spec_b512_k4"] = spec_leg(rssm, torch, WORKLOADS["spec_b512_k4"], max(2, min(K, 32)), W, dev, barrier,
-                                       max_over_ranks, world, peak)
-        torch.cuda.empty_cache()
-        out["split_b256"] = split_leg(rssm, torch, WORKLOADS["split_b256"], max(2, min(K, 50)), W, dev, barrier,
-                                      max_over_ranks, world, peak)
-        torch.cuda.empty_cache()
-        out["prefill_b256"] = prefill_leg(rssm, torch, WORKLOADS["small_b256"], dev, barrier, max_over_ranks, world)
-        torch.cuda.empty_cache()
-        out["batch_sweep_large"] = sweep_leg(rssm, torch, WORKLOADS["large_b512"], max(2, min(K, 20)), W, dev,
-                                             barrier, max_over_ranks, world, peak)
-        torch.cuda.empty_cache()
-        out["stage_b256"] = stage_leg(rssm, torch, max(2, min(K, 10)), W, dev, barrier, max_over_ranks, world)
+        gpu_id = smi_gpu_id(torch, dev.index if dev.index is not None else 0)
+
+        def clocked(fn, *fargs):
+            # the leg's result with the SM clock and throttle reasons sampled while it ran
+            sampler = ClockSampler(gpu_id)
+            sampler.start()
+            t0 = time.time()
+            res = fn(*fargs)
+            t1 = time.time()
+            time.sleep(0.06)
+            sampler.stop()
+            res["clocks"] = sampler.summary(t0, t1)
+            torch.cuda.empty_cache()
+            return res
+
+        out["large_b512"] = clocked(large_leg, rssm, torch, WORKLOADS["large_b512"], max(2, min(K, 50)), W, dev,
+                                    barrier, max_over_ranks, world, peak, args.fused)
+        out["spec_b512_k4"] = clocked(spec_leg, rssm, torch, WORKLOADS["spec_b512_k4"], max(2, min(K, 32)), W, dev,
+                                      barrier, max_over_ranks, world, peak)
+        out["split_b256"] = clocked(split_leg, rssm, torch, WORKLOADS["split_b256"], max(2, min(K, 50)), W, dev,
+                                    barrier, max_over_ranks, world, peak)
+        out["prefill_b256"] = clocked(prefill_leg, rssm, torch, WORKLOADS["small_b256"], dev, barrier,
+                                      max_over_ranks, world)
+        out["batch_sweep_large"] = clocked(sweep_leg, rssm, torch, WORKLOADS["large_b512"], max(2, min(K, 20)), W,
+                                           dev, barrier, max_over_ranks, world, peak)
+        out["stage_b256"] = clocked(stage_leg, rssm, torch, max(2, min(K, 10)), W, dev, barrier, max_over_ranks,
+                                    world)
     if rank == 0 and world == 1 and not args.no_extra:
         out["cpu_baseline"] = cpu_baseline()
     if world > 1:
