@@ -547,12 +547,16 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // memory: three groups of four warps. Verify (K+1 tokens per tile) takes
 // three groups of four warps for every copy (two groups for more than kMidTok
 // tokens, whose registers would spill). Decode of the smaller copies has room
-// for many tiles: bf16 six groups of two warps; e4m3 and FP4 twelve groups of
-// one warp, each tile worked by one warp without group barriers. (B200: FP4
-// decode 102 us with 6 x 2, 93 us with 12 x 1, 114 us with 8 x 1; FP4 verify
+// for many tiles: bf16 seven groups of two warps; e4m3 and FP4 fifteen groups
+// of one warp, each tile worked by one warp without group barriers. Fifteen
+// consumer warps + the producer are 16 warps, the block size at which the
+// register budget stays 128 per thread (13 warps get the same), and group
+// 14 uses the last named barrier (15). (B200, FP4 decode: 93 us with 12 x 1,
+// 102 us with 6 x 2, 114 us with 8 x 1 in the first form of the kernel;
+// 43.1 -> 40.2 us from 12 x 1 to 15 x 1 in the current one; FP4 verify
 // 1163 us with 12 x 1, 934 us with 3 x 4.)
 __host__ __device__ constexpr int pipe_groups(int nt, int rf) {
-    return nt > 1 ? (nt <= kMidTok ? 3 : 2) : (rf == kF32 ? 3 : (rf == kBF16 ? 6 : 12));
+    return nt > 1 ? (nt <= kMidTok ? 3 : 2) : (rf == kF32 ? 3 : (rf == kBF16 ? 7 : 15));
 }
 __host__ __device__ constexpr int pipe_cwarps(int nt, int rf) {
     return nt > 1 ? 4 : (rf == kF32 ? 4 : (rf == kBF16 ? 2 : 1));
