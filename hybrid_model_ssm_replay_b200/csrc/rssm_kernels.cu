@@ -953,11 +953,14 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                 static_cast<const TIn*>(a.C) + b0 * GN + static_cast<size_t>(g) * N);
             if constexpr (NT > 1) {
                 // verify: all tokens' chunks in one branch-free sweep, so a warp
-                // issues its copies in one or two instructions: chunks [0, ntok xc)
-                // are the x rows, then ntok bc of B rows, then ntok bc of C rows
+                // issues its copies in a few instructions: chunks [0, ntok xc)
+                // are the x rows, then ntok bc of B rows, then ntok bc of C rows.
+                // Warps 1 and 2 issue them (warp 0 starts the B.C products at
+                // once, warp CW-1 forms the weights): verify 571 -> 538 us.
                 const int nxc = ntok * xc, nbc = ntok * bc;
                 const int bsh = bc == 16 ? 4 : 5;  // bc = 128 es / 16
-                for (int c = ctid; c < nxc + 2 * nbc; c += CT) {
+                constexpr int pf0 = CW > 2 ? 32 : 0, pfn = CW > 2 ? 64 : CT;
+                for (int c = ctid - pf0; ctid >= pf0 && ctid < pf0 + pfn && c < nxc + 2 * nbc; c += pfn) {
                     const bool isx = c < nxc;
                     const int cb = c - nxc;
                     const bool isb = !isx && cb < nbc;
