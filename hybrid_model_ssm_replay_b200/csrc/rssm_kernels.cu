@@ -938,7 +938,7 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                                            static_cast<size_t>(gi) * lay.xw_bytes);
     // this call's rows of tile kk -> buf: [ntok][P] x, [ntok][N] B, [ntok][N] C in
     // 16-byte chunks, then the scalars dt [ntok], A_h, D_h at nd_off
-    const int xc = (P * es) >> 4, bc = (N * es) >> 4, per_tok = xc + 2 * bc;
+    const int xc = (P * es) >> 4, bc = (N * es) >> 4;  // 16-byte chunks of an x row, of a B or C row
     const float inv_xc = 1.0f / static_cast<float>(xc);
     auto prefetch = [&](int kk, unsigned char* buf) {
         const uint32_t t = blockIdx.x + static_cast<uint32_t>(kk) * gridDim.x;
@@ -951,12 +951,13 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                 static_cast<const TIn*>(a.B) + b0 * GN + static_cast<size_t>(g) * N);
             const unsigned char* cs = reinterpret_cast<const unsigned char*>(
                 static_cast<const TIn*>(a.C) + b0 * GN + static_cast<size_t>(g) * N);
-            if constexpr (NT > 1) {
-                // verify: all tokens' chunks in one branch-free sweep, so a warp
-                // issues its copies in a few instructions: chunks [0, ntok xc)
-                // are the x rows, then ntok bc of B rows, then ntok bc of C rows.
-                // Warps 1 and 2 issue them (warp 0 starts the B.C products at
-                // once, warp CW-1 forms the weights): verify 571 -> 538 us.
+            // every token's chunks in one branch-free sweep, so a warp issues
+            // its copies in a few instructions: chunks [0, ntok xc) are the x
+            // rows, then ntok bc of B rows, then ntok bc of C rows. Warps 1 and
+            // 2 issue them (warp 0 starts the B.C products at once, warp CW-1
+            // forms the weights): verify 571 -> 538 us; one divergent cp.async
+            // per row kind and token had taken ~2,200 cycles per tile.
+            {
                 const int nxc = ntok * xc, nbc = ntok * bc;
                 const int bsh = bc == 16 ? 4 : 5;  // bc = 128 es / 16
                 constexpr int pf0 = CW > 2 ? 32 : 0, pfn = CW > 2 ? 64 : CT;
@@ -973,30 +974,6 @@ __global__ void __launch_bounds__(pipe_threads(NT, RF), 1) k_replay_pipe(const R
                                              : (isb ? lay.nb_off : lay.nc_off) + static_cast<uint32_t>(j * N * es);
                     cp_async16(smem_u32(buf) + dof + 16u * q, src + 16 * q);
                 }
-            }
-            for (int j = 0; NT == 1 && j < ntok; ++j) {
-                // token j: x row (xc chunks of 16 B), B row (bc), C row (bc)
-                // (decode: the group's last threads take the chunks, so that its
-                // first warps start the B.C products at once; measured faster
-                // for decode, slower for verify)
-                for (int r = CT - 1 - ctid; r < per_tok; r += CT) {
-                    const unsigned char* src;
-                    uint32_t dst;
-                    if (r < xc) {
-                        src = xs + 16 * r;
-                        dst = smem_u32(buf + j * P * es) + 16u * r;
-                    } else if (r < xc + bc) {
-                        src = bs + 16 * (r - xc);
-                        dst = smem_u32(buf + lay.nb_off + j * N * es) + 16u * (r - xc);
-                    } else {
-                        src = cs + 16 * (r - xc - bc);
-                        dst = smem_u32(buf + lay.nc_off + j * N * es) + 16u * (r - xc - bc);
-                    }
-                    cp_async16(dst, src);
-                }
-                xs += HP * es;
-                bs += GN * es;
-                cs += GN * es;
             }
             if (ctid < ntok + 2) {  // scalars, 4 bytes each: dt of each token, A_h, D_h
                 const int i = ctid;
