@@ -882,7 +882,8 @@ def split_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
     """Precision split (s4) on the small layer: 16 decodes reading the FP4
     output copy + one refresh of the bf16 (or e4m3) update copy with Philox
     SR, and the shared-copy controls (one FP4 copy, or one bf16 copy with SR,
-    read and updated)."""
+    read and updated). Timed like the headline loop: CUDA graphs of the 16
+    decodes and of the refresh, CUDA events between them."""
     from hybrid_model_ssm_replay_b200.inputs import make_inputs
     shape = wl["shape"]
     L = shape.interval
@@ -916,38 +917,45 @@ def split_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
             st.ckpt.copy_(inp["ckpt"].to(torch.bfloat16 if upd == rssm.RSSM_BF16 else torch.float8_e4m3fn)
                           .view(st.ckpt.dtype))
             rssm.rssm_lowprec_refresh(st, inp["A"], force=True)
-        ev_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K * L)]
-        ev_r = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-
-        def step(k, timed):
+        def decodes():
             for i in range(L):
-                if timed:
-                    ev_d[k * L + i][0].record()
                 rssm.rssm_decode_step(st, inp["x"][i], inp["B"][i], inp["C"][i], inp["dt"][i], inp["A"], inp["D"], y)
-                if timed:
-                    ev_d[k * L + i][1].record()
-            if timed:
-                ev_r[k][0].record()
-            rssm.rssm_lowprec_refresh(st, inp["A"])
-            if timed:
-                ev_r[k][1].record()
 
+        def refresh():
+            rssm.rssm_lowprec_refresh(st, inp["A"])
+
+        # eager warm-up, then the interval as two CUDA graphs (the 16 decodes,
+        # the refresh) replayed with events between them, as the headline loop
         for k in range(W):
-            step(k, False)
+            decodes()
+            refresh()
+        torch.cuda.synchronize()
+        g_dec, g_ref = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_dec):
+            decodes()
+        with torch.cuda.graph(g_ref):
+            refresh()
+        for k in range(W):
+            g_dec.replay()
+            g_ref.replay()
         torch.cuda.synchronize()
         barrier()
-        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
+        stream = torch.cuda.current_stream()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * K + 1)]
         for k in range(K):
-            step(k, True)
-        e.record()
+            ev[2 * k].record(stream)
+            g_dec.replay()
+            ev[2 * k + 1].record(stream)
+            g_ref.replay()
+        ev[2 * K].record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms = max_over_ranks(a.elapsed_time(e))
+        ms = max_over_ranks(ev[0].elapsed_time(ev[2 * K]))
         if rssm.rssm_get_error(st) != 0:
             raise RuntimeError("device error in the precision-split leg")
-        d_us = statistics.mean(x.elapsed_time(z) for x, z in ev_d) * 1e3
-        r_us = statistics.mean(x.elapsed_time(z) for x, z in ev_r) * 1e3
+        del g_dec, g_ref
+        d_us = sum(ev[2 * k].elapsed_time(ev[2 * k + 1]) for k in range(K)) / (K * L) * 1e3
+        r_us = sum(ev[2 * k + 1].elapsed_time(ev[2 * k + 2]) for k in range(K)) / K * 1e3
         dec_bytes = (rd_bytes + tok_other) * shape.batch
         ref_bytes = (2 * upd_bytes + out_bytes + L * b["entry"]) * shape.batch
         out[name] = {"tokens_per_s": world * shape.batch * L * K / (ms / 1e3), "decode_avg_launch_us": d_us,
