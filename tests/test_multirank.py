@@ -48,7 +48,7 @@ def test_single_rank_identity():
 
 
 def test_reference_arm_under_torchrun_prints_one_line():
-    """bench.py --impl reference launched as the driver launches it for N > 1
+    """bench.py --impl reference launched under torchrun for N > 1
     (torchrun, two ranks): rank 0 alone runs the oracle and prints the one
     JSON line; the other rank exits 0 without work."""
     import json
