@@ -190,6 +190,52 @@ def test_fp4_decode_and_refresh_match_oracle(kind, in_dtype, shape):
     assert st.flush_count.cpu().tolist() == [2] * Bz
 
 
+@pytest.mark.parametrize("kind", ["bf16", "e4m3"])
+def test_split_b256_full_size_sampled(kind):
+    """The precision split at the bench's size and launch configuration
+    (split_b256: batch 256, 64 heads, head_dim 64, d_state 128; the
+    persistent replay and fold kernels over every SM): one interval of 16
+    decodes reading the FP4 output copy, then the refresh. For sampled
+    requests, the outputs match the oracle replaying the same dequantised
+    copy; the refreshed update copy and FP4 copy equal, bit for bit, the
+    oracle's stochastic rounding and FP4 quantisation of the fold an fp32
+    twin computed; and that fold matches the oracle's fp64 fold."""
+    w = WORKLOADS["split_b256"]
+    shape = w["shape"]
+    L = shape.interval
+    Bz, H, P = shape.batch, shape.nheads, shape.head_dim
+    inp = make_inputs(shape, L, w["seed"], w["in_dtype"], device="cuda")
+    seed = w["seed"]
+    desc, st = split_state(shape, inp, kind, seed)
+    _, tw = f32_twin(shape, widened(kind, st), seed)
+    rssm.rssm_lowprec_refresh(tw, inp["A"], force=True)
+    y = torch.empty((L, Bz, H, P), device="cuda")
+    y2 = torch.empty_like(y)
+    for t in range(L):
+        args = (inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"])
+        rssm.rssm_decode_step(st, *args, y[t])
+        rssm.rssm_decode_step(tw, *args, y2[t])
+    fc_before = st.flush_count.cpu().tolist()
+    rssm.rssm_lowprec_refresh(st, inp["A"])
+    rssm.rssm_lowprec_refresh(tw, inp["A"])
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
+    assert torch.equal(y, y2)                       # both read the same FP4 copy
+    reqs = sample_requests(Bz, 6)
+    assert_refresh_bits(kind, seed, st, tw, fc_before, reqs, f"{kind} + FP4 refresh at split_b256")
+    for b in reqs:
+        upd0 = copy_bits(initial_update_copy(inp["ckpt"][b], kind))
+        codes0, scales0 = orc.fp4_quant(orc.widen(UPD[kind][1], upd0, None, upd0.shape).astype(np.float32))
+        r = request_inputs(inp, b)
+        req = orc.LowPrecRequest(UPD[kind][1], True, upd0, codes0, scales0, shape.ngroups, L, r["A"], r["D"],
+                                 seed, b)
+        req.flush_count.value = 1
+        ys = np.stack([req.decode(r["x"][t], r["B"][t], r["C"][t], r["dt"][t]) for t in range(L)])
+        assert_close(to_np(y[:, b]), ys, f"FP4-copy decode at split_b256, request {b}")
+        v64 = req.refresh(want_v32=True).astype(np.float64)
+        assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of the refresh at split_b256, request {b}")
+    assert st.flush_count.cpu().tolist() == [2] * Bz
+
+
 # accepted drafts per step and request (steps x batch) for K = 4 and K = 6:
 # three requests reach the interval on the last step, one does not
 SPLIT_SPEC = {
