@@ -1001,11 +1001,11 @@ def prefill_leg(rssm, torch, wl, dev, barrier, max_over_ranks, world, T0=512, re
     flops = 2.0 * H * P * N * T0 * shape.batch
     return {"workload": f"small_b256 shapes, prompt of {T0} tokens per request", "prompt_tokens_per_s":
             world * shape.batch * T0 / (ms / 1e3), "ms_per_prefill": ms,
-            "kernel": "k_prefill_mma (mma.sync bf16, x_w split hi + lo)",
+            "kernel": "k_prefill_mma (mma.sync bf16, x_w split hi + mid + lo)",
             "bound": "hbm", "algorithmic_bytes_per_request": req_bytes, "achieved_gbs": gbs, "peak": peak,
             "peak_source": peak_src, "frac": gbs / peak,
             "contraction_tflops": flops / (ms / 1e3) / 1e12,
-            "note": "fold flops = 2 H P N T0 per request; the hi + lo split issues twice that on the tensor cores"}
+            "note": "fold flops = 2 H P N T0 per request; the hi + mid + lo split issues three times that on the tensor cores"}
 
 
 # ---------------------------------------------------- the CPU oracle arm

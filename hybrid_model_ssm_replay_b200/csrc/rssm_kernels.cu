@@ -2085,8 +2085,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_prefill(const PrefillArgs a) {
 // Per chunk: the x rows, B rows and dt land by cp.async (double-buffered,
 // the next chunk while this one computes); every warp forms the chunk's w_t
 // itself (the same arithmetic in each, so no barrier waits on it); all threads
-// split w_t x_t[p] into bf16 hi + lo parts (x_w carries ~16 bits; B is bf16,
-// exact); warp w accumulates rows 16 (w % 4).. of the product against the
+// split w_t x_t[p] into bf16 hi + mid + lo parts (x_w to ~2^-27; B is bf16,
+// exact; a two-part split, ~2^-17, left the checkpoint of a 512-token prompt
+// 1.5e-4 of its rms from the recurrence); warp w accumulates rows 16 (w % 4)..
+// of the product against the
 // 64 columns 64 (w / 4).. with mma.sync bf16 m16n8k16, operands from shared
 // memory by ldmatrix (rows XOR-swizzled by 16-byte chunk, conflict-free).
 // ---------------------------------------------------------------------------
@@ -2095,8 +2097,8 @@ constexpr int kPfThreads = 256;
 constexpr uint32_t kPfX = kPfChunk * 64 * 2;                 // x rows [64][64] bf16
 constexpr uint32_t kPfB = kPfChunk * kD128 * 2;              // B rows [64][128] bf16 (swizzled)
 constexpr uint32_t kPfBuf = kPfX + kPfB + kPfChunk * 4;      // + dt [64]
-constexpr uint32_t kPfA = kPfChunk * 64 * 2;                 // x_w hi or lo [64 tokens][64 rows] (swizzled)
-constexpr size_t kPfSmem = 2 * static_cast<size_t>(kPfBuf) + 2 * kPfA;
+constexpr uint32_t kPfA = kPfChunk * 64 * 2;                 // x_w hi, mid or lo [64 tokens][64 rows] (swizzled)
+constexpr size_t kPfSmem = 2 * static_cast<size_t>(kPfBuf) + 3 * kPfA;
 
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16u : 0u)
@@ -2115,7 +2117,8 @@ __global__ void __launch_bounds__(kPfThreads, 3) k_prefill_mma(const PrefillArgs
     const int b = blockIdx.x / H, h = blockIdx.x - b * H, g = h / (H / G);
     unsigned char* rec = a.record + (static_cast<size_t>(b) * H + h) * a.rec.bytes;
     unsigned char* aw_hi = smem + 2 * kPfBuf;
-    unsigned char* aw_lo = aw_hi + kPfA;
+    unsigned char* aw_md = aw_hi + kPfA;
+    unsigned char* aw_lo = aw_md + kPfA;
 
     if (tid == 0) s_pos = a.pos[b];  // the only read of pos
     __syncthreads();
@@ -2195,11 +2198,11 @@ __global__ void __launch_bounds__(kPfThreads, 3) k_prefill_mma(const PrefillArgs
             const float w1 = v1 * expf(Ah * (carry + (s1 - v1)));
             const float w0 = v0 * expf(Ah * ((carry + tot1) + (s0 - v0)));
             carry = (carry + tot1) + tot0;
-            // x_w = w_t x_t[p] as bf16 hi + lo: thread -> token tid / 4, rows 16 (tid % 4) ..
+            // x_w = w_t x_t[p] as bf16 hi + mid + lo: thread -> token tid / 4, rows 16 (tid % 4) ..
             const int k = tid >> 2, p0 = 16 * (tid & 3);
             const float wa = __shfl_sync(0xffffffffu, w0, k & 31), wb = __shfl_sync(0xffffffffu, w1, k & 31);
             const float w = k < 32 ? wa : wb;  // uniform over the warp
-            uint32_t hi[8], lo[8];
+            uint32_t hi[8], md[8], lo[8];
             if (p0 < P) {
                 const uint4 u0 = *reinterpret_cast<const uint4*>(base + k * 128 + 2 * p0);
                 const uint4 u1 = *reinterpret_cast<const uint4*>(base + k * 128 + 2 * p0 + 16);
@@ -2210,19 +2213,27 @@ __global__ void __launch_bounds__(kPfThreads, 3) k_prefill_mma(const PrefillArgs
                     const float f1 = w * __uint_as_float(bf16hi_bits(xw[q]));
                     const uint32_t hh = f32x2_to_bf16x2(f0, f1);
                     hi[q] = hh;
-                    lo[q] = f32x2_to_bf16x2(f0 - __uint_as_float(bf16lo_bits(hh)), f1 - __uint_as_float(bf16hi_bits(hh)));
+                    // the residuals below hi, then below mid, are exact in fp32
+                    const float r0 = f0 - __uint_as_float(bf16lo_bits(hh)), r1 = f1 - __uint_as_float(bf16hi_bits(hh));
+                    const uint32_t mm = f32x2_to_bf16x2(r0, r1);
+                    md[q] = mm;
+                    lo[q] = f32x2_to_bf16x2(r0 - __uint_as_float(bf16lo_bits(mm)), r1 - __uint_as_float(bf16hi_bits(mm)));
                 }
             } else {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) hi[q] = lo[q] = 0u;
+                for (int q = 0; q < 8; ++q) hi[q] = md[q] = lo[q] = 0u;
             }
             const int c0 = p0 >> 3;  // 16-byte chunk of the row
             uint4* dh0 = reinterpret_cast<uint4*>(aw_hi + k * 128 + 16 * (c0 ^ (k & 7)));
             uint4* dh1 = reinterpret_cast<uint4*>(aw_hi + k * 128 + 16 * ((c0 + 1) ^ (k & 7)));
+            uint4* dm0 = reinterpret_cast<uint4*>(aw_md + k * 128 + 16 * (c0 ^ (k & 7)));
+            uint4* dm1 = reinterpret_cast<uint4*>(aw_md + k * 128 + 16 * ((c0 + 1) ^ (k & 7)));
             uint4* dl0 = reinterpret_cast<uint4*>(aw_lo + k * 128 + 16 * (c0 ^ (k & 7)));
             uint4* dl1 = reinterpret_cast<uint4*>(aw_lo + k * 128 + 16 * ((c0 + 1) ^ (k & 7)));
             *dh0 = make_uint4(hi[0], hi[1], hi[2], hi[3]);
             *dh1 = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+            *dm0 = make_uint4(md[0], md[1], md[2], md[3]);
+            *dm1 = make_uint4(md[4], md[5], md[6], md[7]);
             *dl0 = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             *dl1 = make_uint4(lo[4], lo[5], lo[6], lo[7]);
         }
@@ -2233,8 +2244,9 @@ __global__ void __launch_bounds__(kPfThreads, 3) k_prefill_mma(const PrefillArgs
             for (int ks = 0; ks < kPfChunk / 16; ++ks) {
                 // A (rows R0.., tokens 16 ks..): matrix j = (rows 8 (j & 1).., tokens 8 (j >> 1)..)
                 const int ka = 16 * ks + r + 8 * (j >> 1), pc = (R0 >> 3) + (j & 1);
-                uint32_t ah[4], al[4];
+                uint32_t ah[4], am[4], al[4];
                 ldsm_x4_trans(smem_u32(aw_hi + ka * 128 + 16 * (pc ^ (ka & 7))), ah[0], ah[1], ah[2], ah[3]);
+                ldsm_x4_trans(smem_u32(aw_md + ka * 128 + 16 * (pc ^ (ka & 7))), am[0], am[1], am[2], am[3]);
                 ldsm_x4_trans(smem_u32(aw_lo + ka * 128 + 16 * (pc ^ (ka & 7))), al[0], al[1], al[2], al[3]);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -2243,8 +2255,10 @@ __global__ void __launch_bounds__(kPfThreads, 3) k_prefill_mma(const PrefillArgs
                     uint32_t b0, b1, b2, b3;
                     ldsm_x4_trans(smem_u32(base + kPfX + kb * (kD128 * 2) + 16 * (ncn ^ (kb & 7))), b0, b1, b2, b3);
                     mma_bf16(acc[2 * q], ah[0], ah[1], ah[2], ah[3], b0, b1);
+                    mma_bf16(acc[2 * q], am[0], am[1], am[2], am[3], b0, b1);
                     mma_bf16(acc[2 * q], al[0], al[1], al[2], al[3], b0, b1);
                     mma_bf16(acc[2 * q + 1], ah[0], ah[1], ah[2], ah[3], b2, b3);
+                    mma_bf16(acc[2 * q + 1], am[0], am[1], am[2], am[3], b2, b3);
                     mma_bf16(acc[2 * q + 1], al[0], al[1], al[2], al[3], b2, b3);
                 }
             }

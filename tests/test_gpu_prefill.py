@@ -10,9 +10,9 @@ import pytest
 import torch
 
 from hybrid_model_ssm_replay_b200 import rssm
-from hybrid_model_ssm_replay_b200.inputs import LayerShape, make_inputs
+from hybrid_model_ssm_replay_b200.inputs import WORKLOADS, LayerShape, make_inputs
 
-from gpu_helpers import assert_close, desc_for, oracle_map, request_inputs, to_np
+from gpu_helpers import assert_close, desc_for, oracle_map, request_inputs, sample_requests, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +57,26 @@ def test_prefill_then_decode_matches_recurrence(shape, T0, in_dtype):
         assert_close(ck[b], snaps[T0 - 1], f"checkpoint after a {T0}-token prefill, request {b}")
         assert_close(to_np(y[:, b]), y_ref[T0:], f"decode after the prefill, request {b}")
     assert set(st.flush_count.cpu().tolist()) == {(steps - T0) // L}
+
+
+def test_prefill_b256_t512_sampled():
+    """The bench's prefill: small_b256 shapes (batch 256, 64 heads, head_dim
+    64, d_state 128, bf16 inputs), 512-token prompts, the tensor-core kernel
+    at its launch configuration; the checkpoint of sampled requests against
+    the fp64 recurrence."""
+    w = WORKLOADS["small_b256"]
+    shape, T0 = w["shape"], 512
+    inp = make_inputs(shape, T0, 43, torch.bfloat16, device="cuda")
+    st = rssm.RssmState(desc_for(shape))
+    st.ckpt.copy_(inp["ckpt"])
+    rssm.rssm_prefill(st, inp["x"], inp["B"], inp["dt"], inp["A"])
+    assert rssm.rssm_get_error(st) == 0
+    assert st.pos.cpu().tolist() == [0] * shape.batch
+    reqs = sample_requests(shape.batch, 6)
+    res = oracle_map([("conv", request_inputs(inp, b), [T0 - 1]) for b in reqs])
+    for b, (_, snaps) in zip(reqs, res):
+        assert_close(st.ckpt[b].double().cpu().numpy(), snaps[T0 - 1], f"checkpoint after a {T0}-token prefill, "
+                                                                        f"request {b}")
 
 
 def test_prefill_needs_an_empty_buffer_and_zero_tokens_change_nothing():
