@@ -303,6 +303,79 @@ def test_speculative_verify_on_split_state_matches_oracle(kind, K):
         assert np.array_equal(st.out_codes[b].cpu().numpy(), codes_start[b])
 
 
+def refresh_bits_of(kind, seed, b, fc, upd_bits, codes, scales, v32, what):
+    """As assert_refresh_bits, for one request's copies taken as arrays."""
+    if kind in ("bf16", "e4m3"):
+        for h in range(v32.shape[0]):
+            exp = orc.sr_head(UPD[kind][1], seed, b, h, int(fc), v32[h])
+            bad = int(np.count_nonzero(upd_bits[h].ravel() != exp.ravel()))
+            assert bad == 0, f"{what}: request {b} head {h}: {bad} update-copy elements differ"
+    c_exp, s_exp = orc.fp4_quant(v32)
+    assert int(np.count_nonzero(codes != c_exp)) == 0, f"{what}: request {b}: FP4 codes differ"
+    assert int(np.count_nonzero(scales != s_exp)) == 0, f"{what}: request {b}: FP4 scales differ"
+
+
+def test_spec_b512_k4_on_split_state_sampled():
+    """Speculative decoding on a split-precision state at the bench's size
+    (spec_b512_k4: batch 512, 128 heads, 64 x 128, K = 4, n ~ U{0..4}, bf16
+    update copy + FP4 output copy) and launch configuration: per step verify
+    + accept + refresh, with an fp32 twin running the same calls. For
+    sampled requests, every verify before the request's first refresh
+    matches the oracle; at that refresh the twin's fp32 fold matches the
+    oracle's fp64 fold and the refreshed copies equal the oracle's rounding
+    of the twin's fold bit for bit."""
+    from hybrid_model_ssm_replay_b200.inputs import accept_lengths
+    w = WORKLOADS["spec_b512_k4"]
+    shape = w["shape"]
+    K, L = shape.max_draft, shape.interval
+    steps, kind, seed = 6, "bf16", w["seed"]
+    inp = make_inputs(shape, steps, w["seed"], w["in_dtype"], device="cuda", ntok=K + 1)
+    n_acc = accept_lengths(steps, shape.batch, K, w["seed"], device="cuda")
+    n_host = n_acc.cpu().numpy()
+    desc, st = split_state(shape, inp, kind, seed)
+    _, tw = f32_twin(shape, widened(kind, st), seed)
+    rssm.rssm_lowprec_refresh(tw, inp["A"], force=True)
+    reqs = sample_requests(shape.batch, 6)
+    y = torch.empty((steps, shape.batch, K + 1, shape.nheads, shape.head_dim), device="cuda")
+    y2 = torch.empty_like(y)
+    snaps = []  # per step, after its refresh: the sampled requests' copies, twin fold and counts
+    fc_prev = st.flush_count.cpu().numpy().copy()
+    for s in range(steps):
+        args = (inp["x"][s], inp["B"][s], inp["C"][s], inp["dt"][s], inp["A"], inp["D"])
+        for state, out in ((st, y), (tw, y2)):
+            rssm.rssm_verify(state, K, *args, out[s])
+            rssm.rssm_accept(state, n_acc[s])
+            rssm.rssm_lowprec_refresh(state, inp["A"])
+        fc_now = st.flush_count.cpu().numpy().copy()
+        snaps.append({b: (copy_bits(st.ckpt[b]), st.out_codes[b].cpu().numpy(), st.out_scales[b].cpu().numpy(),
+                          tw.ckpt[b].cpu().numpy(), int(fc_prev[b]), int(fc_now[b])) for b in reqs})
+        fc_prev = fc_now
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
+    assert torch.equal(y, y2)
+    refreshed = 0
+    for b in reqs:
+        upd0 = copy_bits(initial_update_copy(inp["ckpt"][b], kind))
+        codes0, scales0 = orc.fp4_quant(orc.widen(UPD[kind][1], upd0, None, upd0.shape).astype(np.float32))
+        r = request_inputs(inp, b)
+        req = orc.LowPrecRequest(UPD[kind][1], True, upd0, codes0, scales0, shape.ngroups, L + K, r["A"],
+                                 r["D"], seed, b)
+        req.flush_count.value = 1
+        for s in range(steps):
+            ys = req.verify(r["x"][s], r["B"][s], r["C"][s], r["dt"][s])
+            assert_close(to_np(y[s, b]), ys, f"verify on the FP4 copy at spec_b512_k4, step {s}, request {b}")
+            req.accept(int(n_host[s, b]))
+            if req.pos >= L:
+                upd, codes, scales, v32, fc_b, fc_a = snaps[s][b]
+                assert fc_a == fc_b + 1
+                v64 = req.refresh(want_v32=True).astype(np.float64)
+                assert_close(v32.astype(np.float64), v64, f"fp32 fold at spec_b512_k4, request {b}")
+                refresh_bits_of(kind, seed, b, fc_b, upd, codes, scales, v32,
+                                f"speculative {kind} + FP4 refresh at spec_b512_k4")
+                refreshed += 1
+                break  # later verifies read a copy requantised from the GPU's own fold
+    assert refreshed >= 3
+
+
 @pytest.mark.parametrize("shape", SHAPES, ids=["dstate64", "dstate128"])
 def test_shared_fp4_control_decode_matches_oracle(shape):
     """The shared FP4 control (s4's ablation): decode reads the one FP4 copy
