@@ -411,6 +411,49 @@ def test_shared_fp4_control_decode_matches_oracle(shape):
         assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of the shared FP4 refresh, request {b}")
 
 
+def test_shared_fp4_control_split_b256_sampled():
+    """The shared FP4 control at the bench's size (split_b256) and launch
+    configuration: one interval of decodes reading the FP4 copy and its
+    re-quantising refresh, with an fp32 twin from the same dequantised
+    values. For sampled requests the outputs match the oracle, the twin's
+    fold matches the fp64 fold, and the re-quantised codes and scales equal
+    the oracle's FP4 quantisation of the twin's fold bit for bit."""
+    w = WORKLOADS["split_b256"]
+    shape = w["shape"]
+    L = shape.interval
+    Bz, H, P, N = shape.batch, shape.nheads, shape.head_dim, shape.d_state
+    inp = make_inputs(shape, L, w["seed"], w["in_dtype"], device="cuda")
+    seed = w["seed"]
+    desc, st = fp4_control_state(shape, inp, seed)
+    vals = torch.empty((Bz, H, P, N), dtype=torch.float32, device="cuda")
+    reqs = sample_requests(Bz, 6)
+    codes0, scales0 = {}, {}
+    for b in range(Bz):  # dequantised starting values, request by request
+        c, sc = st.ckpt[b].cpu().numpy(), st.ckpt_scales[b].cpu().numpy()
+        vals[b].copy_(torch.from_numpy(orc.widen(orc.FP4, c, sc, (H, P, N)).astype(np.float32)))
+        if b in reqs:
+            codes0[b], scales0[b] = c, sc
+    _, tw = f32_twin(shape, vals, seed, out_copy=False)
+    y = torch.empty((L, Bz, H, P), device="cuda")
+    y2 = torch.empty_like(y)
+    for t in range(L):
+        args = (inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"])
+        rssm.rssm_decode_step(st, *args, y[t])
+        rssm.rssm_decode_step(tw, *args, y2[t])
+    rssm.rssm_lowprec_refresh(st, inp["A"])
+    rssm.rssm_lowprec_refresh(tw, inp["A"])
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
+    assert_refresh_bits("fp4", seed, st, tw, None, reqs, "shared FP4 refresh at split_b256")
+    for b in reqs:
+        r = request_inputs(inp, b)
+        req = orc.LowPrecRequest(orc.FP4, False, None, codes0[b], scales0[b], shape.ngroups, L, r["A"], r["D"],
+                                 seed, b)
+        ys = np.stack([req.decode(r["x"][t], r["B"][t], r["C"][t], r["dt"][t]) for t in range(L)])
+        assert_close(to_np(y[:, b]), ys, f"shared FP4 decode at split_b256, request {b}")
+        v64 = req.refresh(want_v32=True).astype(np.float64)
+        assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of the shared FP4 refresh at split_b256, request {b}")
+
+
 @pytest.mark.parametrize("shape", SPLIT_SHAPES, ids=SPLIT_IDS)
 @pytest.mark.parametrize("kind", ["bf16", "e4m3"])
 def test_shared_copy_decode_and_refresh_match_oracle(kind, shape):
