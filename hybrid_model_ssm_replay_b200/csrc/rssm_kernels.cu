@@ -2284,6 +2284,261 @@ __global__ void __launch_bounds__(kPfThreads, 3) k_prefill_mma(const PrefillArgs
 }
 
 // ---------------------------------------------------------------------------
+// Prefill on the 5th-generation tensor cores (tcgen05; bf16 inputs, d_state
+// 128, head_dim 64, an even number of heads per group). The same
+// contraction as k_prefill_mma, h_T - exp(A S) h_0 = X_w^T B, for two heads
+// of one group at once: the 128-row operand stacks their X_w (rows 0..63 the
+// first head's head_dim, 64..127 the second's) and both use the group's B.
+// One CTA of 8 warps per (request, head pair) walks the prompt in chunks of
+// 32 tokens from the last to the first (R_t a running suffix sum):
+//  - cp.async brings the chunk's B rows straight into the MMA's B operand
+//    layout, the two heads' x rows and dt (double-buffered);
+//  - warps 0-3 form the first head's w_t, warps 4-7 the second's (each warp
+//    alike, no barrier), and every thread splits w_t x_t[p] into bf16
+//    hi + mid + lo (x_w to ~2^-27) into the A operand;
+//  - one thread issues tcgen05.mma (M128 N128 K16, bf16 x bf16 -> fp32, A and
+//    B MN-major in 128-byte-swizzled atoms of 8 rows) into a 128-column fp32
+//    accumulator in tensor memory, 2 K-steps x 3 parts per chunk, and
+//    tcgen05.commit signals an mbarrier when they have read their operands;
+//  - after the last chunk each warp reads its 32 accumulator rows x 64
+//    columns with tcgen05.ld, adds exp(A S) h_0 and writes the checkpoint.
+// Tensor memory is allocated after the request's position check and freed on
+// every path that allocated it; every wait is bounded.
+// ---------------------------------------------------------------------------
+constexpr int kUmChunk = 32;                                          // prompt tokens per chunk
+constexpr int kUmThreads = 256;
+constexpr uint32_t kUmB = 2u * kUmChunk * 128u;                       // B operand: 2 column blocks x chunk x 128 B
+constexpr uint32_t kUmX = 2u * kUmChunk * 128u;                       // x rows: 2 heads x chunk x 64 bf16
+constexpr uint32_t kUmBuf = (kUmB + kUmX + 2u * kUmChunk * 4u + 1023u) & ~1023u;  // + dt [2 heads][chunk]; atom-aligned
+constexpr uint32_t kUmA = 2u * kUmChunk * 128u;                       // one A part: 2 heads x chunk x 128 B
+constexpr size_t kUmSmem = 1024 + 2 * static_cast<size_t>(kUmBuf) + 3 * static_cast<size_t>(kUmA);
+constexpr uint32_t kUmCols = 128;                                     // tensor-memory columns (fp32 D, N = 128)
+
+// Shared-memory matrix descriptor of a 128-byte-swizzled operand (start
+// address, leading and stride byte offsets in 16-byte units, descriptor
+// version 1, layout type 2 = 128-byte swizzle).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor: fp32 accumulator, bf16 A and B, both MN-major,
+// N = 128 (n_dim = N / 8), M = 128 (m_dim = M / 16).
+constexpr uint32_t kUmIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) | ((128u >> 3) << 17) |
+                              ((128u >> 4) << 24);
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kUmIdesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's accumulator row (lane quadrant of the warp).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__global__ void __launch_bounds__(kUmThreads, 3) k_prefill_umma(const PrefillArgs a) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t mma_bar;
+    __shared__ uint32_t s_tmem;
+    __shared__ float s_alpha[2];
+    __shared__ int s_pos;
+    const int H = a.s.H, G = a.s.G, batch = a.s.batch, T0 = a.T0;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int pairs = H >> 1;
+    const int b = blockIdx.x / pairs, h0 = 2 * (blockIdx.x - b * pairs), g = h0 / (H / G);
+    // operand buffers on a 1024-byte boundary (the swizzle atoms)
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    unsigned char* smem = smem_raw + (sbase - smem_u32(smem_raw));
+    const uint32_t s_a = sbase + 2 * kUmBuf;  // A parts: hi, mid, lo, kUmA bytes each
+
+    if (tid == 0) s_pos = a.pos[b];  // the only read of pos
+    __syncthreads();
+    if (s_pos != 0) {
+        if (tid == 0) set_error(a.err, RSSM_DEVERR_POS_RANGE);
+        return;
+    }
+    if (T0 <= 0) return;
+    if (warp == 0) {  // tensor memory for the accumulator (one warp allocates and frees)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                     "r"(kUmCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) mbar_init(smem_u32(&mma_bar), 1);
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = s_tmem;
+
+    const size_t HP = static_cast<size_t>(H) * 64, GN = static_cast<size_t>(G) * kD128;
+    const __nv_bfloat16* xin = static_cast<const __nv_bfloat16*>(a.x) + static_cast<size_t>(b) * HP + h0 * 64;
+    const __nv_bfloat16* Bin = static_cast<const __nv_bfloat16*>(a.B) + static_cast<size_t>(b) * GN +
+                               static_cast<size_t>(g) * kD128;
+    const size_t xstep = static_cast<size_t>(batch) * HP, bstep = static_cast<size_t>(batch) * GN;
+    const int nchunk = (T0 + kUmChunk - 1) / kUmChunk;
+
+    // chunk c (tokens 32c ..) into buffer `buf`: B rows in the operand layout
+    // (column block n / 64, token row k, 16-byte chunk (n % 64) / 8 ^ (k & 7)),
+    // the two heads' x rows [head][k][64], dt [head][k]; zeros past T0
+    auto fetch = [&](int c, int buf) {
+        const uint32_t base = sbase + static_cast<uint32_t>(buf) * kUmBuf;
+        const int t0 = c * kUmChunk;
+        for (int i = tid; i < kUmChunk * 16; i += kUmThreads) {
+            const int k = i >> 4, j = i & 15, t = t0 + k;
+            const bool ok = t < T0;
+            const uint32_t dst = base + (j >> 3) * (kUmChunk * 128) + k * 128 + 16 * ((j & 7) ^ (k & 7));
+            cp_async16_zfill(dst, Bin + static_cast<size_t>(ok ? t : t0) * bstep + 8 * j, ok);
+        }
+        for (int i = tid; i < kUmChunk * 16; i += kUmThreads) {
+            const int k = i >> 4, j = i & 15, t = t0 + k;  // j: head j / 8, 16-byte chunk j % 8 of its row
+            const bool ok = t < T0;
+            const uint32_t dst = base + kUmB + (j >> 3) * (kUmChunk * 128) + k * 128 + 16 * (j & 7);
+            cp_async16_zfill(dst, xin + static_cast<size_t>(ok ? t : t0) * xstep + 8 * j, ok);
+        }
+        if (tid < 2 * kUmChunk) {
+            const int hh = tid / kUmChunk, k = tid % kUmChunk, t = t0 + k;
+            const bool ok = t < T0;
+            cp_async4_zfill(base + kUmB + kUmX + 4 * (hh * kUmChunk + k),
+                            a.dt + (static_cast<size_t>(ok ? t : t0) * batch + b) * H + h0 + hh, ok);
+        }
+        cp_async_commit();
+    };
+
+    const int wh = warp >> 2;  // the head whose weights this warp forms
+    const float Ah = a.A[h0 + wh];
+    float carry = 0.f;  // dt sum of the chunks already folded (this warp's head)
+    bool timed_out = false;
+
+    fetch(nchunk - 1, (nchunk - 1) & 1);
+    for (int c = nchunk - 1, i = 0; c >= 0; --c, ++i) {
+        const int buf = c & 1;
+        const uint32_t base = sbase + static_cast<uint32_t>(buf) * kUmBuf;
+        const unsigned char* gbase = smem + static_cast<size_t>(buf) * kUmBuf;
+        cp_async_wait_all();
+        // the previous chunk's MMAs have read the A parts and their B buffer
+        if (i > 0 && !mbar_wait_bounded(smem_u32(&mma_bar), (i - 1) & 1, kWaitNs)) timed_out = true;
+        __syncthreads();  // chunk c landed for every thread; the buffers above are free
+        if (c > 0) fetch(c - 1, buf ^ 1);
+        // w_t = dt_t exp(A R_t) of this warp's head: lane l takes token l
+        const float* dts = reinterpret_cast<const float*>(gbase + kUmB + kUmX) + wh * kUmChunk;
+        const float v = dts[lane];
+        float s = v;  // inclusive suffix sum
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float u = __shfl_down_sync(0xffffffffu, s, off);
+            if (lane + off < 32) s += u;
+        }
+        const float tot = __shfl_sync(0xffffffffu, s, 0);
+        const float wl = v * expf(Ah * (carry + (s - v)));
+        carry += tot;
+        {
+            // x_w = w_t x_t[p] as bf16 hi + mid + lo: thread -> head tid / 128,
+            // token (tid % 128) / 4, rows 16 (tid % 4) .. + 15
+            const int hh = tid >> 7, k = (tid & 127) >> 2, p0 = 16 * (tid & 3);
+            const float w = __shfl_sync(0xffffffffu, wl, k);  // warps of head hh hold its weights
+            const unsigned char* xrow = gbase + kUmB + hh * (kUmChunk * 128) + k * 128 + 2 * p0;
+            const uint4 u0 = *reinterpret_cast<const uint4*>(xrow);
+            const uint4 u1 = *reinterpret_cast<const uint4*>(xrow + 16);
+            const uint32_t xw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            uint32_t hi[8], md[8], lo[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float f0 = w * __uint_as_float(bf16lo_bits(xw[q]));
+                const float f1 = w * __uint_as_float(bf16hi_bits(xw[q]));
+                const uint32_t hh2 = f32x2_to_bf16x2(f0, f1);
+                hi[q] = hh2;
+                const float r0 = f0 - __uint_as_float(bf16lo_bits(hh2)), r1 = f1 - __uint_as_float(bf16hi_bits(hh2));
+                const uint32_t mm = f32x2_to_bf16x2(r0, r1);
+                md[q] = mm;
+                lo[q] = f32x2_to_bf16x2(r0 - __uint_as_float(bf16lo_bits(mm)), r1 - __uint_as_float(bf16hi_bits(mm)));
+            }
+            // A part layout: [head][token k][128 B], 16-byte chunk (p / 8) ^ (k & 7)
+            const int c0 = p0 >> 3;
+            const uint32_t row = static_cast<uint32_t>(hh * (kUmChunk * 128) + k * 128);
+            const uint32_t d0 = row + 16 * (c0 ^ (k & 7)), d1 = row + 16 * ((c0 + 1) ^ (k & 7));
+            unsigned char* ap = smem + (s_a - sbase);
+            *reinterpret_cast<uint4*>(ap + d0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(ap + d1) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+            *reinterpret_cast<uint4*>(ap + kUmA + d0) = make_uint4(md[0], md[1], md[2], md[3]);
+            *reinterpret_cast<uint4*>(ap + kUmA + d1) = make_uint4(md[4], md[5], md[6], md[7]);
+            *reinterpret_cast<uint4*>(ap + 2 * kUmA + d0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            *reinterpret_cast<uint4*>(ap + 2 * kUmA + d1) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+        }
+        // the operands written by ordinary stores and cp.async, visible to the tensor cores
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+        if (tid == 0) {
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll
+            for (int ks = 0; ks < kUmChunk / 16; ++ks) {
+                // K-step: 16 tokens = two 8-row atoms (SBO 1024 B); A: head blocks
+                // 64 rows apart in M (LBO = chunk x 128 B); B: column blocks of 64
+#pragma unroll
+                for (int part = 0; part < 3; ++part) {
+                    const uint64_t ad = umma_desc_sw128(s_a + part * kUmA + ks * 2048, kUmChunk * 128, 1024);
+                    const uint64_t bd = umma_desc_sw128(base + ks * 2048, kUmChunk * 128, 1024);
+                    umma_f16(tmem, ad, bd, (i > 0 || ks > 0 || part > 0) ? 1u : 0u);
+                }
+            }
+            umma_commit(smem_u32(&mma_bar));
+        }
+    }
+    // the last chunk's products complete
+    if (!mbar_wait_bounded(smem_u32(&mma_bar), (nchunk - 1) & 1, kWaitNs)) timed_out = true;
+    if (lane == 0 && (warp == 0 || warp == 4)) s_alpha[wh] = expf(Ah * carry);
+    if (timed_out) set_error(a.err, RSSM_DEVERR_TIMEOUT);
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    {
+        // warp w reads accumulator lanes 32 (w % 4) .. (rows = head_dim rows of
+        // head (w % 4) / 2) and columns 64 (w / 4) ..
+        const int q = warp & 3, half = warp >> 2;
+        const int r = 32 * q + lane, hh = r >> 6, p = r & 63;
+        const float alpha = s_alpha[hh];
+        float* hrow = reinterpret_cast<float*>(a.record + (static_cast<size_t>(b) * H + h0 + hh) * a.rec.bytes) +
+                      static_cast<size_t>(p) * kD128;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            const int col = 64 * half + 16 * cc;
+            float d[16];
+            tmem_ld16(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(col), d);
+            float4* hp = reinterpret_cast<float4*>(hrow + col);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+                const float4 h = hp[v4];
+                hp[v4] = make_float4(fmaf(alpha, h.x, d[4 * v4]), fmaf(alpha, h.y, d[4 * v4 + 1]),
+                                     fmaf(alpha, h.z, d[4 * v4 + 2]), fmaf(alpha, h.w, d[4 * v4 + 3]));
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kUmCols) : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Conventional scheme (in-run comparison, s1/s3): per token
 //   h <- exp(dt A) h + dt x B^T, write h, y = h C + D x.
 // VERIFY: read copy cur[b], write the state after token j to copy j.
@@ -2762,6 +3017,14 @@ cudaError_t launch_fold(const FoldArgs& a, int in_bf16, int uf, cudaStream_t st)
 }
 
 cudaError_t launch_prefill(const PrefillArgs& a, int in_bf16, cudaStream_t st) {
+    if (in_bf16 && a.s.N == 128 && a.s.P == 64 && (a.s.H / a.s.G) % 2 == 0) {
+        if (a.s.batch * a.s.H <= 0) return cudaSuccess;
+        cudaError_t e = cudaFuncSetAttribute(k_prefill_umma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kUmSmem));
+        if (e != cudaSuccess) return e;
+        k_prefill_umma<<<a.s.batch * (a.s.H / 2), kUmThreads, kUmSmem, st>>>(a);
+        return cudaGetLastError();
+    }
     if (in_bf16 && a.s.N == 128 && a.s.P % 16 == 0 && a.s.P <= 64) {
         if (a.s.batch * a.s.H <= 0) return cudaSuccess;
         cudaError_t e = cudaFuncSetAttribute(k_prefill_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
