@@ -2410,7 +2410,7 @@ __global__ void __launch_bounds__(kUmThreads, 3) k_prefill_umma(const PrefillArg
         for (int i = tid; i < kUmChunk * 16; i += kUmThreads) {
             const int k = i >> 4, j = i & 15, t = t0 + k;  // j: head j / 8, 16-byte chunk j % 8 of its row
             const bool ok = t < T0;
-            const uint32_t dst = base + kUmB + (j >> 3) * (kUmChunk * 128) + k * 128 + 16 * (j & 7);
+            const uint32_t dst = base + kUmB + (j >> 3) * (kUmChunk * 128) + k * 128 + 16 * ((j & 7) ^ (k & 7));
             cp_async16_zfill(dst, xin + static_cast<size_t>(ok ? t : t0) * xstep + 8 * j, ok);
         }
         if (tid < 2 * kUmChunk) {
@@ -2454,9 +2454,10 @@ __global__ void __launch_bounds__(kUmThreads, 3) k_prefill_umma(const PrefillArg
             // token (tid % 128) / 4, rows 16 (tid % 4) .. + 15
             const int hh = tid >> 7, k = (tid & 127) >> 2, p0 = 16 * (tid & 3);
             const float w = __shfl_sync(0xffffffffu, wl, k);  // warps of head hh hold its weights
-            const unsigned char* xrow = gbase + kUmB + hh * (kUmChunk * 128) + k * 128 + 2 * p0;
-            const uint4 u0 = *reinterpret_cast<const uint4*>(xrow);
-            const uint4 u1 = *reinterpret_cast<const uint4*>(xrow + 16);
+            // (x rows are staged with 16-byte chunk (p / 8) ^ (k & 7), conflict-free here)
+            const unsigned char* xrow = gbase + kUmB + hh * (kUmChunk * 128) + k * 128;
+            const uint4 u0 = *reinterpret_cast<const uint4*>(xrow + 16 * ((p0 >> 3) ^ (k & 7)));
+            const uint4 u1 = *reinterpret_cast<const uint4*>(xrow + 16 * (((p0 >> 3) + 1) ^ (k & 7)));
             const uint32_t xw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
             uint32_t hi[8], md[8], lo[8];
 #pragma unroll
