@@ -1001,7 +1001,8 @@ def prefill_leg(rssm, torch, wl, dev, barrier, max_over_ranks, world, T0=512, re
     flops = 2.0 * H * P * N * T0 * shape.batch
     return {"workload": f"small_b256 shapes, prompt of {T0} tokens per request", "prompt_tokens_per_s":
             world * shape.batch * T0 / (ms / 1e3), "ms_per_prefill": ms,
-            "kernel": "k_prefill_mma (mma.sync bf16, x_w split hi + mid + lo)",
+            "kernel": "k_prefill_umma (tcgen05.mma M128 N128 K16 bf16 -> fp32 in tensor memory, two heads per CTA, "
+                      "x_w split hi + mid + lo)",
             "bound": "hbm", "algorithmic_bytes_per_request": req_bytes, "achieved_gbs": gbs, "peak": peak,
             "peak_source": peak_src, "frac": gbs / peak,
             "contraction_tflops": flops / (ms / 1e3) / 1e12,
