@@ -34,7 +34,7 @@ def split(inp, T0):
 @pytest.mark.parametrize("shape,T0", [(LayerShape(4, 4, 40, 128, 2), 50), (LayerShape(3, 4, 17, 64, 1), 33),
                                       (LayerShape(2, 2, 8, 16, 1), 16), (LayerShape(3, 4, 64, 128, 2), 150),
                                       (LayerShape(2, 4, 32, 128, 2), 64), (LayerShape(2, 2, 48, 128, 1), 200)],
-                         ids=["d128", "ragged", "one-chunk", "mma-3chunks", "mma-1chunk", "mma-headdim48"])
+                         ids=["d128", "ragged", "one-chunk", "umma-5chunks", "mma-1chunk", "mma-headdim48"])
 def test_prefill_then_decode_matches_recurrence(shape, T0, in_dtype):
     steps = T0 + 24
     inp = make_inputs(shape, steps, 41, in_dtype, device="cuda")
@@ -57,6 +57,24 @@ def test_prefill_then_decode_matches_recurrence(shape, T0, in_dtype):
         assert_close(ck[b], snaps[T0 - 1], f"checkpoint after a {T0}-token prefill, request {b}")
         assert_close(to_np(y[:, b]), y_ref[T0:], f"decode after the prefill, request {b}")
     assert set(st.flush_count.cpu().tolist()) == {(steps - T0) // L}
+
+
+@pytest.mark.parametrize("T0", [1, 31, 32, 33, 65])
+def test_prefill_tensor_memory_chunk_edges(T0):
+    """The tcgen05 prefill (head_dim 64, two heads per group) at prompt
+    lengths around its 32-token chunks: one token, a chunk minus one, one
+    chunk, a chunk plus one, two chunks plus one; every request's checkpoint
+    against the recurrence."""
+    shape = LayerShape(3, 8, 64, 128, 2)
+    inp = make_inputs(shape, T0, 44 + T0, torch.bfloat16, device="cuda")
+    st = rssm.RssmState(desc_for(shape))
+    st.ckpt.copy_(inp["ckpt"])
+    rssm.rssm_prefill(st, inp["x"], inp["B"], inp["dt"], inp["A"])
+    assert rssm.rssm_get_error(st) == 0
+    res = oracle_map([("conv", request_inputs(inp, b), [T0 - 1]) for b in range(shape.batch)])
+    for b, (_, snaps) in enumerate(res):
+        assert_close(st.ckpt[b].double().cpu().numpy(), snaps[T0 - 1], f"checkpoint after a {T0}-token prefill, "
+                                                                        f"request {b}")
 
 
 def test_prefill_b256_t512_sampled():
