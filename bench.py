@@ -894,7 +894,10 @@ def split_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
     fp4 = H * P * N // 2 + H * P * N // 16
     tok_other = sum(i * b["entry"] for i in range(L)) / L + b["entry"] + b["inputs"] + b["y"]
     out = {"workload": "split_b256: batch 256, 64 heads, 64 x 128, 8 groups, interval 16; decode reads the FP4 "
-                       "copy, refresh every 16 tokens", "steps": K}
+                       "copy, refresh every 16 tokens", "steps": K,
+           "refresh_kernel": "k_fold_umma (the fold of two heads of a group as one tcgen05.mma M128 N128 K16 "
+                             "per 16 buffered tokens into tensor memory, x_w split bf16 hi + mid + lo; epilogue "
+                             "one accumulator row per thread: Philox SR and FP4 blocks in registers)"}
     hpn = H * P * N
     # (name, update dtype, output copy, bytes of the copy decode reads, of the update copy, of the output copy)
     modes = [("bf16_fp4", rssm.RSSM_BF16, rssm.RSSM_OUTCOPY_FP4, fp4, 2 * hpn, fp4),
@@ -961,6 +964,7 @@ def split_leg(rssm, torch, wl, K, W, dev, barrier, max_over_ranks, world, peak):
         out[name] = {"tokens_per_s": world * shape.batch * L * K / (ms / 1e3), "decode_avg_launch_us": d_us,
                      "decode_gbs": dec_bytes / (d_us / 1e6) / 1e9, "decode_frac": dec_bytes / (d_us / 1e6) / 1e9 / peak,
                      "refresh_avg_launch_us": r_us, "refresh_gbs": ref_bytes / (r_us / 1e6) / 1e9,
+                     "refresh_frac": ref_bytes / (r_us / 1e6) / 1e9 / peak,
                      "step_bytes_per_token": (dec_bytes * L + ref_bytes) / (shape.batch * L)}
         del st
         torch.cuda.empty_cache()

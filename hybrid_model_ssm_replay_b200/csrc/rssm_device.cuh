@@ -175,7 +175,7 @@ struct PhiloxKeys {
     uint32_t x[10], y[10];
 };
 
-__device__ __forceinline__ PhiloxKeys philox_keys(uint64_t seed) {
+__host__ __device__ __forceinline__ PhiloxKeys philox_keys(uint64_t seed) {
     PhiloxKeys K;
     uint32_t kx = static_cast<uint32_t>(seed), ky = static_cast<uint32_t>(seed >> 32);
 #pragma unroll
@@ -201,6 +201,44 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys& K) {
 
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
     return philox4x32_10(c, philox_keys(static_cast<uint64_t>(k.x) | (static_cast<uint64_t>(k.y) << 32)));
+}
+
+// Draws whose counters (c0, c1, c2, c3) share c1, c2, c3 (one head of one
+// request at one flush): the parts of the first two rounds that do not
+// depend on c0 -- the second word's multiply in round one and the first
+// word's in round two -- are formed once (PhiloxFixed); each draw then runs
+// the same ten rounds with two multiplies fewer.
+struct PhiloxFixed {
+    uint32_t f1k;  // round-one output y, xored with round two's x key
+    uint32_t g, h;  // round two's multiply of round-one output x: high half ^ y key, low half
+    uint32_t c3k;  // c3 ^ round one's y key
+};
+
+__device__ __forceinline__ PhiloxFixed philox_fixed(uint32_t c1, uint32_t c2, uint32_t c3, const PhiloxKeys& K) {
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c2;
+    const uint32_t x1 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ K.x[0];
+    const uint64_t q0 = static_cast<uint64_t>(0xD2511F53u) * x1;
+    PhiloxFixed F;
+    F.f1k = static_cast<uint32_t>(p1) ^ K.x[1];
+    F.g = static_cast<uint32_t>(q0 >> 32) ^ K.y[1];
+    F.h = static_cast<uint32_t>(q0);
+    F.c3k = c3 ^ K.y[0];
+    return F;
+}
+
+__device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, const PhiloxFixed& F, const PhiloxKeys& K) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c0;  // round one: (x1, y1, z1, w1)
+    const uint32_t z1 = static_cast<uint32_t>(p0 >> 32) ^ F.c3k, w1 = static_cast<uint32_t>(p0);
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * z1;  // round two
+    uint4 c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ F.f1k, static_cast<uint32_t>(p1), F.g ^ w1, F.h);
+#pragma unroll
+    for (int i = 2; i < 10; ++i) {
+        const uint64_t q0 = static_cast<uint64_t>(0xD2511F53u) * c.x;
+        const uint64_t q1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+        c = make_uint4(static_cast<uint32_t>(q1 >> 32) ^ c.y ^ K.x[i], static_cast<uint32_t>(q1),
+                       static_cast<uint32_t>(q0 >> 32) ^ c.w ^ K.y[i], static_cast<uint32_t>(q0));
+    }
+    return c;
 }
 
 // ------------------------------------------------------ stochastic rounding
@@ -287,6 +325,28 @@ __device__ __forceinline__ float4 e2m1x4_val(uint32_t codes16) {
     return make_float4(a.x, a.y, b.x, b.y);
 }
 
+// Eight e2m1 codes (32 bits, element 0 in the low nibble) as floats times
+// scale (exact: hardware conversion of each byte to an fp16 pair). The word
+// is split into its four bytes inside one asm block.
+__device__ __forceinline__ void e2m1x8_val(uint32_t w, float scale, float* v) {
+    uint32_t h0, h1, h2, h3;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+        : "r"(w));
+    const uint32_t h[4] = {h0, h1, h2, h3};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = h2_f2(h[i]);
+        v[2 * i] = f.x * scale;
+        v[2 * i + 1] = f.y * scale;
+    }
+}
+
 // Dot product of eight e2m1 codes (32 bits, element 0 in the low nibble)
 // with c[0..7], unscaled, added to acc in element order.
 __device__ __forceinline__ float e2m1x8_dot(uint32_t w, const float* c, float acc) {
@@ -364,6 +424,51 @@ __device__ __forceinline__ uint32_t fp4_quant_quad(float4 v, uint32_t* scale_cod
     const uint32_t c01 = e2m1x2_rn(__fdiv_rn(v.x, s), __fdiv_rn(v.y, s));
     const uint32_t c23 = e2m1x2_rn(__fdiv_rn(v.z, s), __fdiv_rn(v.w, s));
     return c01 | (c23 << 8);
+}
+
+// Eight e2m1 codes (nearest even, saturating to +-6) of v[0..7] scaled by
+// m: element i in nibble i.
+__device__ __forceinline__ uint32_t e2m1x8_rn(const float* v, float m) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(v[0] * m), "f"(v[1] * m), "f"(v[2] * m), "f"(v[3] * m), "f"(v[4] * m), "f"(v[5] * m),
+          "f"(v[6] * m), "f"(v[7] * m));
+    return out;
+}
+
+// FP4 copy of one block of 16 contiguous values held by one thread: the
+// scale and codes of fp4_quant_quad (the same bracketed quotients), with
+// the block maximum taken in registers. Returns the 64 code bits, element i
+// in nibble i % 8 of word i / 8, and sets *scale_code.
+__device__ __forceinline__ uint2 fp4_quant16(const float (&v)[16], uint32_t* scale_code) {
+    float m8[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(v[i]), fabsf(v[i + 8]));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m8[i] = fmaxf(m8[i], m8[i + 4]);
+    const float amax = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
+    constexpr float kSixthLo = 0x1.555554p-3f, kSixthHi = 0x1.555556p-3f;  // adjacent floats around 1/6
+    uint32_t sc = e4m3_rn(amax * kSixthLo);
+    if (sc != e4m3_rn(amax * kSixthHi)) sc = e4m3_rn(__fdiv_rn(amax, 6.0f));
+    *scale_code = sc;
+    const float s = e4m3_val(sc);
+    if (s == 0.0f) return make_uint2(0u, 0u);
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));  // s >= 2^-9: never subnormal
+    const float rlo = r * (1.0f - 0x1p-19f), rhi = r * (1.0f + 0x1p-19f);
+    const uint2 lo = make_uint2(e2m1x8_rn(v, rlo), e2m1x8_rn(v + 8, rlo));
+    const uint2 hi = make_uint2(e2m1x8_rn(v, rhi), e2m1x8_rn(v + 8, rhi));
+    if (lo.x == hi.x && lo.y == hi.y) return lo;
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(v[i], s);
+    return make_uint2(e2m1x8_rn(q, 1.0f), e2m1x8_rn(q + 8, 1.0f));
 }
 
 }  // namespace rssm

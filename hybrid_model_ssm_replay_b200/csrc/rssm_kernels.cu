@@ -2540,6 +2540,526 @@ __global__ void __launch_bounds__(kUmThreads, 3) k_prefill_umma(const PrefillArg
 }
 
 // ---------------------------------------------------------------------------
+// Low-precision refresh with the fold on the 5th-generation tensor cores
+// (bf16 inputs, d_state 128, head_dim 64, an even number of heads per
+// group). The fold of s1, v = exp(A S_T) h_0 + X_w^T B with X_w[s][p] =
+// dt_s exp(A (S_T - S_s)) x_s[p], is a K = T contraction; two heads of one
+// group share the request's B rows and position, so a head pair is one
+// M128 N128 tcgen05.mma per 16 buffered tokens (rows 0..63 the first head's
+// head_dim, 64..127 the second's). One persistent CTA per SM: a producer
+// warp brings each due pair into a stage (both update copies, dt and x
+// rows, the group's B rows; bulk copies on an mbarrier ring, as in
+// k_fold_pipe) and consumer groups of four warps take the pairs in turn:
+//  - warps 0 and 1 form the two heads' weights, then the group builds one
+//    K-step's operands: X_w split into bf16 hi + mid + lo (~2^-27
+//    relative) and the B rows (exact in bf16), MN-major in 128-byte-swizzled
+//    atoms, zero past T;
+//  - one thread issues the three MMAs into the group's 128-column fp32
+//    accumulator in tensor memory and commits them to the group's mbarrier;
+//  - each thread then owns one accumulator row (warp w reads lanes
+//    32 (w % 4) ..): 16 columns at a time it reads the row with tcgen05.ld,
+//    adds exp(A S_T) h_0 from the stage and runs the format's epilogue -- a
+//    Philox draw per 4 consecutive columns and the stochastic rounding, an
+//    FP4 block of 16 columns quantised in registers -- storing straight to
+//    global memory.
+// Every wait is bounded; tensor memory is allocated once per CTA and freed
+// on every path.
+// ---------------------------------------------------------------------------
+struct FoldUmmaLayout {
+    uint32_t hb;           // one head's block in a stage: update copy (+ scales), dt row, x rows
+    uint32_t st_dt, st_x;  // offsets of the dt row and the x rows in a head block
+    uint32_t brows;        // the group's B rows [cap][128] (bf16), after the two head blocks
+    uint32_t meta;
+    uint32_t stage_bytes;
+    int stages;
+    FastDiv divPr;    // head pair -> request (H / 2 pairs per request)
+    FastDiv divHpg;   // head -> group
+    PhiloxKeys keys;  // the ten round keys of the seed (read from the parameter space)
+};
+
+constexpr int kFuK = 16;                        // buffered tokens per MMA K-step
+constexpr uint32_t kFuPart = 2u * kFuK * 128u;  // one A part: 2 heads x 16 tokens x 128 B
+constexpr uint32_t kFuOps = 4u * kFuPart;       // A hi, mid, lo + B (2 column blocks x 16 tokens x 128 B)
+// meta words of a stage: pair index (-1: end), position, flush count, A of both heads, tag
+constexpr int kUMetaPair = 0, kUMetaPos = 1, kUMetaFc = 2, kUMetaA0 = 3, kUMetaTag = 5;
+
+// Consumer groups per update format and warps per group (4: a thread owns
+// a whole row; 8: half a row, the two halves of the row's columns on warps
+// w and w + 4). A group holds its stage for the whole pair, so there must be
+// at least as many stages as groups (bf16 stages are ~41 KB). B200, split_b256
+// refresh: bf16 3 x 4 warps 234 us (3 x 8: 246); e4m3 3 x 8 306 us (4 x 4:
+// 366 before the epilogue loop was unrolled by 2); FP4 4 x 4 91 us (3 x 8: 96).
+__host__ __device__ constexpr int fu_groups(int uf) { return uf == kF32 ? 2 : (uf == kFP4 ? 4 : 3); }
+__host__ __device__ constexpr int fu_cwarps(int uf) { return uf == kE4M3 ? 8 : 4; }
+__host__ __device__ constexpr int fu_threads(int uf) { return (fu_cwarps(uf) * fu_groups(uf) + 1) * 32; }
+__host__ __device__ constexpr uint32_t fu_cols(int uf) { return fu_groups(uf) <= 2 ? 256u : 512u; }
+
+// 16 consecutive values (row p, columns 16 cc ..) of a 64 x 128 tile in
+// shared memory, in format F (FP4: codes, and the block scales at sc).
+template <int F>
+__device__ __forceinline__ void row16_load(const unsigned char* t, const unsigned char* sc, int p, int cc,
+                                           float (&v)[16]) {
+    if constexpr (F == kF32) {
+        const float4* q = reinterpret_cast<const float4*>(t + p * 512 + cc * 64);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 f = q[i];
+            v[4 * i] = f.x;
+            v[4 * i + 1] = f.y;
+            v[4 * i + 2] = f.z;
+            v[4 * i + 3] = f.w;
+        }
+    } else if constexpr (F == kBF16) {
+        const uint4* q = reinterpret_cast<const uint4*>(t + p * 256 + cc * 32);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const uint4 u = q[i];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                v[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
+                v[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+            }
+        }
+    } else if constexpr (F == kE4M3) {
+        const uint4 u = *reinterpret_cast<const uint4*>(t + p * 128 + cc * 16);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float4 f = e4m3x4_val(w[k]);
+            v[4 * k] = f.x;
+            v[4 * k + 1] = f.y;
+            v[4 * k + 2] = f.z;
+            v[4 * k + 3] = f.w;
+        }
+    } else {
+        const uint2 u = *reinterpret_cast<const uint2*>(t + p * 64 + cc * 8);
+        const float s = e4m3_val(sc[p * 8 + cc]);
+        e2m1x8_val(u.x, s, v);
+        e2m1x8_val(u.y, s, v + 8);
+    }
+}
+
+template <int UF, int OUT4>
+__global__ void __launch_bounds__(fu_threads(UF), 1) k_fold_umma(const FoldArgs a, const __grid_constant__ FoldUmmaLayout lay) {
+    constexpr int CG = fu_groups(UF), CW = fu_cwarps(UF), CT = CW * 32;
+    constexpr int NCC = 8 * 4 / CW;  // 16-column steps per thread
+    static_assert(CW == 4 || CW == 8, "a group covers the 128 accumulator lanes with 4 or 8 warps");
+    static_assert(128 * CG <= static_cast<int>(fu_cols(UF)), "each group's 128 accumulator columns are allocated");
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[kPipeStagesMax];
+    __shared__ __align__(8) uint64_t empty_bar[kPipeStagesMax];
+    __shared__ __align__(8) uint64_t mma_bar[CG];
+    __shared__ float s_cw[CG][2][kMaxCap];  // dt_s exp(A_j (S_T - S_s)) of head j of the group's pair
+    __shared__ float s_alpha[CG][2];        // exp(A_j S_T)
+    __shared__ uint32_t s_tmem;
+    __shared__ volatile int s_abort;
+
+    const int H = a.s.H, G = a.s.G, cap = a.s.cap, L = a.s.L;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int S = lay.stages;
+    const int hp = H >> 1;  // head pairs per request
+    const int npairs = a.s.batch * hp;
+    const uint32_t tbu = tile_bytes(UF, 64, kD128) + scale_bytes(UF, 64, kD128);
+    const bool in_record = a.upd == a.record;
+    // the groups' operand areas (1024-byte swizzle atoms) first, then the stages
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    unsigned char* smem = smem_raw + (sbase - smem_u32(smem_raw));
+    unsigned char* stg = smem + CG * kFuOps;
+
+    pdl_prologue();
+    if (warp == 0) {  // one warp allocates the accumulators (128 columns per group) and frees them
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                     "r"(fu_cols(UF))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 32) {
+        for (int st = 0; st < S; ++st) {
+            mbar_init(smem_u32(&full_bar[st]), 1);
+            mbar_init(smem_u32(&empty_bar[st]), CW);
+            reinterpret_cast<int*>(stg + static_cast<size_t>(st) * lay.stage_bytes + lay.meta)[kUMetaTag] = -1;
+        }
+        for (int g = 0; g < CG; ++g) mbar_init(smem_u32(&mma_bar[g]), 1);
+        s_abort = 0;
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = s_tmem;
+
+    if (warp == CG * CW) {
+        // ------------------------------------------------------------ producer
+        int p0 = 0, p1 = 0;
+        uint32_t f0 = 0, f1 = 0;
+        float2 A0 = make_float2(0.f, 0.f), A1 = A0;
+        auto fetch = [&](int kbase, int& pp, uint32_t& ff, float2& AA) {
+            const uint32_t u = blockIdx.x + static_cast<uint32_t>(kbase + lane) * gridDim.x;
+            if (u < static_cast<uint32_t>(npairs)) {
+                const int bb = fdiv(u, lay.divPr);
+                const int hh = 2 * (static_cast<int>(u) - bb * hp);
+                pp = a.pos[bb];
+                ff = a.flush_count[bb];
+                AA = make_float2(a.A[hh], a.A[hh + 1]);
+            }
+        };
+        fetch(0, p0, f0, A0);
+        fetch(32, p1, f1, A1);
+        int q = 0, st = 0, use = 0;  // stage sequence of the due pairs
+        int q_issued = -1;
+        bool aborted = false;
+        auto take_stage = [&]() {
+            int live = 1;
+            if (lane == 0) {
+                if (use > 0 && !mbar_wait_bounded(smem_u32(&empty_bar[st]), (use - 1) & 1, kWaitNs)) {
+                    set_error(a.err, RSSM_DEVERR_TIMEOUT);
+                    s_abort = 1;
+                }
+                live = !s_abort;
+            }
+            return __shfl_sync(0xffffffffu, live, 0) != 0;
+        };
+        auto next_stage = [&]() {
+            q_issued = q;
+            ++q;
+            if (++st == S) {
+                st = 0;
+                ++use;
+            }
+        };
+        for (int k = 0; blockIdx.x + static_cast<uint32_t>(k) * gridDim.x < static_cast<uint32_t>(npairs); ++k) {
+            const uint32_t u = blockIdx.x + static_cast<uint32_t>(k) * gridDim.x;
+            const bool cur = (k >> 5) & 1;
+            const int sel = k & 31;
+            if (sel == 0 && k > 0) {
+                if (cur)
+                    fetch(k + 32, p0, f0, A0);
+                else
+                    fetch(k + 32, p1, f1, A1);
+            }
+            const int pos = __shfl_sync(0xffffffffu, cur ? p1 : p0, sel);
+            const uint32_t fc = __shfl_sync(0xffffffffu, cur ? f1 : f0, sel);
+            const float Aa = __shfl_sync(0xffffffffu, cur ? A1.x : A0.x, sel);
+            const float Ab = __shfl_sync(0xffffffffu, cur ? A1.y : A0.y, sel);
+            if (pos < 0 || pos > cap) {
+                if (lane == 0) set_error(a.err, RSSM_DEVERR_POS_RANGE);
+                continue;
+            }
+            if (!((pos >= L) || (a.mode >= 1 && pos > 0) || (a.mode == 2))) continue;  // not due
+            if (!take_stage()) {
+                aborted = true;
+                break;
+            }
+            if (lane == 0) {
+                unsigned char* sp = stg + static_cast<size_t>(st) * lay.stage_bytes;
+                const uint32_t fb = smem_u32(&full_bar[st]);
+                int* meta = reinterpret_cast<int*>(sp + lay.meta);
+                meta[kUMetaPair] = static_cast<int>(u);
+                meta[kUMetaPos] = pos;
+                meta[kUMetaFc] = static_cast<int>(fc);
+                reinterpret_cast<float*>(meta)[kUMetaA0] = Aa;
+                reinterpret_cast<float*>(meta)[kUMetaA0 + 1] = Ab;
+                reinterpret_cast<volatile int*>(meta)[kUMetaTag] = q;
+                const int b = fdiv(u, lay.divPr), h0 = 2 * (static_cast<int>(u) - b * hp);
+                const size_t t0 = static_cast<size_t>(b) * H + h0;
+                const uint32_t nx = static_cast<uint32_t>(pos) * 128u, nb = static_cast<uint32_t>(pos) * 256u;
+                const uint32_t ndx = (a.rec.x - a.rec.dt) + nx;  // dt row and x rows, contiguous in the record
+                const uint32_t per = in_record ? a.rec.x + nx : tbu + ndx;
+                mbar_expect_tx(fb, 2u * per + nb);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const unsigned char* rec = a.record + (t0 + j) * a.rec.bytes;
+                    unsigned char* hbp = sp + j * lay.hb;
+                    if (in_record) {
+                        bulk_g2s(smem_u32(hbp), rec, a.rec.x + nx, fb);
+                    } else {
+                        bulk_g2s(smem_u32(hbp), a.upd + (t0 + j) * a.upd_stride, tbu, fb);
+                        bulk_g2s(smem_u32(hbp + lay.st_dt), rec + a.rec.dt, ndx, fb);
+                    }
+                }
+                if (nb > 0) {
+                    const size_t bg = static_cast<size_t>(b) * G + fdiv(static_cast<uint32_t>(h0), lay.divHpg);
+                    bulk_g2s(smem_u32(sp + lay.brows),
+                             static_cast<const unsigned char*>(a.bbuf) + bg * static_cast<size_t>(cap) * 256u, nb, fb);
+                }
+            }
+            next_stage();
+            __syncwarp();
+        }
+        // one end marker per consumer group
+        for (int e = 0; e < CG && !aborted; ++e) {
+            if (!take_stage()) {
+                aborted = true;
+                break;
+            }
+            if (lane == 0) {
+                unsigned char* sp = stg + static_cast<size_t>(st) * lay.stage_bytes;
+                int* meta = reinterpret_cast<int*>(sp + lay.meta);
+                meta[kUMetaPair] = -1;
+                reinterpret_cast<volatile int*>(meta)[kUMetaTag] = q;
+                mbar_expect_tx(smem_u32(&full_bar[st]), 0u);
+            }
+            next_stage();
+            __syncwarp();
+        }
+        if (aborted && lane == 0) {
+            for (int qq = q_issued; qq >= 0 && qq > q_issued - S; --qq)
+                mbar_wait_bounded(smem_u32(&full_bar[qq % S]), (qq / S) & 1, kWaitNs);
+        }
+        return;
+    }
+
+    // --------------------------------------------------------------- consumers
+    const int gi = warp / CW, cw = warp - gi * CW, ctid = tid - gi * CT;
+    const PhiloxKeys& pkeys = lay.keys;
+    unsigned char* ops = smem + gi * kFuOps;
+    const uint32_t ops_u = sbase + gi * kFuOps;
+    const uint32_t tacc = tmem + 128u * gi;                                     // the group's accumulator
+    // this thread's row (accumulator lane 32 (cw % 4) + lane: head jr, row pr)
+    // and its columns, 16 cc0 .. 16 (cc0 + NCC) - 1
+    const int jr = (32 * (cw & 3) + lane) >> 6, pr = (32 * (cw & 3) + lane) & 63, cc0 = (cw >> 2) * NCC;
+    const uint32_t trow = tacc + (static_cast<uint32_t>(32 * (cw & 3)) << 16);  // this warp's lanes
+    const uint32_t mbar = smem_u32(&mma_bar[gi]);
+    uint32_t ncommit = 0;
+    bool timed_out = false;
+    int st = gi, use = 0;
+    while (st >= S) {
+        st -= S;
+        ++use;
+    }
+    int pend_b = -1;
+    uint32_t pend_old = 0;
+    for (int q = gi;; q += CG) {
+        unsigned char* sp = stg + static_cast<size_t>(st) * lay.stage_bytes;
+        const int* meta = reinterpret_cast<const int*>(sp + lay.meta);
+        int stop = 0;
+        if (ctid == 0) {
+            stop = s_abort;
+            const volatile int* tag = reinterpret_cast<const volatile int*>(meta) + kUMetaTag;
+            if (!stop && !smem_wait_eq_bounded(tag, q, kWaitNs)) {
+                set_error(a.err, RSSM_DEVERR_TIMEOUT);
+                s_abort = 1;
+                stop = 1;
+            }
+            if (!stop && !mbar_wait_bounded(smem_u32(&full_bar[st]), use & 1, kWaitNs)) {
+                set_error(a.err, RSSM_DEVERR_TIMEOUT);
+                s_abort = 1;
+                stop = 1;
+                mbar_wait_bounded(smem_u32(&full_bar[st]), use & 1, kWaitNs);
+            }
+        }
+        if (group_sync_or(gi, CT, stop)) break;
+        const int u = meta[kUMetaPair];
+        if (u < 0) {  // end of this group's sequence: hand the stage back and stop
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+            break;
+        }
+        const int T = meta[kUMetaPos];
+        const uint32_t fc = static_cast<uint32_t>(meta[kUMetaFc]);
+        const int b = fdiv(static_cast<uint32_t>(u), lay.divPr), h0 = 2 * (u - b * hp);
+        if (cw < 2) {
+            // weights of head cw: lane l takes buffered token l (T <= 32)
+            const float Aj = reinterpret_cast<const float*>(meta)[kUMetaA0 + cw];
+            const float dts = (lane < T) ? reinterpret_cast<const float*>(sp + cw * lay.hb + lay.st_dt)[lane] : 0.f;
+            const float Sx = warp_prefix(dts);
+            const float Stot = T > 0 ? __shfl_sync(0xffffffffu, Sx, T - 1) : 0.f;
+            s_cw[gi][cw][lane] = (lane < T) ? dts * expf(Aj * (Stot - Sx)) : 0.f;
+            if (lane == 0) s_alpha[gi][cw] = expf(Aj * Stot);
+            if (cw == 0 && lane == 0) {
+                // every CTA read pos[b] before processing b's pairs; the last arrival resets it
+                if (pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 2)) {
+                    a.arrive[pend_b] = 0u;
+                    a.pos[pend_b] = 0;
+                    a.flush_count[pend_b] += 1u;
+                }
+                pend_b = b;
+                pend_old = atomicAdd(&a.arrive[b], 2u);
+            }
+        }
+        group_sync(gi, CT);  // weights ready
+        const int nks = (T + kFuK - 1) / kFuK;
+        for (int ks = 0; ks < nks; ++ks) {
+            // the previous K-step's MMAs have read the operands
+            if (ks > 0 && !mbar_wait_bounded(mbar, (ncommit - 1) & 1, kWaitNs)) timed_out = true;
+            // B operand: tokens 16 ks .. (zero past T) as column block n / 64,
+            // token row k, 16-byte chunk (n % 64) / 8 ^ (k & 7)
+            for (int i = ctid; i < kFuK * 16; i += CT) {
+                const int k = i >> 4, jn = i & 15, s = kFuK * ks + k;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (s < T) v = *reinterpret_cast<const uint4*>(sp + lay.brows + s * 256 + 16 * jn);
+                *reinterpret_cast<uint4*>(ops + 3 * kFuPart + (jn >> 3) * (kFuK * 128) + k * 128 +
+                                          16 * ((jn & 7) ^ (k & 7))) = v;
+            }
+            // A parts, x_w = w_s x_s[p] as bf16 hi + mid + lo, 8 rows at a time:
+            // item -> head i / 128, token (i / 8) % 16, rows 8 (i % 8) .. + 7
+            for (int i = ctid; i < 2 * kFuK * 8; i += CT) {
+                const int hh = i >> 7, k = (i >> 3) & (kFuK - 1), c = i & 7, s = kFuK * ks + k;
+                uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+                float w = 0.f;
+                if (s < T) {
+                    w = s_cw[gi][hh][s];
+                    xv = *reinterpret_cast<const uint4*>(sp + hh * lay.hb + lay.st_x + s * 128 + 16 * c);
+                }
+                const uint32_t xr[4] = {xv.x, xv.y, xv.z, xv.w};
+                uint32_t hi[4], md[4], lo[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float f0 = w * __uint_as_float(bf16lo_bits(xr[q]));
+                    const float f1 = w * __uint_as_float(bf16hi_bits(xr[q]));
+                    const uint32_t hh2 = f32x2_to_bf16x2(f0, f1);
+                    hi[q] = hh2;
+                    const float r0 = f0 - __uint_as_float(bf16lo_bits(hh2)), r1 = f1 - __uint_as_float(bf16hi_bits(hh2));
+                    const uint32_t mm = f32x2_to_bf16x2(r0, r1);
+                    md[q] = mm;
+                    lo[q] = f32x2_to_bf16x2(r0 - __uint_as_float(bf16lo_bits(mm)), r1 - __uint_as_float(bf16hi_bits(mm)));
+                }
+                // A part layout: [head][token k][128 B], 16-byte chunk (p / 8) ^ (k & 7)
+                const uint32_t d = static_cast<uint32_t>(hh * (kFuK * 128) + k * 128 + 16 * (c ^ (k & 7)));
+                *reinterpret_cast<uint4*>(ops + d) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(ops + kFuPart + d) = make_uint4(md[0], md[1], md[2], md[3]);
+                *reinterpret_cast<uint4*>(ops + 2 * kFuPart + d) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            // the operands written by ordinary stores, visible to the tensor cores
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            group_sync(gi, CT);
+            if (ctid == 0) {
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                // A: head blocks 64 rows apart in M (LBO = 16 x 128 B), 8-token atoms
+                // (SBO 1024 B); B: column blocks of 64 (LBO), 8-token atoms (SBO)
+                const uint64_t bd = umma_desc_sw128(ops_u + 3 * kFuPart, kFuK * 128, 1024);
+#pragma unroll
+                for (int part = 0; part < 3; ++part)
+                    umma_f16(tacc, umma_desc_sw128(ops_u + part * kFuPart, kFuK * 128, 1024), bd,
+                             (ks > 0 || part > 0) ? 1u : 0u);
+                umma_commit(mbar);
+            }
+            ++ncommit;
+        }
+        if (nks > 0) {
+            if (!mbar_wait_bounded(mbar, (ncommit - 1) & 1, kWaitNs)) timed_out = true;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        }
+        __syncwarp();  // converged for the warp-wide accumulator reads
+        {
+            // this thread's part of its row: v = exp(A S_T) h_0 + acc, 16 columns at a time
+            const float alpha = s_alpha[gi][jr];
+            const int hj = h0 + jr;
+            const size_t tj = static_cast<size_t>(b) * H + hj;
+            const unsigned char* tile = sp + jr * lay.hb;
+            const unsigned char* tsc = tile + (in_record ? a.rec.scales : align16(tile_bytes(UF, 64, kD128)));
+            unsigned char* updj = a.upd + tj * a.upd_stride;
+            unsigned char* recj = a.record + tj * a.rec.bytes;
+            uint32_t su0 = 0u, su1 = 0u, so0 = 0u, so1 = 0u;  // the FP4 block scales (update, output copy)
+            const PhiloxFixed pfix = philox_fixed(static_cast<uint32_t>(hj), static_cast<uint32_t>(b), fc, pkeys);
+            // unrolled by 2 only: the fully unrolled epilogue (32 Philox draws)
+            // outgrew the instruction cache (bf16 refresh 310 -> 234 us)
+#pragma unroll 2
+            for (int c8 = 0; c8 < NCC; ++c8) {
+                const int cc = cc0 + c8;
+                float v[16];
+                if (nks > 0) {
+                    tmem_ld16(trow + 16u * cc, v);
+                } else {
+                    // nothing buffered: fma(alpha, h, -0) is alpha h exactly, signed zeros included
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = -0.0f;
+                }
+                {
+                    float h[16];
+                    row16_load<UF>(tile, tsc, pr, cc, h);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = fmaf(alpha, h[i], v[i]);
+                }
+                const uint32_t e0 = static_cast<uint32_t>(pr * kD128 + 16 * cc);  // element of v[0] in the head
+                if constexpr (UF == kF32) {
+                    float* o = reinterpret_cast<float*>(updj) + e0;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        stream_store4(o + 4 * i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+                } else if constexpr (UF == kBF16 || UF == kE4M3) {
+                    uint32_t wv[UF == kBF16 ? 8 : 4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        // Philox counter (e/4, head, request, flush_count)
+                        const uint4 rw = philox4x32_10((e0 >> 2) + i, pfix, pkeys);
+                        if constexpr (UF == kBF16) {
+                            wv[2 * i] = sr_bf16(v[4 * i], rw.x) | (sr_bf16(v[4 * i + 1], rw.y) << 16);
+                            wv[2 * i + 1] = sr_bf16(v[4 * i + 2], rw.z) | (sr_bf16(v[4 * i + 3], rw.w) << 16);
+                        } else {
+                            wv[i] = sr_e4m3(v[4 * i], rw.x) | (sr_e4m3(v[4 * i + 1], rw.y) << 8) |
+                                    (sr_e4m3(v[4 * i + 2], rw.z) << 16) | (sr_e4m3(v[4 * i + 3], rw.w) << 24);
+                        }
+                    }
+                    if constexpr (UF == kBF16) {
+                        uint4* o = reinterpret_cast<uint4*>(updj + 2u * e0);
+                        o[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                        o[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+                    } else {
+                        *reinterpret_cast<uint4*>(updj + e0) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                    }
+                } else {
+                    uint32_t scv;
+                    *reinterpret_cast<uint2*>(updj + e0 / 2) = fp4_quant16(v, &scv);
+                    if (c8 < 4)
+                        su0 |= scv << (8 * c8);
+                    else
+                        su1 |= scv << (8 * (c8 - 4));
+                }
+                if constexpr (OUT4 != 0) {
+                    uint32_t scv;
+                    *reinterpret_cast<uint2*>(recj + e0 / 2) = fp4_quant16(v, &scv);
+                    if (c8 < 4)
+                        so0 |= scv << (8 * c8);
+                    else
+                        so1 |= scv << (8 * (c8 - 4));
+                }
+            }
+            // the block scales of this thread's columns: bytes cc0 .. cc0 + NCC - 1 of the row's 8
+            if constexpr (UF == kFP4) {
+                if constexpr (NCC == 8)
+                    *reinterpret_cast<uint2*>(updj + a.rec.scales + pr * 8) = make_uint2(su0, su1);
+                else
+                    *reinterpret_cast<uint32_t*>(updj + a.rec.scales + pr * 8 + cc0) = su0;
+            }
+            if constexpr (OUT4 != 0) {
+                if constexpr (NCC == 8)
+                    *reinterpret_cast<uint2*>(recj + a.rec.scales + pr * 8) = make_uint2(so0, so1);
+                else
+                    *reinterpret_cast<uint32_t*>(recj + a.rec.scales + pr * 8 + cc0) = so0;
+            }
+        }
+        if (timed_out && ctid == 0) {
+            set_error(a.err, RSSM_DEVERR_TIMEOUT);
+            s_abort = 1;
+        }
+        // the accumulator reads done before the group's next MMA; the stage back to the producer
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+        st += CG;
+        while (st >= S) {
+            st -= S;
+            ++use;
+        }
+    }
+    if (cw == 0 && lane == 0 && pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 2)) {
+        a.arrive[pend_b] = 0u;  // the last pending arrival of this group
+        a.pos[pend_b] = 0;
+        a.flush_count[pend_b] += 1u;
+    }
+    // no MMA of the group in flight (a timed-out wait is retried once), then
+    // every consumer is past its last accumulator read: free tensor memory
+    if (timed_out && ncommit > 0) mbar_wait_bounded(mbar, (ncommit - 1) & 1, kWaitNs);
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    asm volatile("bar.sync %0, %1;" ::"r"(CG + 1), "r"(CG * CT) : "memory");
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(fu_cols(UF)) : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Conventional scheme (in-run comparison, s1/s3): per token
 //   h <- exp(dt A) h + dt x B^T, write h, y = h C + D x.
 // VERIFY: read copy cur[b], write the state after token j to copy j.
@@ -2996,7 +3516,82 @@ static FoldPipeLayout fold_pipe_layout(const FoldArgs& a, int uf, int in_bf16, s
     return L;
 }
 
+// The tensor-core refresh (k_fold_umma): bf16 inputs, d_state 128, head_dim
+// 64, head pairs inside a group; the low-precision update copies, and an
+// fp32 update copy when it also writes the FP4 output copy.
+static bool fold_umma_shape(const FoldArgs& a, int in_bf16, int uf) {
+    return in_bf16 && a.s.N == kD128 && a.s.P == 64 && a.s.H % 2 == 0 && (a.s.H / a.s.G) % 2 == 0 &&
+           a.s.cap <= kMaxCap && (uf != kF32 || a.out_fp4) && !(uf == kFP4 && a.out_fp4);
+}
+
+// Stage layout of k_fold_umma: two head blocks (update copy (+ scales), dt
+// row, x rows: the record's offsets when the update copy is the record's own
+// copy), the group's B rows, meta. The groups' operand areas come first.
+static FoldUmmaLayout fold_umma_layout(const FoldArgs& a, int uf, size_t budget) {
+    const Shape& s = a.s;
+    FoldUmmaLayout L;
+    if (a.upd == a.record) {
+        L.st_dt = a.rec.dt;
+        L.st_x = a.rec.x;
+    } else {
+        L.st_dt = align16(align16(tile_bytes(uf, s.P, s.N)) + scale_bytes(uf, s.P, s.N));
+        L.st_x = L.st_dt + (a.rec.x - a.rec.dt);
+    }
+    L.hb = (L.st_x + static_cast<uint32_t>(s.cap * s.P) * 2u + 127u) & ~127u;
+    L.brows = 2u * L.hb;
+    L.meta = L.brows + align16(static_cast<uint32_t>(s.cap * s.N) * 2u);
+    L.stage_bytes = (L.meta + 64u + 127u) & ~127u;
+    const size_t ops = 1024 + static_cast<size_t>(fu_groups(uf)) * kFuOps;
+    const size_t n = budget > ops ? (budget - ops) / L.stage_bytes : 0;
+    L.stages = static_cast<int>(n < static_cast<size_t>(kPipeStagesMax) ? n : kPipeStagesMax);
+    L.divPr = make_fastdiv(static_cast<uint32_t>(s.H / 2));
+    L.divHpg = make_fastdiv(static_cast<uint32_t>(s.H / s.G));
+    L.keys = philox_keys(a.seed);
+    return L;
+}
+
+static cudaError_t fold_umma_dispatch(const FoldArgs& a, const FoldUmmaLayout& L, int uf, int grid, size_t smem,
+                                      cudaStream_t st) {
+    auto go = [&](auto kernel, int threads) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 static_cast<int>(cudaSharedmemCarveoutMaxShared));
+        if (e != cudaSuccess) return e;
+        return launch_pdl(kernel, grid, threads, smem, st, a, L);
+    };
+    if (a.out_fp4) {
+        switch (uf) {
+            case kF32: return go(k_fold_umma<kF32, 1>, fu_threads(kF32));
+            case kBF16: return go(k_fold_umma<kBF16, 1>, fu_threads(kBF16));
+            case kE4M3: return go(k_fold_umma<kE4M3, 1>, fu_threads(kE4M3));
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    switch (uf) {
+        case kBF16: return go(k_fold_umma<kBF16, 0>, fu_threads(kBF16));
+        case kE4M3: return go(k_fold_umma<kE4M3, 0>, fu_threads(kE4M3));
+        case kFP4: return go(k_fold_umma<kFP4, 0>, fu_threads(kFP4));
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 cudaError_t launch_fold(const FoldArgs& a, int in_bf16, int uf, cudaStream_t st) {
+    if (fold_umma_shape(a, in_bf16, uf)) {
+        const DeviceInfo di = device_info();
+        if (di.sms > 0) {
+            const size_t budget = di.smem_optin > 8192 ? di.smem_optin - 8192 : 0;
+            const FoldUmmaLayout L = fold_umma_layout(a, uf, budget);
+            if (L.stages >= fu_groups(uf)) {
+                const int npairs = a.s.batch * (a.s.H / 2);
+                if (npairs <= 0) return cudaSuccess;
+                const int grid = npairs < di.sms ? npairs : di.sms;
+                const size_t smem = 1024 + static_cast<size_t>(fu_groups(uf)) * kFuOps +
+                                    static_cast<size_t>(L.stages) * L.stage_bytes;
+                return fold_umma_dispatch(a, L, uf, grid, smem, st);
+            }
+        }
+    }
     if (a.s.N == 128 && a.s.P % 8 == 0) {
         const DeviceInfo di = device_info();
         if (di.sms > 0) {

@@ -79,10 +79,13 @@ def widened(kind, st):
 
 def f32_twin(shape, values, seed, in_dtype=torch.bfloat16, out_copy=True):
     """An fp32 update copy holding exactly `values` (fp32), with an FP4
-    output copy when out_copy. Refreshing it runs the same fold as the
-    low-precision state it shadows -- same inputs, same operation order --
+    output copy when out_copy. With the output copy, refreshing it runs the
+    refresh kernel of the low-precision state it shadows -- same inputs,
+    same operation order, the tensor-core fold where the shape takes it --
     and stores the fp32 result unrounded: that result is what the
-    low-precision refresh rounds."""
+    low-precision refresh rounds. Without it the refresh is the plain fp32
+    flush, whose fold (CUDA cores) may round differently; such a twin
+    serves for decode outputs and the fold's accuracy only."""
     desc = desc_for(shape, in_dtype, update_dtype=rssm.RSSM_F32,
                     out_copy=rssm.RSSM_OUTCOPY_FP4 if out_copy else rssm.RSSM_OUTCOPY_NONE, seed=seed)
     st = rssm.RssmState(desc)
@@ -118,11 +121,13 @@ def assert_refresh_bits(kind, seed, st, twin, fc_before, requests, what):
             assert bad == 0, f"{what}: request {b}: {bad} scales of the {name} differ"
 
 
-# d_state 64 runs the one-CTA-per-tile fold, d_state 128 the persistent pipelined one
-SHAPES = [LayerShape(3, 4, 32, 64, 2), LayerShape(3, 4, 32, 128, 2)]
+# d_state 64 runs the one-CTA-per-tile fold, d_state 128 the persistent
+# pipelined one; head_dim 64 with head pairs in a group the tensor-core one
+SHAPES = [LayerShape(3, 4, 32, 64, 2), LayerShape(3, 4, 32, 128, 2), LayerShape(3, 4, 64, 128, 2)]
+SHAPE_IDS = ["dstate64", "dstate128", "tensorcore"]
 
 
-@pytest.mark.parametrize("shape", SHAPES, ids=["dstate64", "dstate128"])
+@pytest.mark.parametrize("shape", SHAPES, ids=SHAPE_IDS)
 @pytest.mark.parametrize("kind", ["bf16", "e4m3", "f32"])
 def test_refresh_at_empty_buffer_builds_fp4_copy_bit_exact(kind, shape):
     inp = make_inputs(shape, 1, 30, torch.bfloat16, device="cuda")
@@ -376,7 +381,25 @@ def test_spec_b512_k4_on_split_state_sampled():
     assert refreshed >= 3
 
 
-@pytest.mark.parametrize("shape", SHAPES, ids=["dstate64", "dstate128"])
+@pytest.mark.parametrize("shape", SHAPES, ids=SHAPE_IDS)
+def test_shared_fp4_forced_refresh_requantises_bit_exact(shape):
+    """A forced refresh of the shared FP4 copy with an empty buffer folds
+    nothing (v = h_0, the dequantised copy): the re-quantised codes and
+    scales equal the oracle's FP4 quantisation of the dequantised values,
+    bit for bit (s4's shared-precision control)."""
+    Bz, H, P, N = shape.batch, shape.nheads, shape.head_dim, shape.d_state
+    inp = make_inputs(shape, 1, 33, torch.bfloat16, device="cuda")
+    desc, st = fp4_control_state(shape, inp, 6)
+    c0, s0 = st.ckpt.cpu().numpy(), st.ckpt_scales.cpu().numpy()
+    codes, scales = orc.fp4_quant(orc.widen(orc.FP4, c0, s0, (Bz, H, P, N)).astype(np.float32))
+    rssm.rssm_lowprec_refresh(st, inp["A"], force=True)
+    assert rssm.rssm_get_error(st) == 0
+    assert int(np.count_nonzero(st.ckpt.cpu().numpy() != codes.reshape(c0.shape))) == 0
+    assert int(np.count_nonzero(st.ckpt_scales.cpu().numpy() != scales.reshape(s0.shape))) == 0
+    assert st.flush_count.cpu().tolist() == [1] * Bz and st.pos.cpu().tolist() == [0] * Bz
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=SHAPE_IDS)
 def test_shared_fp4_control_decode_matches_oracle(shape):
     """The shared FP4 control (s4's ablation): decode reads the one FP4 copy
     and the refresh re-quantises it. Outputs match the oracle; the
@@ -391,16 +414,20 @@ def test_shared_fp4_control_decode_matches_oracle(shape):
     assert np.array_equal(st.ckpt.cpu().numpy(), codes0) and np.array_equal(st.ckpt_scales.cpu().numpy(), scales0)
     vals = orc.widen(orc.FP4, codes0, scales0, (Bz, H, P, N)).astype(np.float32)
     _, tw = f32_twin(shape, torch.from_numpy(vals).cuda(), 5, out_copy=False)
+    _, tf = f32_twin(shape, torch.from_numpy(vals).cuda(), 5)   # the refresh kernel's fp32 fold
     y = torch.empty((L, Bz, H, P), device="cuda")
     y2 = torch.empty_like(y)
+    y3 = torch.empty_like(y)
     for t in range(L):
         args = (inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"])
         rssm.rssm_decode_step(st, *args, y[t])
         rssm.rssm_decode_step(tw, *args, y2[t])
+        rssm.rssm_decode_step(tf, *args, y3[t])
     rssm.rssm_lowprec_refresh(st, inp["A"])
     rssm.rssm_lowprec_refresh(tw, inp["A"])
-    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
-    assert_refresh_bits("fp4", 5, st, tw, None, range(Bz), "shared FP4 refresh")
+    rssm.rssm_lowprec_refresh(tf, inp["A"])
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0 and rssm.rssm_get_error(tf) == 0
+    assert_refresh_bits("fp4", 5, st, tf, None, range(Bz), "shared FP4 refresh")
     for b in range(Bz):
         r = request_inputs(inp, b)
         req = orc.LowPrecRequest(orc.FP4, False, None, codes0[b], scales0[b], shape.ngroups, L, r["A"], r["D"], 5, b)
@@ -409,6 +436,7 @@ def test_shared_fp4_control_decode_matches_oracle(shape):
         assert_close(to_np(y2[:, b]), ys, f"fp32 twin decode, request {b}")
         v64 = req.refresh(want_v32=True).astype(np.float64)
         assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of the shared FP4 refresh, request {b}")
+        assert_close(to_np(tf.ckpt[b]), v64, f"fp32 fold of the refresh kernel, request {b}")
 
 
 def test_shared_fp4_control_split_b256_sampled():
@@ -434,16 +462,21 @@ def test_shared_fp4_control_split_b256_sampled():
         if b in reqs:
             codes0[b], scales0[b] = c, sc
     _, tw = f32_twin(shape, vals, seed, out_copy=False)
+    _, tf = f32_twin(shape, vals, seed)   # the refresh kernel's fp32 fold
+    del vals
     y = torch.empty((L, Bz, H, P), device="cuda")
     y2 = torch.empty_like(y)
+    y3 = torch.empty_like(y)
     for t in range(L):
         args = (inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"])
         rssm.rssm_decode_step(st, *args, y[t])
         rssm.rssm_decode_step(tw, *args, y2[t])
+        rssm.rssm_decode_step(tf, *args, y3[t])
     rssm.rssm_lowprec_refresh(st, inp["A"])
     rssm.rssm_lowprec_refresh(tw, inp["A"])
-    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
-    assert_refresh_bits("fp4", seed, st, tw, None, reqs, "shared FP4 refresh at split_b256")
+    rssm.rssm_lowprec_refresh(tf, inp["A"])
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0 and rssm.rssm_get_error(tf) == 0
+    assert_refresh_bits("fp4", seed, st, tf, None, reqs, "shared FP4 refresh at split_b256")
     for b in reqs:
         r = request_inputs(inp, b)
         req = orc.LowPrecRequest(orc.FP4, False, None, codes0[b], scales0[b], shape.ngroups, L, r["A"], r["D"],
@@ -452,6 +485,7 @@ def test_shared_fp4_control_split_b256_sampled():
         assert_close(to_np(y[:, b]), ys, f"shared FP4 decode at split_b256, request {b}")
         v64 = req.refresh(want_v32=True).astype(np.float64)
         assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of the shared FP4 refresh at split_b256, request {b}")
+        assert_close(to_np(tf.ckpt[b]), v64, f"fp32 fold of the refresh kernel at split_b256, request {b}")
 
 
 @pytest.mark.parametrize("shape", SPLIT_SHAPES, ids=SPLIT_IDS)
@@ -470,18 +504,22 @@ def test_shared_copy_decode_and_refresh_match_oracle(kind, shape):
     st = rssm.RssmState(desc)
     st.ckpt.copy_(initial_update_copy(inp["ckpt"], kind))
     _, tw = f32_twin(shape, widened(kind, st), seed, out_copy=False)
+    _, tf = f32_twin(shape, widened(kind, st), seed)   # the refresh kernel's fp32 fold
     upd0 = copy_bits(initial_update_copy(inp["ckpt"], kind))
     y = torch.empty((L, Bz, H, P), device="cuda")
     y2 = torch.empty_like(y)
+    y3 = torch.empty_like(y)
     for t in range(L):
         args = (inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"])
         rssm.rssm_decode_step(st, *args, y[t])
         rssm.rssm_decode_step(tw, *args, y2[t])
+        rssm.rssm_decode_step(tf, *args, y3[t])
     fc_before = st.flush_count.cpu().tolist()
     rssm.rssm_lowprec_refresh(st, inp["A"])
     rssm.rssm_lowprec_refresh(tw, inp["A"])
-    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
-    assert_refresh_bits(kind, seed, st, tw, fc_before, range(Bz), f"shared {kind} refresh")
+    rssm.rssm_lowprec_refresh(tf, inp["A"])
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0 and rssm.rssm_get_error(tf) == 0
+    assert_refresh_bits(kind, seed, st, tf, fc_before, range(Bz), f"shared {kind} refresh")
     for b in range(Bz):
         r = request_inputs(inp, b)
         req = orc.LowPrecRequest(UPD[kind][1], False, upd0[b], None, None, shape.ngroups, L, r["A"], r["D"], seed, b)
@@ -489,6 +527,7 @@ def test_shared_copy_decode_and_refresh_match_oracle(kind, shape):
         assert_close(to_np(y[:, b]), ys, f"shared {kind} decode, request {b}")
         v64 = req.refresh(want_v32=True).astype(np.float64)
         assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of the shared {kind} refresh, request {b}")
+        assert_close(to_np(tf.ckpt[b]), v64, f"fp32 fold of the refresh kernel, request {b}")
     assert st.flush_count.cpu().tolist() == [1] * Bz and st.pos.cpu().tolist() == [0] * Bz
 
 
@@ -509,17 +548,19 @@ def test_speculative_verify_on_shared_copy_matches_oracle(kind, K):
     st = rssm.RssmState(desc)
     st.ckpt.copy_(initial_update_copy(inp["ckpt"], kind))
     _, tw = f32_twin(shape, widened(kind, st), seed, out_copy=False)
+    _, tf = f32_twin(shape, widened(kind, st), seed)   # the refresh kernel's fp32 fold
     upd0 = copy_bits(initial_update_copy(inp["ckpt"], kind))
     y = torch.empty((steps, shape.batch, K + 1, shape.nheads, shape.head_dim), device="cuda")
     y2 = torch.empty_like(y)
+    y3 = torch.empty_like(y)
     fc_before = st.flush_count.cpu().tolist()
     for s in range(steps):
         args = (inp["x"][s], inp["B"][s], inp["C"][s], inp["dt"][s], inp["A"], inp["D"])
-        for state, out in ((st, y), (tw, y2)):
+        for state, out in ((st, y), (tw, y2), (tf, y3)):
             rssm.rssm_verify(state, K, *args, out[s])
             rssm.rssm_accept(state, n_acc[s])
             rssm.rssm_lowprec_refresh(state, inp["A"])
-    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0 and rssm.rssm_get_error(tf) == 0
     folded = []
     for b in range(shape.batch):
         r = request_inputs(inp, b)
@@ -535,7 +576,7 @@ def test_speculative_verify_on_shared_copy_matches_oracle(kind, K):
                 folded.append(b)
         assert st.pos[b].item() == req.pos
     assert len(folded) == 3
-    assert_refresh_bits(kind, seed, st, tw, fc_before, folded, f"speculative shared {kind} refresh")
+    assert_refresh_bits(kind, seed, st, tf, fc_before, folded, f"speculative shared {kind} refresh")
 
 
 def run_lowprec(desc, st, inp, steps):
