@@ -245,12 +245,18 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, const PhiloxFixed& F
 // |v| = q (m + f) with q the target spacing at |v|; the magnitude rounds up
 // iff r < floor(f * 2^32). Worked on the fp32 bit pattern.
 
-// bf16 keeps the top 16 bits of fp32, so f * 2^16 is the low 16 bits.
-__device__ __forceinline__ uint32_t sr_bf16(float v, uint32_t r) {
-    const uint32_t u = __float_as_uint(v);
-    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (u >> 16) | 0x40u;  // NaN stays NaN
-    return (u >> 16) + ((r >> 16) < (u & 0xFFFFu) ? 1u : 0u);
+// bf16 keeps the top 16 bits of fp32, so f * 2^16 is the low 16 bits L and
+// the result is (u >> 16) + [(r >> 16) < L]. One add forms it: L + 0xFFFF -
+// (r >> 16) reaches 2^16 exactly when (r >> 16) < L, so the carry into the
+// high half is the rounding increment. Two values packed into one word
+// (v0 in the low half); a NaN stays a NaN (quiet bit set).
+__device__ __forceinline__ uint32_t sr_bf16x2(float v0, float v1, uint32_t r0, uint32_t r1) {
+    const uint32_t u0 = __float_as_uint(v0), u1 = __float_as_uint(v1);
+    const uint32_t t0 = (v0 != v0) ? (u0 | 0x00400000u) : u0 + (0xFFFFu - (r0 >> 16));
+    const uint32_t t1 = (v1 != v1) ? (u1 | 0x00400000u) : u1 + (0xFFFFu - (r1 >> 16));
+    return __byte_perm(t0, t1, 0x7632);  // the high halves of t0, t1
 }
+
 
 // OCP e4m3 ("fn"): bias 7, spacing 2^(E-3) for |v| >= 2^-6, 2^-9 below;
 // |v| >= 448 (and inf) saturates to 448, NaN -> 0x7F.
@@ -265,10 +271,12 @@ __device__ __forceinline__ uint32_t sr_e4m3(float v, uint32_t r) {
         // normal: the exponent and top 3 mantissa bits re-biased (127 -> 7);
         // the 20 bits below them are the fraction
         code = (a >> 20) - (120u << 3);
-        F = (a & 0xFFFFFu) << 12;
+        F = a << 12;
     } else {
         // below 2^-6: t = |v| 2^9 < 8 is exact, code = floor(t), and the
-        // fraction scaled by 2^32 is exact too (at most 24 significant bits)
+        // fraction scaled by 2^32 is exact too (at most 24 significant bits).
+        // Float arithmetic on purpose: an integer-only form (a 32.32
+        // fixed-point shift) costs more ALU issue, the refresh's bound.
         const float t = __uint_as_float(a) * 512.0f;
         const float m = truncf(t);
         code = static_cast<uint32_t>(m);

@@ -1608,8 +1608,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_fold(const FoldArgs a) {
                 // Philox counter (e/4, head, request, flush_count)
                 const uint4 rw = philox4x32_10(make_uint4(e >> 2, h, b, fc), pkeys);
                 if constexpr (UF == kBF16) {
-                    const uint2 w = make_uint2(sr_bf16(v.x, rw.x) | (sr_bf16(v.y, rw.y) << 16),
-                                               sr_bf16(v.z, rw.z) | (sr_bf16(v.w, rw.w) << 16));
+                    const uint2 w = make_uint2(sr_bf16x2(v.x, v.y, rw.x, rw.y), sr_bf16x2(v.z, v.w, rw.z, rw.w));
                     *reinterpret_cast<uint2*>(upd + 2u * e) = w;
                 } else {
                     const uint32_t w = sr_e4m3(v.x, rw.x) | (sr_e4m3(v.y, rw.y) << 8) |
@@ -1935,8 +1934,7 @@ __global__ void __launch_bounds__(fold_threads(UF), 1) k_fold_pipe(const FoldArg
                 } else if constexpr (UF == kBF16 || UF == kE4M3) {
                     const uint4 rw = philox4x32_10(make_uint4(e >> 2, h, b, fc), pkeys);
                     if constexpr (UF == kBF16) {
-                        const uint2 wv = make_uint2(sr_bf16(v.x, rw.x) | (sr_bf16(v.y, rw.y) << 16),
-                                                    sr_bf16(v.z, rw.z) | (sr_bf16(v.w, rw.w) << 16));
+                        const uint2 wv = make_uint2(sr_bf16x2(v.x, v.y, rw.x, rw.y), sr_bf16x2(v.z, v.w, rw.z, rw.w));
                         *reinterpret_cast<uint2*>(upd + 2u * e) = wv;
                     } else {
                         const uint32_t wv = sr_e4m3(v.x, rw.x) | (sr_e4m3(v.y, rw.y) << 8) |
@@ -2650,8 +2648,6 @@ __global__ void __launch_bounds__(fu_threads(UF), 1) k_fold_umma(const FoldArgs 
     __shared__ __align__(8) uint64_t full_bar[kPipeStagesMax];
     __shared__ __align__(8) uint64_t empty_bar[kPipeStagesMax];
     __shared__ __align__(8) uint64_t mma_bar[CG];
-    __shared__ float s_cw[CG][2][kMaxCap];  // dt_s exp(A_j (S_T - S_s)) of head j of the group's pair
-    __shared__ float s_alpha[CG][2];        // exp(A_j S_T)
     __shared__ uint32_t s_tmem;
     __shared__ volatile int s_abort;
 
@@ -2858,26 +2854,28 @@ __global__ void __launch_bounds__(fu_threads(UF), 1) k_fold_umma(const FoldArgs 
         const int T = meta[kUMetaPos];
         const uint32_t fc = static_cast<uint32_t>(meta[kUMetaFc]);
         const int b = fdiv(static_cast<uint32_t>(u), lay.divPr), h0 = 2 * (u - b * hp);
-        if (cw < 2) {
-            // weights of head cw: lane l takes buffered token l (T <= 32)
-            const float Aj = reinterpret_cast<const float*>(meta)[kUMetaA0 + cw];
-            const float dts = (lane < T) ? reinterpret_cast<const float*>(sp + cw * lay.hb + lay.st_dt)[lane] : 0.f;
+        // both heads' weights dt_s exp(A_j (S_T - S_s)) and exp(A_j S_T), in
+        // every warp (no barrier): lane l takes buffered token l (T <= 32)
+        float wl[2], alpha2[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const float Aj = reinterpret_cast<const float*>(meta)[kUMetaA0 + j];
+            const float dts = (lane < T) ? reinterpret_cast<const float*>(sp + j * lay.hb + lay.st_dt)[lane] : 0.f;
             const float Sx = warp_prefix(dts);
             const float Stot = T > 0 ? __shfl_sync(0xffffffffu, Sx, T - 1) : 0.f;
-            s_cw[gi][cw][lane] = (lane < T) ? dts * expf(Aj * (Stot - Sx)) : 0.f;
-            if (lane == 0) s_alpha[gi][cw] = expf(Aj * Stot);
-            if (cw == 0 && lane == 0) {
-                // every CTA read pos[b] before processing b's pairs; the last arrival resets it
-                if (pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 2)) {
-                    a.arrive[pend_b] = 0u;
-                    a.pos[pend_b] = 0;
-                    a.flush_count[pend_b] += 1u;
-                }
-                pend_b = b;
-                pend_old = atomicAdd(&a.arrive[b], 2u);
-            }
+            wl[j] = (lane < T) ? dts * expf(Aj * (Stot - Sx)) : 0.f;
+            alpha2[j] = expf(Aj * Stot);
         }
-        group_sync(gi, CT);  // weights ready
+        if (cw == 0 && lane == 0) {
+            // every CTA read pos[b] before processing b's pairs; the last arrival resets it
+            if (pend_b >= 0 && pend_old == static_cast<uint32_t>(H - 2)) {
+                a.arrive[pend_b] = 0u;
+                a.pos[pend_b] = 0;
+                a.flush_count[pend_b] += 1u;
+            }
+            pend_b = b;
+            pend_old = atomicAdd(&a.arrive[b], 2u);
+        }
         const int nks = (T + kFuK - 1) / kFuK;
         for (int ks = 0; ks < nks; ++ks) {
             // the previous K-step's MMAs have read the operands
@@ -2895,10 +2893,11 @@ __global__ void __launch_bounds__(fu_threads(UF), 1) k_fold_umma(const FoldArgs 
             // item -> head i / 128, token (i / 8) % 16, rows 8 (i % 8) .. + 7
             for (int i = ctid; i < 2 * kFuK * 8; i += CT) {
                 const int hh = i >> 7, k = (i >> 3) & (kFuK - 1), c = i & 7, s = kFuK * ks + k;
+                const float w0 = __shfl_sync(0xffffffffu, wl[0], s), w1 = __shfl_sync(0xffffffffu, wl[1], s);
                 uint4 xv = make_uint4(0u, 0u, 0u, 0u);
                 float w = 0.f;
                 if (s < T) {
-                    w = s_cw[gi][hh][s];
+                    w = hh ? w1 : w0;
                     xv = *reinterpret_cast<const uint4*>(sp + hh * lay.hb + lay.st_x + s * 128 + 16 * c);
                 }
                 const uint32_t xr[4] = {xv.x, xv.y, xv.z, xv.w};
@@ -2943,7 +2942,7 @@ __global__ void __launch_bounds__(fu_threads(UF), 1) k_fold_umma(const FoldArgs 
         __syncwarp();  // converged for the warp-wide accumulator reads
         {
             // this thread's part of its row: v = exp(A S_T) h_0 + acc, 16 columns at a time
-            const float alpha = s_alpha[gi][jr];
+            const float alpha = jr ? alpha2[1] : alpha2[0];
             const int hj = h0 + jr;
             const size_t tj = static_cast<size_t>(b) * H + hj;
             const unsigned char* tile = sp + jr * lay.hb;
@@ -2984,8 +2983,8 @@ __global__ void __launch_bounds__(fu_threads(UF), 1) k_fold_umma(const FoldArgs 
                         // Philox counter (e/4, head, request, flush_count)
                         const uint4 rw = philox4x32_10((e0 >> 2) + i, pfix, pkeys);
                         if constexpr (UF == kBF16) {
-                            wv[2 * i] = sr_bf16(v[4 * i], rw.x) | (sr_bf16(v[4 * i + 1], rw.y) << 16);
-                            wv[2 * i + 1] = sr_bf16(v[4 * i + 2], rw.z) | (sr_bf16(v[4 * i + 3], rw.w) << 16);
+                            wv[2 * i] = sr_bf16x2(v[4 * i], v[4 * i + 1], rw.x, rw.y);
+                            wv[2 * i + 1] = sr_bf16x2(v[4 * i + 2], v[4 * i + 3], rw.z, rw.w);
                         } else {
                             wv[i] = sr_e4m3(v[4 * i], rw.x) | (sr_e4m3(v[4 * i + 1], rw.y) << 8) |
                                     (sr_e4m3(v[4 * i + 2], rw.z) << 16) | (sr_e4m3(v[4 * i + 3], rw.w) << 24);
@@ -3192,7 +3191,15 @@ __global__ void k_round_test(int op, int64_t n, const float* v, uint64_t seed, u
                                    make_uint2(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32)));
     const uint32_t r = (i & 3) == 0 ? rw.x : (i & 3) == 1 ? rw.y : (i & 3) == 2 ? rw.z : rw.w;
     switch (op) {
-        case 0: static_cast<uint16_t*>(out)[i] = static_cast<uint16_t>(sr_bf16(v[i], r)); break;
+        case 0: {
+            // the packed pair the refresh kernels use: elements i & ~1 and i | 1
+            const bool hi = (i & 1) != 0;
+            const float v0 = v[i & ~static_cast<int64_t>(1)], v1 = (i | 1) < n ? v[i | 1] : 0.0f;
+            const uint32_t r0 = (i & 2) ? rw.z : rw.x, r1 = (i & 2) ? rw.w : rw.y;
+            const uint32_t w = sr_bf16x2(v0, v1, r0, r1);
+            static_cast<uint16_t*>(out)[i] = static_cast<uint16_t>(hi ? w >> 16 : w & 0xFFFFu);
+            break;
+        }
         case 1: static_cast<uint8_t*>(out)[i] = static_cast<uint8_t>(sr_e4m3(v[i], r)); break;
         case 2: static_cast<uint8_t*>(out)[i] = static_cast<uint8_t>(e4m3_rn(v[i])); break;
         default: static_cast<uint32_t*>(out)[i] = r; break;
