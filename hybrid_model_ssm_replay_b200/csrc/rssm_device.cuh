@@ -258,6 +258,7 @@ __device__ __forceinline__ uint32_t sr_bf16x2(float v0, float v1, uint32_t r0, u
 }
 
 
+
 // OCP e4m3 ("fn"): bias 7, spacing 2^(E-3) for |v| >= 2^-6, 2^-9 below;
 // |v| >= 448 (and inf) saturates to 448, NaN -> 0x7F.
 __device__ __forceinline__ uint32_t sr_e4m3(float v, uint32_t r) {
@@ -277,6 +278,24 @@ __device__ __forceinline__ uint32_t sr_e4m3(float v, uint32_t r) {
         // fraction scaled by 2^32 is exact too (at most 24 significant bits).
         // Float arithmetic on purpose: an integer-only form (a 32.32
         // fixed-point shift) costs more ALU issue, the refresh's bound.
+        const float t = __uint_as_float(a) * 512.0f;
+        const float m = truncf(t);
+        code = static_cast<uint32_t>(m);
+        F = __float2uint_rz((t - m) * 4294967296.0f);
+    }
+    return sign | (code + (r < F ? 1u : 0u));
+}
+
+// sr_e4m3 for |v| < 448 (not NaN, no saturation).
+__device__ __forceinline__ uint32_t sr_e4m3_in_range(float v, uint32_t r) {
+    const uint32_t u = __float_as_uint(v);
+    const uint32_t sign = (u >> 24) & 0x80u;
+    const uint32_t a = u & 0x7FFFFFFFu;
+    uint32_t code, F;
+    if (a >= 0x3C800000u) {
+        code = (a >> 20) - (120u << 3);
+        F = a << 12;
+    } else {
         const float t = __uint_as_float(a) * 512.0f;
         const float m = truncf(t);
         code = static_cast<uint32_t>(m);
@@ -450,17 +469,31 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float* v, float m) {
     return out;
 }
 
-// FP4 copy of one block of 16 contiguous values held by one thread: the
-// scale and codes of fp4_quant_quad (the same bracketed quotients), with
-// the block maximum taken in registers. Returns the 64 code bits, element i
-// in nibble i % 8 of word i / 8, and sets *scale_code.
-__device__ __forceinline__ uint2 fp4_quant16(const float (&v)[16], uint32_t* scale_code) {
+// max(|v_i|) over a block of 16 held by one thread: with fmaxf (NaN values
+// ignored, as the FP4 scale takes them) or NaN-propagating (NaN iff some v_i
+// is NaN, else the same value).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+    float d;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+template <bool NAN_PROPAGATES>
+__device__ __forceinline__ float absmax16(const float (&v)[16]) {
+    auto mx = [](float a, float b) { return NAN_PROPAGATES ? fmax_nan(a, b) : fmaxf(a, b); };
     float m8[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(v[i]), fabsf(v[i + 8]));
+    for (int i = 0; i < 8; ++i) m8[i] = mx(fabsf(v[i]), fabsf(v[i + 8]));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) m8[i] = fmaxf(m8[i], m8[i + 4]);
-    const float amax = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
+    for (int i = 0; i < 4; ++i) m8[i] = mx(m8[i], m8[i + 4]);
+    return mx(mx(m8[0], m8[2]), mx(m8[1], m8[3]));
+}
+
+// FP4 copy of one block of 16 contiguous values held by one thread: the
+// scale and codes of fp4_quant_quad (the same bracketed quotients), with
+// the block maximum (NaN values ignored) given or taken in registers.
+// Returns the 64 code bits, element i in nibble i % 8 of word i / 8, and
+// sets *scale_code.
+__device__ __forceinline__ uint2 fp4_quant16(const float (&v)[16], float amax, uint32_t* scale_code) {
     constexpr float kSixthLo = 0x1.555554p-3f, kSixthHi = 0x1.555556p-3f;  // adjacent floats around 1/6
     uint32_t sc = e4m3_rn(amax * kSixthLo);
     if (sc != e4m3_rn(amax * kSixthHi)) sc = e4m3_rn(__fdiv_rn(amax, 6.0f));
@@ -477,6 +510,10 @@ __device__ __forceinline__ uint2 fp4_quant16(const float (&v)[16], uint32_t* sca
 #pragma unroll
     for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(v[i], s);
     return make_uint2(e2m1x8_rn(q, 1.0f), e2m1x8_rn(q + 8, 1.0f));
+}
+
+__device__ __forceinline__ uint2 fp4_quant16(const float (&v)[16], uint32_t* scale_code) {
+    return fp4_quant16(v, absmax16<false>(v), scale_code);
 }
 
 }  // namespace rssm

@@ -2971,12 +2971,22 @@ __global__ void __launch_bounds__(fu_threads(UF), 1) k_fold_umma(const FoldArgs 
                     for (int i = 0; i < 16; ++i) v[i] = fmaf(alpha, h[i], v[i]);
                 }
                 const uint32_t e0 = static_cast<uint32_t>(pr * kD128 + 16 * cc);  // element of v[0] in the head
+                float amax = 0.f;  // the block's max |v| (FP4 scale)
                 if constexpr (UF == kF32) {
                     float* o = reinterpret_cast<float*>(updj) + e0;
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         stream_store4(o + 4 * i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
                 } else if constexpr (UF == kBF16 || UF == kE4M3) {
+                    // e4m3: the block's NaN-propagating |max| (shared with the FP4
+                    // scale below); below 448, no value of the block needs the
+                    // rounding's special cases (NaN, infinity, saturation). (bf16
+                    // keeps its per-value NaN select: a block test measured slower.)
+                    bool plain = false;
+                    if constexpr (UF == kE4M3) {
+                        amax = absmax16<true>(v);
+                        plain = amax < 448.0f;
+                    }
                     uint32_t wv[UF == kBF16 ? 8 : 4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
@@ -2985,6 +2995,10 @@ __global__ void __launch_bounds__(fu_threads(UF), 1) k_fold_umma(const FoldArgs 
                         if constexpr (UF == kBF16) {
                             wv[2 * i] = sr_bf16x2(v[4 * i], v[4 * i + 1], rw.x, rw.y);
                             wv[2 * i + 1] = sr_bf16x2(v[4 * i + 2], v[4 * i + 3], rw.z, rw.w);
+                        } else if (plain) {
+                            wv[i] = sr_e4m3_in_range(v[4 * i], rw.x) | (sr_e4m3_in_range(v[4 * i + 1], rw.y) << 8) |
+                                    (sr_e4m3_in_range(v[4 * i + 2], rw.z) << 16) |
+                                    (sr_e4m3_in_range(v[4 * i + 3], rw.w) << 24);
                         } else {
                             wv[i] = sr_e4m3(v[4 * i], rw.x) | (sr_e4m3(v[4 * i + 1], rw.y) << 8) |
                                     (sr_e4m3(v[4 * i + 2], rw.z) << 16) | (sr_e4m3(v[4 * i + 3], rw.w) << 24);
@@ -3007,7 +3021,12 @@ __global__ void __launch_bounds__(fu_threads(UF), 1) k_fold_umma(const FoldArgs 
                 }
                 if constexpr (OUT4 != 0) {
                     uint32_t scv;
-                    *reinterpret_cast<uint2*>(recj + e0 / 2) = fp4_quant16(v, &scv);
+                    if constexpr (UF == kE4M3) {
+                        if (amax != amax) amax = absmax16<false>(v);  // a NaN value: the scale ignores it
+                    } else {
+                        amax = absmax16<false>(v);
+                    }
+                    *reinterpret_cast<uint2*>(recj + e0 / 2) = fp4_quant16(v, amax, &scv);
                     if (c8 < 4)
                         so0 |= scv << (8 * c8);
                     else
