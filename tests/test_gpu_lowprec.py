@@ -241,6 +241,49 @@ def test_split_b256_full_size_sampled(kind):
     assert st.flush_count.cpu().tolist() == [2] * Bz
 
 
+@pytest.mark.parametrize("T", [1, 15, 17, 32])
+@pytest.mark.parametrize("kind", ["bf16", "e4m3"])
+def test_tensor_core_refresh_at_each_buffer_fill(kind, T):
+    """The tensor-core refresh (head_dim 64, head pairs in a group) folds 16
+    buffered tokens per MMA K-step. A forced refresh after T decodes (T = 1
+    and 15: one partial step; 17: a full step and a one-token step; 32: two
+    full steps, the buffer's capacity) leaves update and FP4 copies equal,
+    bit for bit, to the oracle's rounding of the fp32 fold of a twin running
+    the same kernel, and that fold matches the oracle's fp64 fold; the
+    outputs read from the FP4 copy match the oracle."""
+    shape = LayerShape(3, 4, 64, 128, 2, interval=25, max_draft=7)   # capacity 32, the most a buffer holds
+    Bz, H, P = shape.batch, shape.nheads, shape.head_dim
+    inp = make_inputs(shape, T, 37, torch.bfloat16, device="cuda")
+    seed = 0xF00D
+    desc, st = split_state(shape, inp, kind, seed)
+    _, tw = f32_twin(shape, widened(kind, st), seed)
+    rssm.rssm_lowprec_refresh(tw, inp["A"], force=True)
+    upd0 = copy_bits(initial_update_copy(inp["ckpt"], kind))
+    codes0, scales0 = orc.fp4_quant(orc.widen(UPD[kind][1], upd0, None, upd0.shape).astype(np.float32))
+    y = torch.empty((T, Bz, H, P), device="cuda")
+    y2 = torch.empty_like(y)
+    for t in range(T):
+        args = (inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"])
+        rssm.rssm_decode_step(st, *args, y[t])
+        rssm.rssm_decode_step(tw, *args, y2[t])
+    assert torch.equal(y, y2)                       # both read the same FP4 copy
+    fc_before = st.flush_count.cpu().tolist()
+    rssm.rssm_lowprec_refresh(st, inp["A"], force=True)
+    rssm.rssm_lowprec_refresh(tw, inp["A"], force=True)
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
+    assert_refresh_bits(kind, seed, st, tw, fc_before, range(Bz), f"{kind} + FP4 refresh of {T} entries")
+    for b in range(Bz):
+        r = request_inputs(inp, b)
+        req = orc.LowPrecRequest(UPD[kind][1], True, upd0[b], codes0[b], scales0[b], shape.ngroups, 32, r["A"],
+                                 r["D"], seed, b)
+        req.flush_count.value = 1
+        ys = np.stack([req.decode(r["x"][t], r["B"][t], r["C"][t], r["dt"][t]) for t in range(T)])
+        assert_close(to_np(y[:, b]), ys, f"FP4-copy decode, {T} tokens, request {b}")
+        v64 = req.refresh(want_v32=True).astype(np.float64)
+        assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold of {T} entries, request {b}")
+    assert st.pos.cpu().tolist() == [0] * Bz and st.flush_count.cpu().tolist() == [2] * Bz
+
+
 # accepted drafts per step and request (steps x batch) for K = 4 and K = 6:
 # three requests reach the interval on the last step, one does not
 SPLIT_SPEC = {
