@@ -3047,7 +3047,7 @@ __global__ void __launch_bounds__(fu_threads(UF), 1) k_fold_umma(const FoldArgs 
                     *reinterpret_cast<uint32_t*>(recj + a.rec.scales + pr * 8 + cc0) = so0;
             }
         }
-        if (timed_out && ctid == 0) {
+        if (timed_out) {  // any thread whose wait ran out (first error wins)
             set_error(a.err, RSSM_DEVERR_TIMEOUT);
             s_abort = 1;
         }
