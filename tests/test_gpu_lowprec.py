@@ -574,6 +574,46 @@ def test_shared_copy_decode_and_refresh_match_oracle(kind, shape):
     assert st.flush_count.cpu().tolist() == [1] * Bz and st.pos.cpu().tolist() == [0] * Bz
 
 
+def test_shared_bf16_control_split_b256_sampled():
+    """The shared bf16 control (one bf16 copy read by decode and updated
+    with stochastic rounding) at the bench's size (split_b256) and launch
+    configuration: one interval of decodes, then the refresh, beside an
+    fp32 twin with an FP4 output copy that runs the same refresh kernel.
+    For sampled requests the outputs match the oracle reading the same
+    copy, the twin's fold matches the oracle's fp64 fold, and the refreshed
+    copy equals the oracle's rounding of that fold bit for bit."""
+    w = WORKLOADS["split_b256"]
+    shape = w["shape"]
+    L = shape.interval
+    Bz, H, P = shape.batch, shape.nheads, shape.head_dim
+    inp = make_inputs(shape, L, w["seed"], w["in_dtype"], device="cuda")
+    seed = w["seed"]
+    st = rssm.RssmState(desc_for(shape, update_dtype=rssm.RSSM_BF16, seed=seed))
+    st.ckpt.copy_(initial_update_copy(inp["ckpt"], "bf16"))
+    _, tf = f32_twin(shape, widened("bf16", st), seed)   # the refresh kernel's fp32 fold
+    y = torch.empty((L, Bz, H, P), device="cuda")
+    y2 = torch.empty_like(y)
+    for t in range(L):
+        args = (inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"])
+        rssm.rssm_decode_step(st, *args, y[t])
+        rssm.rssm_decode_step(tf, *args, y2[t])
+    fc_before = st.flush_count.cpu().tolist()
+    rssm.rssm_lowprec_refresh(st, inp["A"])
+    rssm.rssm_lowprec_refresh(tf, inp["A"])
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tf) == 0
+    reqs = sample_requests(Bz, 6)
+    assert_refresh_bits("bf16", seed, st, tf, fc_before, reqs, "shared bf16 refresh at split_b256")
+    for b in reqs:
+        upd0 = copy_bits(initial_update_copy(inp["ckpt"][b], "bf16"))
+        r = request_inputs(inp, b)
+        req = orc.LowPrecRequest(orc.BF16, False, upd0, None, None, shape.ngroups, L, r["A"], r["D"], seed, b)
+        ys = np.stack([req.decode(r["x"][t], r["B"][t], r["C"][t], r["dt"][t]) for t in range(L)])
+        assert_close(to_np(y[:, b]), ys, f"shared bf16 decode at split_b256, request {b}")
+        v64 = req.refresh(want_v32=True).astype(np.float64)
+        assert_close(to_np(tf.ckpt[b]), v64, f"fp32 fold of the shared bf16 refresh at split_b256, request {b}")
+    assert st.flush_count.cpu().tolist() == [1] * Bz and st.pos.cpu().tolist() == [0] * Bz
+
+
 @pytest.mark.parametrize("K", [4, 6])
 @pytest.mark.parametrize("kind", ["bf16", "e4m3"])
 def test_speculative_verify_on_shared_copy_matches_oracle(kind, K):
