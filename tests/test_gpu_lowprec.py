@@ -284,6 +284,44 @@ def test_tensor_core_refresh_at_each_buffer_fill(kind, T):
     assert st.pos.cpu().tolist() == [0] * Bz and st.flush_count.cpu().tolist() == [2] * Bz
 
 
+@pytest.mark.parametrize("batch", [1, 5])
+def test_tensor_core_refresh_single_pair_requests(batch):
+    """Degenerate launches of the tensor-core refresh: requests of one head
+    pair (2 heads, 1 group), so the grid is batch CTAs, most consumer groups
+    get only their end marker, and each request's arrival count reaches H
+    with one pair. One interval: bf16 + FP4 copies bit-exact against the
+    oracle's rounding of the fp32 twin's fold, that fold against the oracle's
+    fp64 fold, positions reset and flush counts advanced."""
+    shape = LayerShape(batch, 2, 64, 128, 1)
+    L = shape.interval
+    inp = make_inputs(shape, L, 38, torch.bfloat16, device="cuda")
+    seed = 0xABBA
+    desc, st = split_state(shape, inp, "bf16", seed)
+    _, tw = f32_twin(shape, widened("bf16", st), seed)
+    rssm.rssm_lowprec_refresh(tw, inp["A"], force=True)
+    upd0 = copy_bits(initial_update_copy(inp["ckpt"], "bf16"))
+    codes0, scales0 = orc.fp4_quant(orc.widen(orc.BF16, upd0, None, upd0.shape).astype(np.float32))
+    y = torch.empty((L, batch, 2, 64), device="cuda")
+    for t in range(L):
+        args = (inp["x"][t], inp["B"][t], inp["C"][t], inp["dt"][t], inp["A"], inp["D"])
+        rssm.rssm_decode_step(st, *args, y[t])
+        rssm.rssm_decode_step(tw, *args, y[t])
+    fc_before = st.flush_count.cpu().tolist()
+    rssm.rssm_lowprec_refresh(st, inp["A"])
+    rssm.rssm_lowprec_refresh(tw, inp["A"])
+    assert rssm.rssm_get_error(st) == 0 and rssm.rssm_get_error(tw) == 0
+    assert_refresh_bits("bf16", seed, st, tw, fc_before, range(batch), "single-pair refresh")
+    for b in range(batch):
+        r = request_inputs(inp, b)
+        req = orc.LowPrecRequest(orc.BF16, True, upd0[b], codes0[b], scales0[b], 1, L, r["A"], r["D"], seed, b)
+        req.flush_count.value = 1
+        for t in range(L):
+            req.decode(r["x"][t], r["B"][t], r["C"][t], r["dt"][t])
+        v64 = req.refresh(want_v32=True).astype(np.float64)
+        assert_close(to_np(tw.ckpt[b]), v64, f"fp32 fold, single-pair request {b}")
+    assert st.pos.cpu().tolist() == [0] * batch and st.flush_count.cpu().tolist() == [2] * batch
+
+
 # accepted drafts per step and request (steps x batch) for K = 4 and K = 6:
 # three requests reach the interval on the last step, one does not
 SPLIT_SPEC = {
