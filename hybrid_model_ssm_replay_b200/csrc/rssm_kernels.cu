@@ -2547,18 +2547,21 @@ __global__ void __launch_bounds__(kUmThreads, 3) k_prefill_umma(const PrefillArg
 // head_dim, 64..127 the second's). One persistent CTA per SM: a producer
 // warp brings each due pair into a stage (both update copies, dt and x
 // rows, the group's B rows; bulk copies on an mbarrier ring, as in
-// k_fold_pipe) and consumer groups of four warps take the pairs in turn:
-//  - warps 0 and 1 form the two heads' weights, then the group builds one
-//    K-step's operands: X_w split into bf16 hi + mid + lo (~2^-27
-//    relative) and the B rows (exact in bf16), MN-major in 128-byte-swizzled
-//    atoms, zero past T;
+// k_fold_pipe) and consumer groups of four or eight warps take the pairs in
+// turn:
+//  - every warp forms both heads' weights (no barrier), then the group
+//    builds one K-step's operands: X_w split into bf16 hi + mid + lo
+//    (~2^-27 relative) and the B rows (exact in bf16), MN-major in
+//    128-byte-swizzled atoms, zero past T;
 //  - one thread issues the three MMAs into the group's 128-column fp32
 //    accumulator in tensor memory and commits them to the group's mbarrier;
-//  - each thread then owns one accumulator row (warp w reads lanes
-//    32 (w % 4) ..): 16 columns at a time it reads the row with tcgen05.ld,
-//    adds exp(A S_T) h_0 from the stage and runs the format's epilogue -- a
-//    Philox draw per 4 consecutive columns and the stochastic rounding, an
-//    FP4 block of 16 columns quantised in registers -- storing straight to
+//  - each thread then owns one accumulator row, or half of one with eight
+//    warps (warp w reads lanes 32 (w % 4) ..): 16 columns at a time it reads
+//    the row with tcgen05.ld, adds exp(A S_T) h_0 from the stage and runs the
+//    format's epilogue -- a Philox draw per 4 consecutive columns and the
+//    stochastic rounding, an FP4 block of 16 columns quantised in registers
+//    (for e4m3 the block's NaN-propagating max also decides whether any of
+//    its values needs the rounding's special cases) -- storing straight to
 //    global memory.
 // Every wait is bounded; tensor memory is allocated once per CTA and freed
 // on every path.
